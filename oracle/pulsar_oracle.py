@@ -1,0 +1,332 @@
+"""Plain fp64 restatement of the Star / Pulsar attention path (test oracle).
+
+TEST INFRASTRUCTURE ONLY -- never imported by the product path.
+
+Sources (web pages, cited by title and section):
+
+* [P]  "Dropping the Anchor: Statistical Context Summarization for Distributed
+       Systems via Pulsar Attention", project page: §1 (the anchor problem),
+       §2 (method), §2.1 (selecting summaries with Max-IDF), Figure 2 (toy
+       example), §2.2 (query phase), §4 (efficiency), §5 (code / CLI flags).
+* [PS] "Technische Samenvatting: Pulsar Attention" (Dutch technical summary),
+       sections "Fase 1" and "Fase 2".
+* [S]  Star Attention review (machine review of arXiv 2411.17116): summary,
+       key_machinery, and the referee's minor comments on the online-softmax
+       update of Algorithm 2 and on c'_1 = c_1.
+
+Everything is computed in float64 from the inputs exactly as stored (bf16 and
+fp32 inputs are widened to fp64 by the caller).  Library primitives used as
+single steps: ``np.unique`` (set of ids in a block), ``np.matmul`` (dot
+products), ``np.exp`` / ``np.log``.  No blocking, fusion or reordering beyond
+the definitions below; computing a subset of attention rows evaluates each
+requested row by its own definition.
+
+Readings of points the pages leave open (each also listed in the design notes):
+
+* IDF(t) = ln(N / df(t)) with N blocks as documents, no smoothing ([P] §2.1;
+  Figure 2 gives IDF 0 for a token present in every block).
+* Ties in chunk score: lower chunk index first.
+* Budget: k = floor(0.125 * block / chunk) chunks per block ([P] §2.1).
+* Host 0 has no prefix (c'_1 = c_1, [S] minor comment); hosts i >= 1 see
+  [sink || Sigma_0 || ... || Sigma_{i-1} || B_i] ([PS] Fase 1; [P] §2).
+* Summary chunks of block 0 that overlap the sink are not removed.
+* The causal mask is over the concatenated host row index, not position id.
+* Every host row produces an output (a layer's output for all of its rows).
+* RoPE: rotate-half convention, omega_m = theta^(-2m/d), no frequency scaling.
+* Phase-2 query attends to every retained key (no mask); shard h covers keys
+  [h*ceil(T/S), min((h+1)*ceil(T/S), T)); an empty shard has lse = -inf and
+  weight 0; if every shard is empty, O = 0 and lse = -inf.
+
+Parity pins (tests/test_oracle_*.py): brute-force top-k and a Figure-2
+analogue (selection); N = 1 reduces to library causal attention, full-budget
+/ zero-sink hosts equal dense causal attention rows, the uniform-score closed
+form lse = ln(r+1), and complex-multiplication RoPE (Phase 1); the shard merge
+equals library dense attention over the concatenated cache (Phase 2).
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+# ----------------------------------------------------------------------------
+# Max-IDF summary selection  ([P] §2.1; [PS] Fase 1, "Heuristiek" / "Selectie")
+# ----------------------------------------------------------------------------
+
+
+def _blocks(ids: np.ndarray, block: int) -> list[np.ndarray]:
+    """Contiguous blocks of ``block`` tokens ([P] §1: the context is split into
+    contiguous blocks, one per host)."""
+    ids = np.asarray(ids)
+    if ids.size % block:
+        raise ValueError("sequence length must be a multiple of the block size")
+    return [ids[j * block:(j + 1) * block] for j in range(ids.size // block)]
+
+
+def document_frequency(ids: np.ndarray, block: int, vocab: int) -> np.ndarray:
+    """df(t) = number of blocks that contain token t, blocks being the documents
+    ([P] §2.1).  Returns int64 [vocab]."""
+    df = np.zeros(vocab, dtype=np.int64)
+    for blk in _blocks(ids, block):
+        present = np.unique(blk)            # the set of ids in this document
+        df[present] += 1
+    return df
+
+
+def idf_table(df: np.ndarray, n_blocks: int) -> np.ndarray:
+    """IDF(t) = ln(N / df(t)) for every token present in the sequence; NaN for
+    tokens that never occur (they are never looked up)."""
+    out = np.full(df.shape, np.nan, dtype=np.float64)
+    m = df > 0
+    out[m] = np.log(float(n_blocks) / df[m].astype(np.float64))
+    return out
+
+
+def chunk_scores(ids: np.ndarray, block: int, chunk: int, idf: np.ndarray) -> np.ndarray:
+    """Score of every non-overlapping ``chunk``-token chunk of every block: the
+    maximum IDF over its tokens ("scored by its rarest token", [P] §2.1).
+    Returns float64 [N][block // chunk]."""
+    if block % chunk:
+        raise ValueError("block must be a multiple of the chunk size")
+    blocks = _blocks(ids, block)
+    C = block // chunk
+    out = np.empty((len(blocks), C), dtype=np.float64)
+    for j, blk in enumerate(blocks):
+        for c in range(C):
+            out[j, c] = max(idf[t] for t in blk[c * chunk:(c + 1) * chunk].tolist())
+    return out
+
+
+def chunk_min_df(ids: np.ndarray, block: int, chunk: int, df: np.ndarray) -> np.ndarray:
+    """Smallest df over the tokens of each chunk, int64 [N * (block // chunk)]
+    in sequence order (the integer twin of ``chunk_scores``: ln(N/df) is
+    strictly decreasing in df, so the chunk's max IDF is the IDF of its min df)."""
+    blocks = _blocks(ids, block)
+    C = block // chunk
+    out = np.empty(len(blocks) * C, dtype=np.int64)
+    for j, blk in enumerate(blocks):
+        for c in range(C):
+            out[j * C + c] = min(int(df[t]) for t in blk[c * chunk:(c + 1) * chunk].tolist())
+    return out
+
+
+def select_summaries(ids: np.ndarray, block: int, chunk: int, k: int, vocab: int,
+                     return_scores: bool = False):
+    """Top-k chunks per block by Max-IDF score, kept in original order
+    ([P] §2.1: "the top-k chunks, kept in their original order, form the
+    summary").  Equal scores: the lower chunk index wins.
+
+    Returns int64 [N][k] local chunk indices, ascending within each block
+    (and the [N][C] score table when ``return_scores``)."""
+    n_blocks = len(ids) // block
+    C = block // chunk
+    if not 0 <= k <= C:
+        raise ValueError("k must be in [0, block/chunk]")
+    df = document_frequency(ids, block, vocab)
+    idf = idf_table(df, n_blocks)
+    scores = chunk_scores(ids, block, chunk, idf)
+    sel = np.empty((n_blocks, k), dtype=np.int64)
+    for j in range(n_blocks):
+        order = sorted(range(C), key=lambda c: (-scores[j, c], c))
+        sel[j] = sorted(order[:k])
+    return (sel, scores) if return_scores else sel
+
+
+# ----------------------------------------------------------------------------
+# Phase 1: host inputs  ([PS] Fase 1; [P] §2, Figure 1; [S] key_machinery)
+# ----------------------------------------------------------------------------
+
+
+def host_positions(L: int, block: int, sink: int, chunk: int, sel, star: bool = False):
+    """Original position ids of every row of every host's Phase-1 input.
+
+    Pulsar ([PS] Fase 1): host i >= 1 encodes [S_sink || Sigma_0 || ... ||
+    Sigma_{i-1} || B_i]; S_sink is the first ``sink`` tokens of the sequence,
+    Sigma_j the selected chunks of block j in original order.
+    Star ([S] key_machinery): host i >= 1 encodes [B_0 || B_i].
+    Host 0 encodes B_0 alone in both (c'_1 = c_1, [S] minor comment)."""
+    n = L // block
+    hosts = [np.arange(0, block, dtype=np.int64)]
+    for i in range(1, n):
+        parts = []
+        if star:
+            parts.append(np.arange(0, block, dtype=np.int64))
+        else:
+            parts.append(np.arange(0, sink, dtype=np.int64))
+            for j in range(i):
+                for c in sel[j]:
+                    start = j * block + int(c) * chunk
+                    parts.append(np.arange(start, start + chunk, dtype=np.int64))
+        parts.append(np.arange(i * block, (i + 1) * block, dtype=np.int64))
+        hosts.append(np.concatenate(parts))
+    return hosts
+
+
+def host_row_offsets(positions) -> np.ndarray:
+    """Row offsets of the hosts in the packed output: [N + 1] int64."""
+    off = np.zeros(len(positions) + 1, dtype=np.int64)
+    off[1:] = np.cumsum([len(p) for p in positions])
+    return off
+
+
+def rope(x: np.ndarray, pos: np.ndarray, theta: float) -> np.ndarray:
+    """Rotary embedding, rotate-half convention, at position ids ``pos``
+    ([P] §2.1: hosts encode "with original position IDs").
+
+    x: [n][H][d] float64.  For m < d/2, with omega_m = theta^(-2m/d) and
+    a = p * omega_m:  x'[m] = x[m] cos a - x[m + d/2] sin a,
+                      x'[m + d/2] = x[m + d/2] cos a + x[m] sin a."""
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    half = d // 2
+    m = np.arange(half, dtype=np.float64)
+    omega = theta ** (-2.0 * m / d)
+    ang = np.asarray(pos, dtype=np.float64)[:, None] * omega[None, :]  # [n][d/2]
+    c = np.cos(ang)[:, None, :]
+    s = np.sin(ang)[:, None, :]
+    x1, x2 = x[..., :half], x[..., half:]
+    return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
+
+
+def causal_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, rows=None):
+    """Causal softmax attention over one host's concatenated rows.
+
+    q: [n][Hq][d], k/v: [n][Hkv][d] (already rotated), fp64.  Query head h
+    reads kv head h // (Hq / Hkv).  Row r attends to rows c <= r:
+    s_rc = q_r . k_c / sqrt(d);  o_r = sum_c softmax(s_r)_c v_c;
+    lse_r = ln sum_{c <= r} exp(s_rc).
+    Returns (o [len(rows)][Hq][d], lse [len(rows)][Hq])."""
+    n, hq, d = q.shape
+    hkv = k.shape[1]
+    if hq % hkv:
+        raise ValueError("Hq must be a multiple of Hkv")
+    g = hq // hkv
+    rows = np.arange(n) if rows is None else np.asarray(rows, dtype=np.int64)
+    o = np.zeros((rows.size, hq, d), dtype=np.float64)
+    lse = np.zeros((rows.size, hq), dtype=np.float64)
+    if rows.size == 0:
+        return o, lse
+    ncols = int(rows.max()) + 1
+    scale = 1.0 / math.sqrt(d)
+    mask = np.arange(ncols)[None, :] > rows[:, None]          # True where c > r
+    for h in range(hq):
+        kh = k[:ncols, h // g, :]
+        vh = v[:ncols, h // g, :]
+        s = (q[rows, h, :] @ kh.T) * scale
+        s[mask] = -np.inf
+        mx = s.max(axis=1, keepdims=True)
+        e = np.exp(s - mx)
+        z = e.sum(axis=1, keepdims=True)
+        o[:, h, :] = (e @ vh) / z
+        lse[:, h] = (mx + np.log(z))[:, 0]
+    return o, lse
+
+
+def phase1_encode(q, k, v, positions, theta: float, rows_per_host=None):
+    """Phase-1 encoding of every host: RoPE at the original positions, then
+    causal attention over the host's rows ([S] summary; [PS] Fase 1).
+
+    q: [L][Hq][d], k/v: [L][Hkv][d] fp64 (unrotated).  ``positions`` from
+    ``host_positions``.  ``rows_per_host``: optional list of row subsets.
+    Returns a list of (o, lse) per host."""
+    out = []
+    for i, pos in enumerate(positions):
+        rows = None if rows_per_host is None else rows_per_host[i]
+        upto = len(pos) if rows is None or len(rows) == 0 else int(np.max(rows)) + 1
+        p = pos[:upto]
+        qh = rope(q[p], p, theta)
+        kh = rope(k[p], p, theta)
+        vh = np.asarray(v[p], dtype=np.float64)
+        out.append(causal_attention(qh, kh, vh, rows))
+    return out
+
+
+def retained_kv(k, v, theta: float):
+    """KV kept after Phase 1: only each host's own block B_i survives, so the
+    retained cache over all hosts is the whole sequence's K (rotated at its
+    original positions) and V ([P] §2.1 "discards the sink and summary KV";
+    §2.2 "holds the KV cache of its own block only").  Layout [L][Hkv][d] ==
+    [N][block][Hkv][d]."""
+    L = k.shape[0]
+    return rope(k, np.arange(L), theta), np.asarray(v, dtype=np.float64)
+
+
+def phase1_flops(positions, hq: int, d: int) -> float:
+    """Algorithmic Phase-1 FLOPs: QK^T and PV over the causal pairs (diagonal
+    included), 4 * d * Hq * n(n+1)/2 per host."""
+    return float(sum(4.0 * d * hq * len(p) * (len(p) + 1) / 2.0 for p in positions))
+
+
+# ----------------------------------------------------------------------------
+# Phase 2: split-KV query attention and exact merge
+# ([P] §2.2; [PS] Fase 2; [S] key_machinery and Algorithm 2 minor comment)
+# ----------------------------------------------------------------------------
+
+
+def shard_bounds(T: int, n_shards: int):
+    """[start, end) of each shard: equal contiguous shards of ceil(T/S) keys,
+    the last ones shorter or empty."""
+    step = -(-T // n_shards) if n_shards else 0
+    return [(min(h * step, T), min((h + 1) * step, T)) for h in range(n_shards)]
+
+
+def phase2_partials(q, k_cache, v_cache, n_shards: int):
+    """Local attention of the (already rotated) query over each shard.
+
+    q: [B][Tq][Hq][d]; k_cache, v_cache: [B][T][Hkv][d] (K rotated), fp64.
+    For shard h: A_h = softmax(q K_h^T / sqrt(d)) V_h and s_h = ln sum exp
+    (every key of the shard visible).  Returns A [B][S][Tq][Hq][d] and
+    s [B][S][Tq][Hq]; an empty shard gives A_h = 0, s_h = -inf."""
+    B, Tq, hq, d = q.shape
+    T, hkv = k_cache.shape[1], k_cache.shape[2]
+    g = hq // hkv
+    scale = 1.0 / math.sqrt(d)
+    A = np.zeros((B, n_shards, Tq, hq, d), dtype=np.float64)
+    s = np.full((B, n_shards, Tq, hq), -np.inf, dtype=np.float64)
+    for b in range(B):
+        for h, (lo, hi) in enumerate(shard_bounds(T, n_shards)):
+            if hi <= lo:
+                continue
+            for head in range(hq):
+                kk = k_cache[b, lo:hi, head // g, :]
+                vv = v_cache[b, lo:hi, head // g, :]
+                sc = (q[b, :, head, :] @ kk.T) * scale               # [Tq][n]
+                mx = sc.max(axis=1, keepdims=True)
+                e = np.exp(sc - mx)
+                z = e.sum(axis=1, keepdims=True)
+                A[b, h, :, head, :] = (e @ vv) / z
+                s[b, h, :, head] = (mx + np.log(z))[:, 0]
+    return A, s
+
+
+def lse_merge(A, s):
+    """Exact merge of shard partials ([S] Algorithm 2 as corrected in the
+    referee's minor comment): s_global = ln sum_h exp(s_h);
+    A = sum_h exp(s_h - s_global) * A_h.  Shard axis is axis 1.
+    All shards empty: A = 0, s_global = -inf."""
+    B, S = s.shape[0], s.shape[1]
+    m = np.max(s, axis=1)                                 # [B][Tq][Hq]
+    finite = np.isfinite(m)
+    m_safe = np.where(finite, m, 0.0)
+    w = np.exp(s - m_safe[:, None])                       # exp(-inf) = 0
+    z = w.sum(axis=1)
+    s_global = np.where(finite, m_safe + np.log(np.where(finite, z, 1.0)), -np.inf)
+    coef = np.where(finite[:, None], np.exp(s - np.where(finite, s_global, 0.0)[:, None]), 0.0)
+    out = (coef[..., None] * A).sum(axis=1)
+    return out, s_global
+
+
+def phase2_attend(q, k_cache, v_cache, n_shards: int, q_pos0: int, theta: float):
+    """Phase-2 global query attention: rotate the query at positions
+    q_pos0 + j (if theta > 0), attend to every shard, merge exactly.
+    q: [B][Tq][Hq][d] pre-RoPE; caches [B][T][Hkv][d] with K rotated.
+    Returns (O [B][Tq][Hq][d], lse [B][Tq][Hq], A, s)."""
+    q = np.asarray(q, dtype=np.float64)
+    if theta > 0:
+        B, Tq = q.shape[:2]
+        pos = q_pos0 + np.arange(Tq)
+        q = np.stack([rope(q[b], pos, theta) for b in range(B)])
+    A, s = phase2_partials(q, np.asarray(k_cache, np.float64), np.asarray(v_cache, np.float64),
+                           n_shards)
+    o, lse = lse_merge(A, s)
+    return o, lse, A, s
