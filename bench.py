@@ -1,0 +1,459 @@
+"""Benchmark of the Star / Pulsar two-phase attention hot path on B200.
+
+One step = one pass of the whole path over one 128K-token sequence of the
+Llama-3.1-8B attention shape (32 q / 8 kv heads, d = 128, bf16, RoPE theta
+500000, 8 blocks of 16384, 64-token sink, 32-token chunks, 2048-token
+summaries): Max-IDF selection -> Pulsar Phase-1 encoding of all 8 hosts ->
+Phase-2 attention of a 64-token query over the 8 retained shards with the
+exact LSE merge.  value = context tokens encoded per second (whole job).
+
+Also measured in the same run (reported beside the headline, not as bench
+lines of their own): the Star anchor-variant Phase 1 on the same input, and
+the Phase-2 decode of 16 single-token queries over a 128K bf16 cache in 8
+shards (GB/s against HBM).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (torchrun, one process per GPU) every rank encodes its own
+independent sequence (weak scaling, no data-path collective); the time is the
+max over ranks.  `--impl reference` times the fp64 CPU oracle on a bounded
+sample of the same step (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from long_context_blockwise_max_b200 import workloads  # noqa: E402
+
+METRIC = "Phase-1 encode tokens/s (%bf16 TC peak); Phase-2 query attn GB/s (%HBM) @128K"
+WORKLOAD = workloads.LLAMA_128K
+DECODE = workloads.DECODE_128K
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# --------------------------------------------------------------------------
+# clocks during the timed region
+# --------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in (self.out or "").strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx = max(mx, float(f[1]))
+            except ValueError:
+                continue
+            for n, val in zip(names, f[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------
+# our implementation
+# --------------------------------------------------------------------------
+class Step:
+    """Preallocated buffers and the calls of one hot-path step."""
+
+    def __init__(self, w, dev, seed_offset=0):
+        from long_context_blockwise_max_b200 import pulsar as P
+        self.P, self.w, self.dev = P, w, dev
+        ids = w.token_ids()
+        if seed_offset:
+            ids = np.roll(ids, seed_offset * 4099)
+        self.ids_h = torch.from_numpy(ids).pin_memory() if torch.cuda.is_available() else torch.from_numpy(ids)
+        q, k, v = w.qkv(device=dev)
+        self.q, self.k, self.v = q, k, v
+        self.query = w.query(device=dev)
+        self.ids = self.ids_h.to(dev)
+        n = w.n_blocks
+        summ = w.k_chunks * w.chunk
+        self.row_off = P.pa_phase1_layout(w.L, w.block, w.sink, summ, False)
+        R = self.row_off[-1]
+        self.sel = torch.empty((n, w.k_chunks), dtype=torch.int32, device=dev)
+        self.ws_sel = torch.empty(P.pa_select_workspace_size(w.L, w.vocab, w.block, w.chunk), dtype=torch.uint8,
+                                  device=dev)
+        self.o1 = torch.empty((R, w.hq, w.d), dtype=w.dtype, device=dev)
+        self.lse1 = torch.empty((R, w.hq), dtype=torch.float32, device=dev)
+        self.k_ret = torch.empty_like(k)
+        self.v_ret = torch.empty_like(v)
+        self.ws1 = torch.empty(P.pa_phase1_workspace_size(w.L, w.hq, w.hkv, w.d, 1, w.block, w.sink, summ, False),
+                               dtype=torch.uint8, device=dev)
+        self.o2 = torch.empty_like(self.query)
+        self.lse2 = torch.empty((1, w.q_tokens, w.hq), dtype=torch.float32, device=dev)
+        self.ws2 = torch.empty(P.pa_phase2_workspace_size(1, w.q_tokens, w.L, n, w.hq, w.hkv, w.d),
+                               dtype=torch.uint8, device=dev)
+        self.attn_events = None
+
+    def run(self):
+        P, w = self.P, self.w
+        P.pulsar_select_summaries(self.ids, w.vocab, w.block, w.chunk, w.k_chunks, sel=self.sel, ws=self.ws_sel)
+        if self.attn_events is not None:
+            P.pa_set_profile_events(*self.attn_events)
+        P.pulsar_phase1_encode(self.q, self.k, self.v, w.rope_theta, w.block, w.sink, w.chunk, w.k_chunks,
+                               self.sel, o=self.o1, lse=self.lse1, k_ret=self.k_ret, v_ret=self.v_ret,
+                               ws=self.ws1)
+        if self.attn_events is not None:
+            P.pa_set_profile_events(None, None)
+        P.star_phase2_attend(self.query, self.k_ret[None], self.v_ret[None], w.n_blocks, q_pos0=w.L,
+                             rope_theta=w.rope_theta, o=self.o2, lse=self.lse2, ws=self.ws2)
+
+    # kernels of ours launched by one step (selection 3, Phase 1 3, Phase 2 3)
+    LAUNCHES = 9
+
+
+def host_lengths(w, star):
+    n = w.n_blocks
+    summ = w.k_chunks * w.chunk
+    return [w.block] + [(2 * w.block if star else w.sink + i * summ + w.block) for i in range(1, n)]
+
+
+def attn_flops(w, star=False):
+    """Algorithmic Phase-1 FLOPs: 4 * d * Hq * n(n+1)/2 per host (QK^T and PV
+    over the causal pairs, diagonal included; softmax not counted)."""
+    return float(sum(4.0 * w.d * w.hq * n * (n + 1) / 2.0 for n in host_lengths(w, star)))
+
+
+def sync_all(dist_on):
+    torch.cuda.synchronize()
+    if dist_on:
+        torch.distributed.barrier()
+        torch.cuda.synchronize()
+
+
+def max_over_ranks(x: float, dist_on: bool) -> float:
+    if not dist_on:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_ours(args, rank, world, local_rank, dist_on):
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = WORKLOAD
+    peaks, peak_kind = load_peaks()
+    step = Step(w, dev, seed_offset=rank)
+    for _ in range(args.warmup):
+        step.run()
+    st = step.P.pa_workspace_status(step.ws1)
+    if st != 0:
+        raise RuntimeError(f"Phase-1 device status {st}")
+
+    # ---- timed region: K steps -----------------------------------------
+    K = args.steps
+    ev_attn = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for a, b in ev_attn:      # torch creates the CUDA event on its first record
+        a.record()
+        b.record()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sync_all(dist_on)
+    with ClockSampler(local_rank) as clk:
+        t0.record()
+        for i in range(K):
+            step.attn_events = ev_attn[i]
+            step.run()
+        t1.record()
+        torch.cuda.synchronize()
+    step.attn_events = None
+    sync_all(dist_on)
+    ms = max_over_ranks(t0.elapsed_time(t1), dist_on) / K
+    attn_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_attn)
+
+    flops = attn_flops(w)
+    tokens_per_s = w.L * world / (ms * 1e-3)
+    peak_tf = peaks["bf16_tflops_sustained"]
+    attn_tf = flops / (attn_ms * 1e-3) / 1e12
+
+    # ---- end to end through the public API with host buffers ------------
+    q_h = step.q.cpu().pin_memory()
+    k_h = step.k.cpu().pin_memory()
+    v_h = step.v.cpu().pin_memory()
+    query_h = step.query.cpu().pin_memory()
+    o2_h = torch.empty(step.o2.shape, dtype=step.o2.dtype).pin_memory()
+    lse2_h = torch.empty(step.lse2.shape, dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (step.ids_h, q_h, k_h, v_h, query_h))
+    d2h = o2_h.numel() * o2_h.element_size() + lse2_h.numel() * 4
+
+    def e2e_step():
+        step.ids.copy_(step.ids_h, non_blocking=True)
+        step.q.copy_(q_h, non_blocking=True)
+        step.k.copy_(k_h, non_blocking=True)
+        step.v.copy_(v_h, non_blocking=True)
+        step.query.copy_(query_h, non_blocking=True)
+        step.run()
+        o2_h.copy_(step.o2, non_blocking=True)
+        lse2_h.copy_(step.lse2, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    sync_all(dist_on)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(K):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    sync_all(dist_on)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist_on) / K
+
+    # ---- side measurements: Star Phase 1, Phase-2 decode ----------------
+    P = step.P
+    extra = {}
+    if not args.headline_only:
+        row_star = P.pa_phase1_layout(w.L, w.block, 0, 0, True)[-1]
+        o_star = torch.empty((row_star, w.hq, w.d), dtype=w.dtype, device=dev)
+        ws_star = torch.empty(P.pa_phase1_workspace_size(w.L, w.hq, w.hkv, w.d, 1, w.block, 0, 0, True),
+                              dtype=torch.uint8, device=dev)
+        del step.o1, step.lse1
+        torch.cuda.empty_cache()
+
+        def star():
+            P.star_phase1_encode(step.q, step.k, step.v, w.rope_theta, w.block, o=o_star, lse=None,
+                                 k_ret=step.k_ret, v_ret=step.v_ret, ws=ws_star, want_lse=False)
+        star()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = max(1, min(K, 3))
+        torch.cuda.synchronize()
+        s0.record()
+        for _ in range(reps):
+            star()
+        s1.record()
+        torch.cuda.synchronize()
+        star_ms = s0.elapsed_time(s1) / reps
+        sf = attn_flops(w, star=True)
+        extra["star_phase1"] = {"ms": round(star_ms, 3), "tflop": round(sf / 1e12, 3),
+                                "tflop_s": round(sf / (star_ms * 1e-3) / 1e12, 1),
+                                "flop_ratio_star_over_pulsar": round(sf / flops, 3)}
+        del o_star, ws_star
+        torch.cuda.empty_cache()
+
+        dq, dk, dv = DECODE.decode_inputs(device=dev)
+        B, T, S = DECODE.decode_batch, DECODE.decode_T, DECODE.decode_shards
+        do = torch.empty_like(dq)
+        dl = torch.empty((B, 1, DECODE.hq), dtype=torch.float32, device=dev)
+        dws = torch.empty(P.pa_phase2_workspace_size(B, 1, T, S, DECODE.hq, DECODE.hkv, DECODE.d),
+                          dtype=torch.uint8, device=dev)
+        pev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        for a, b in pev:
+            a.record()
+            b.record()
+
+        def dec():
+            P.star_phase2_attend(dq, dk, dv, S, q_pos0=T, rope_theta=DECODE.rope_theta, o=do, lse=dl, ws=dws)
+        for _ in range(3):
+            dec()
+        torch.cuda.synchronize()
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        d0.record()
+        for i in range(K):
+            P.pa_set_profile_events(*pev[i])
+            dec()
+        P.pa_set_profile_events(None, None)
+        d1.record()
+        torch.cuda.synchronize()
+        dec_ms = d0.elapsed_time(d1) / K
+        dec_kernel_ms = statistics.mean(a.elapsed_time(b) for a, b in pev)
+        kv_bytes = 2.0 * B * T * DECODE.hkv * DECODE.d * 2
+        extra["phase2_decode"] = {
+            "workload": DECODE.name, "ms": round(dec_ms, 4), "kernel_ms": round(dec_kernel_ms, 4),
+            "gb_s": round(kv_bytes / (dec_ms * 1e-3) / 1e9, 1),
+            "kernel_gb_s": round(kv_bytes / (dec_kernel_ms * 1e-3) / 1e9, 1),
+            "frac_hbm": round(kv_bytes / (dec_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+            "bytes_per_call": kv_bytes}
+        del dq, dk, dv
+        torch.cuda.empty_cache()
+
+    q2_bytes = 2.0 * w.L * w.hkv * w.d * 2
+    clocks = clk.summary()
+    line = {
+        "metric": METRIC, "value": round(tokens_per_s, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "L": w.L, "block": w.block, "n_blocks": w.n_blocks, "hq": w.hq,
+                   "hkv": w.hkv, "d": w.d, "sink": w.sink, "chunk": w.chunk,
+                   "summary_tokens": w.k_chunks * w.chunk, "q_tokens": w.q_tokens,
+                   "rope_theta": w.rope_theta, "per_rank": "one independent 128K sequence",
+                   "l2": "inputs larger than L2 (Q alone is 1 GiB)"},
+        "clocks": clocks,
+        "e2e": {"value": round(w.L * world / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3)},
+        "gpu_launches": Step.LAUNCHES * K,
+        "roofline": {"bound": "tensor", "kernel": "phase-1 attention", "achieved": round(attn_tf, 1),
+                     "peak": peak_tf, "unit": "TFLOP/s", "frac": round(attn_tf / peak_tf, 4),
+                     "peak_kind": f"{peak_kind} bf16 sustained", "traffic": None,
+                     "kernel_ms": round(attn_ms, 3), "flop_per_launch": flops},
+        "phase1": {"attn_ms": round(attn_ms, 3), "tflop": round(flops / 1e12, 3),
+                   "tflop_s": round(attn_tf, 1)},
+        "phase2_query": {"kv_bytes": q2_bytes},
+    }
+    line.update(extra)
+    return line
+
+
+# --------------------------------------------------------------------------
+# the oracle on the host cores (cpu_baseline leg and --impl reference)
+# --------------------------------------------------------------------------
+def oracle_sample(w, target_s=12.0, seed=0):
+    """Time the fp64 oracle on a bounded sample of one step and extrapolate.
+    Returns (estimated step seconds, sample description, threads)."""
+    import oracle
+    from threadpoolctl import threadpool_info
+
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    ids = w.token_ids()
+    t = time.perf_counter()
+    sel = oracle.select_summaries(ids, w.block, w.chunk, w.k_chunks, w.vocab)
+    t_sel = time.perf_counter() - t
+    pos = oracle.host_positions(w.L, w.block, w.sink, w.chunk, sel)
+    last = len(pos) - 1
+    n = len(pos[last])
+    q, k, v = w.qkv()
+    qf = q.to(torch.float64).numpy()
+    kf = k.to(torch.float64).numpy()
+    vf = v.to(torch.float64).numpy()
+    rng = np.random.default_rng(seed)
+    nrows = 4
+    t_p1 = 0.0
+    sample_flops = 0.0
+    while True:
+        rows = np.sort(rng.choice(n, size=nrows, replace=False))
+        t = time.perf_counter()
+        oracle.phase1_encode(qf, kf, vf, [pos[last]], w.rope_theta, [rows])
+        dt = time.perf_counter() - t
+        t_p1 += dt
+        sample_flops += float(sum(4.0 * w.d * w.hq * (r + 1) for r in rows))
+        if t_p1 >= target_s * 0.7 or nrows >= 256:
+            break
+        nrows *= 2
+    total_flops = attn_flops(w)
+    t_p1_est = t_p1 * total_flops / sample_flops
+    kc, vc = oracle.retained_kv(kf[:, :1], vf[:, :1], w.rope_theta)   # one kv head
+    g = w.hq // w.hkv
+    qq = w.query().to(torch.float64).numpy()[:, :, :g]
+    t = time.perf_counter()
+    oracle.phase2_attend(qq, kc[None], vc[None], w.n_blocks, w.L, w.rope_theta)
+    t_p2 = time.perf_counter() - t
+    t_p2_est = t_p2 * w.hkv
+    est = t_sel + t_p1_est + t_p2_est
+    desc = (f"full selection ({t_sel:.2f} s); Phase-1 rows of the last host ({int(sample_flops / 1e9)} GFLOP "
+            f"of {total_flops / 1e12:.1f} TFLOP, {t_p1:.1f} s, extrapolated by FLOPs); Phase-2 one kv group "
+            f"of {w.hkv} ({t_p2:.1f} s, x{w.hkv})")
+    return est, desc, threads
+
+
+def run_reference(args):
+    w = WORKLOAD
+    ests, desc, threads = [], "", 1
+    for i in range(args.warmup):
+        oracle_sample(w, target_s=2.0, seed=100 + i)
+    for i in range(args.steps):
+        est, desc, threads = oracle_sample(w, target_s=8.0, seed=i)
+        ests.append(est)
+    est = statistics.mean(ests)
+    value = w.L / est
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(est * 1e3, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": w.name, "L": w.L, "block": w.block},
+            "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--headline-only", action="store_true", help="skip the side measurements")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    dist_on = world > 1
+    if dist_on:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, rank, world, local_rank, dist_on)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            est, desc, threads = oracle_sample(WORKLOAD)
+            line["cpu_baseline"] = {"value": round(WORKLOAD.L / est, 3), "unit": "tokens/s", "cores": threads,
+                                    "kind": "oracle", "sample": desc}
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if dist_on:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,229 @@
+/*
+ * pulsar.h -- C ABI of the B200 (sm_100a) Star / Pulsar two-phase blockwise
+ * attention path.
+ *
+ * Sources (web pages, cited by title and section):
+ *  [P]  "Dropping the Anchor: Statistical Context Summarization for
+ *       Distributed Systems via Pulsar Attention" (project page): §1 the
+ *       anchor problem, §2 method, §2.1 Max-IDF selection, Figure 2,
+ *       §2.2 query phase, §4 efficiency, §5 code and CLI flags.
+ *  [PS] "Technische Samenvatting: Pulsar Attention", sections "Fase 1"
+ *       (host input [S_sink || Sigma_0 .. Sigma_{i-1} || B_i], KV discard)
+ *       and "Fase 2" (broadcast query, online-softmax merge).
+ *  [S]  Star Attention machine review (arXiv 2411.17116): summary,
+ *       key_machinery (anchor block with original positions, distributed
+ *       log-sum-exp aggregation), referee minor comments (Algorithm 2 uses
+ *       exp(s_h - s_global) * A_h; the first block has no anchor).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every pointer argument is a DEVICE pointer owned by the caller, unless
+ *    the argument is documented as a host pointer.  The library allocates
+ *    nothing and keeps no state between calls.
+ *  - Scratch memory is the caller's `ws` buffer of at least the size the
+ *    matching *_workspace_size() returns, 256-byte aligned.  Its first 256
+ *    bytes hold a status block that each call clears at its start and that
+ *    kernels set when they detect an error on the device (see
+ *    pa_workspace_status).  A workspace must not be shared by calls that may
+ *    run concurrently.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call
+ *    is stream-ordered and asynchronous: it validates its arguments on the
+ *    host, enqueues kernels and returns; nothing synchronises the device
+ *    except pa_workspace_status.
+ *  - Tensors are dense, row-major, with the innermost dimension listed last,
+ *    e.g. [L][H][d] means element (t, h, m) is at ((t * H) + h) * d + m.
+ *  - dtype is PA_F32 (float) or PA_BF16 (bfloat16, stored as uint16).
+ *  - Return value: PA_OK or a negative pa_status.  On a host-side error no
+ *    kernel is launched and no output is written.
+ */
+#ifndef PULSAR_B200_H
+#define PULSAR_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define PA_ABI_VERSION 1
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID = -1,     /* bad argument: NULL pointer, size mismatch, out-of-range id/index */
+  PA_ERR_UNSUPPORTED = -2, /* valid but not implemented: dtype, head_dim, block count, alignment */
+  PA_ERR_WORKSPACE = -3,   /* ws NULL, misaligned, or smaller than *_workspace_size() */
+  PA_ERR_CUDA = -4,        /* a CUDA launch or memset failed */
+  PA_ERR_TIMEOUT = -5,     /* a bounded device-side wait expired (device status only) */
+  PA_ERR_RANGE = -6        /* a value left the range of an internal format (device status only) */
+} pa_status;
+
+typedef enum { PA_F32 = 0, PA_BF16 = 1 } pa_dtype;
+
+/* Version of this ABI (PA_ABI_VERSION of the built library). */
+int pa_abi_version(void);
+
+/* Static text for a pa_status value. */
+const char* pa_status_string(int status);
+
+/*
+ * Waits for `stream`, then returns the device status recorded in `ws` by the
+ * last call that used this workspace: PA_OK, PA_ERR_INVALID (an id out of
+ * [0, vocab) or a chunk index out of range met on the device), PA_ERR_RANGE
+ * (a rotated Q/K value outside the fp16 range used internally for bf16
+ * inputs) or PA_ERR_TIMEOUT.  Returns PA_ERR_CUDA if the copy fails.  This
+ * is the only synchronising call of the library.
+ */
+int pa_workspace_status(const void* ws, void* stream);
+
+/*
+ * Measurement hook.  When both arguments are non-NULL cudaEvent_t handles
+ * (created by the caller), every later Phase-1 or Phase-2 call made from
+ * this host thread records `start` on its stream right before its dominant
+ * kernel (the attention kernel of Phase 1, the split-KV partial kernel of
+ * Phase 2) and `stop` right after it.  (NULL, NULL) turns recording off.
+ * Returns PA_ERR_INVALID if exactly one argument is NULL.
+ */
+int pa_set_profile_events(void* start, void* stop);
+
+/* ------------------------------------------------------------------------ */
+/* (a1-a3) Max-IDF summary selection        [P] §2.1, Figure 2; [PS] Fase 1 */
+/* ------------------------------------------------------------------------ */
+
+/* Bytes of scratch pulsar_select_summaries needs. 0 if arguments are invalid. */
+size_t pa_select_workspace_size(int64_t L, int32_t vocab, int32_t block, int32_t chunk);
+
+/*
+ * Selects each block's summary: the context of L tokens is cut into
+ * N = L / block contiguous blocks (the documents); df(t) is the number of
+ * blocks containing token t; each block is cut into block / chunk
+ * non-overlapping chunks scored by their rarest token,
+ * max_t ln(N / df(t)) -- computed exactly as the integer min_t df(t), since
+ * ln(N / df) is strictly decreasing in df; the k_chunks best chunks of every
+ * block are kept in original order, equal scores going to the lower chunk
+ * index.
+ *
+ *  ids            [L] int32 token ids, each in [0, vocab).
+ *  L, block       L % block == 0, 1 <= N = L / block <= 64.
+ *  chunk          block % chunk == 0.
+ *  k_chunks       0 <= k_chunks <= block / chunk (the page's budget is
+ *                 floor(0.125 * block / chunk)).
+ *  sel            out [N][k_chunks] int32 local chunk indices, ascending.
+ *  df_opt         out [vocab] int32 document frequency, or NULL.
+ *  chunk_mindf_opt out [L / chunk] int32 min df of every chunk, or NULL.
+ *
+ * Errors: PA_ERR_INVALID for the size rules above or NULL ids/sel (sel may
+ * be NULL only when k_chunks == 0); PA_ERR_UNSUPPORTED for N > 64.  An id
+ * outside [0, vocab) is skipped and sets PA_ERR_INVALID in the workspace
+ * status; the outputs are then unspecified.  Results are bit-exact and
+ * deterministic.
+ */
+int pulsar_select_summaries(const int32_t* ids, int64_t L, int32_t vocab, int32_t block,
+                            int32_t chunk, int32_t k_chunks, int32_t* sel, int32_t* df_opt,
+                            int32_t* chunk_mindf_opt, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* (a4-a5) Phase-1 context encoding   [PS] Fase 1; [P] §2, §2.1; [S] summary */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Host row layout of Phase 1 (HOST pointer row_off, [N + 1] int64).
+ * Host 0 encodes B_0 alone (n_0 = block).  Host i >= 1 encodes
+ *   Pulsar (star == 0): [sink tokens || Sigma_0 || .. || Sigma_{i-1} || B_i],
+ *                       n_i = sink + i * summary_tokens + block;
+ *   Star   (star != 0): [B_0 || B_i], n_i = 2 * block.
+ * row_off[i] is the first packed output row of host i, row_off[N] the total.
+ * Returns PA_ERR_INVALID for L % block != 0, block <= 0, N < 1, sink > block
+ * or summary_tokens > block.
+ */
+int pa_phase1_layout(int64_t L, int32_t block, int32_t sink, int32_t summary_tokens, int star,
+                     int64_t* row_off);
+
+/* Bytes of scratch the Phase-1 calls need (star selects the variant). */
+size_t pa_phase1_workspace_size(int64_t L, int32_t hq, int32_t hkv, int32_t d, int dtype,
+                                int32_t block, int32_t sink, int32_t summary_tokens, int star);
+
+/*
+ * Pulsar Phase-1 encoding of every host of one attention layer, all hosts
+ * batched on this GPU.  Each row carries its ORIGINAL position id p; Q and
+ * K are rotated (RoPE, rotate-half, omega_m = rope_theta^(-2m/d)) at p; host
+ * i runs causal softmax attention over its concatenated rows (row r sees
+ * rows c <= r); query head h reads kv head h / (hq / hkv).
+ *
+ *  q              [L][hq][d]  dtype, unrotated.
+ *  k, v           [L][hkv][d] dtype, unrotated.
+ *  L, block       as in pulsar_select_summaries.
+ *  sink, chunk, k_chunks  sink % 16 == 0, chunk % 16 == 0, sink <= block,
+ *                 k_chunks * chunk <= block.
+ *  sel            [N][k_chunks] int32 device array from
+ *                 pulsar_select_summaries (row N-1 is not read).
+ *  o              out [row_off[N]][hq][d] dtype: every host row's output,
+ *                 hosts packed in order (pa_phase1_layout).
+ *  lse_opt        out [row_off[N]][hq] float: natural-log sum of exp of the
+ *                 row's scaled scores, or NULL.
+ *  k_ret, v_ret   out [N][block][hkv][d] dtype == [L][hkv][d]: the retained
+ *                 cache -- only each host's own block survives, K rotated
+ *                 at its positions, V unchanged ([P] §2.1, §2.2).  v_ret
+ *                 may equal v (then it is not written).
+ *
+ * d must be 64 or 128, hq % hkv == 0.  For PA_BF16, rotated Q and K are
+ * carried in fp16 for the QK^T product (status PA_ERR_RANGE if a rotated
+ * value exceeds 65504); P is rounded to bf16 for the PV product; all sums
+ * are fp32.  For PA_F32 the whole path is fp32.
+ */
+int pulsar_phase1_encode(const void* q, const void* k, const void* v, int dtype, int64_t L,
+                         int32_t hq, int32_t hkv, int32_t d, double rope_theta, int32_t block,
+                         int32_t sink, int32_t chunk, int32_t k_chunks, const int32_t* sel,
+                         void* o, float* lse_opt, void* k_ret, void* v_ret, void* ws,
+                         size_t ws_bytes, void* stream);
+
+/*
+ * Star Attention anchor variant of Phase 1 ([S] key_machinery): host i >= 1
+ * encodes [B_0 || B_i] with B_0 at its original positions, host 0 encodes
+ * B_0 alone.  Arguments and outputs as pulsar_phase1_encode; row layout
+ * pa_phase1_layout(.., star = 1).
+ */
+int star_phase1_encode(const void* q, const void* k, const void* v, int dtype, int64_t L,
+                       int32_t hq, int32_t hkv, int32_t d, double rope_theta, int32_t block,
+                       void* o, float* lse_opt, void* k_ret, void* v_ret, void* ws,
+                       size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* (a6-a7) Phase-2 split-KV attention + exact LSE merge                     */
+/*         [P] §2.2; [PS] Fase 2; [S] key_machinery, Algorithm 2 comment     */
+/* ------------------------------------------------------------------------ */
+
+/* Bytes of scratch star_phase2_attend needs. */
+size_t pa_phase2_workspace_size(int32_t B, int32_t Tq, int64_t T, int32_t n_shards, int32_t hq,
+                                int32_t hkv, int32_t d);
+
+/*
+ * Global query attention over a retained cache split into n_shards shards
+ * (shard h = keys [h * ceil(T / n_shards), min((h + 1) * ceil(T / n_shards), T))).
+ * Each shard yields a partial (A_h, s_h) = (softmax(q K_h^T / sqrt(d)) V_h,
+ * ln sum exp(q K_h^T / sqrt(d))); the exact merge is
+ * s = ln sum_h exp(s_h), O = sum_h exp(s_h - s) A_h.  Every key is visible.
+ *
+ *  q              [B][Tq][hq][d] dtype, unrotated; row j is rotated at
+ *                 position q_pos0 + j when rope_theta > 0, used as given
+ *                 otherwise.
+ *  k_ret, v_ret   [B][T][hkv][d] dtype: batch element b has its own cache
+ *                 (K already rotated, as written by Phase 1).
+ *  o              out [B][Tq][hq][d] dtype.
+ *  lse            out [B][Tq][hq] float.
+ *  part_o_opt     out [B][n_shards][Tq][hq][d] float (A_h) or NULL.
+ *  part_lse_opt   out [B][n_shards][Tq][hq] float (s_h) or NULL.
+ *
+ * An empty shard has s_h = -inf and A_h = 0; with T == 0, O = 0 and
+ * lse = -inf.  d must be 64 or 128, hq % hkv == 0, 1 <= n_shards <= 4096.
+ */
+int star_phase2_attend(const void* q, int dtype, int32_t B, int32_t Tq, int64_t q_pos0,
+                       double rope_theta, const void* k_ret, const void* v_ret, int64_t T,
+                       int32_t n_shards, int32_t hq, int32_t hkv, int32_t d, void* o, float* lse,
+                       float* part_o_opt, float* part_lse_opt, void* ws, size_t ws_bytes,
+                       void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PULSAR_B200_H */

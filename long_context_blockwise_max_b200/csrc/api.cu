@@ -1,0 +1,282 @@
+// C ABI of the library (declared in include/pulsar.h): host-side argument
+// validation, workspace carving and kernel launches.  No exception crosses
+// this boundary, nothing here allocates device memory, and the only
+// synchronising call is pa_workspace_status.
+#include <cmath>
+#include <cstring>
+
+#include "pa_internal.h"
+
+using namespace pa;
+
+namespace pa {
+ProfileEvents& profile_events() {
+  static thread_local ProfileEvents ev;
+  return ev;
+}
+}  // namespace pa
+
+namespace {
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_ws(void* ws, size_t ws_bytes, size_t need) {
+  if (ws == nullptr || !aligned(ws, kAlign) || ws_bytes < need) return PA_ERR_WORKSPACE;
+  return PA_OK;
+}
+
+int clear_status(void* ws, cudaStream_t s) {
+  return cudaMemsetAsync(ws, 0, kStatusBytes, s) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+// Row layout of Phase 1 (see pa_phase1_layout).  Returns PA_OK or an error.
+int layout(int64_t L, int32_t block, int32_t sink, int32_t summary_tokens, int star,
+           int64_t* row_off, int* n_out) {
+  if (block <= 0 || L <= 0 || L % block != 0) return PA_ERR_INVALID;
+  const int64_t n = L / block;
+  if (sink < 0 || sink > block || summary_tokens < 0 || summary_tokens > block)
+    return PA_ERR_INVALID;
+  if (n > kMaxBlocks) return PA_ERR_UNSUPPORTED;
+  row_off[0] = 0;
+  for (int64_t i = 0; i < n; ++i) {
+    int64_t ni;
+    if (i == 0) ni = block;
+    else if (star) ni = 2 * (int64_t)block;
+    else ni = sink + i * (int64_t)summary_tokens + block;
+    row_off[i + 1] = row_off[i] + ni;
+  }
+  *n_out = (int)n;
+  return PA_OK;
+}
+
+int check_heads(int32_t hq, int32_t hkv, int32_t d, int dtype) {
+  if (hq <= 0 || hkv <= 0 || hq % hkv != 0) return PA_ERR_INVALID;
+  if (d != 64 && d != 128) return PA_ERR_UNSUPPORTED;
+  if (dtype != PA_F32 && dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+  return PA_OK;
+}
+
+int phase1_common(const void* q, const void* k, const void* v, int dtype, int64_t L, int32_t hq,
+                  int32_t hkv, int32_t d, double rope_theta, int32_t block, int32_t sink,
+                  int32_t chunk, int32_t k_chunks, const int32_t* sel, int star, void* o,
+                  float* lse_opt, void* k_ret, void* v_ret, void* ws, size_t ws_bytes,
+                  cudaStream_t s) {
+  int rc = check_heads(hq, hkv, d, dtype);
+  if (rc) return rc;
+  if (!q || !k || !v || !o || !k_ret || !v_ret) return PA_ERR_INVALID;
+  if (!(rope_theta > 0.0) || !std::isfinite(rope_theta)) return PA_ERR_INVALID;
+  if (!star) {
+    if (chunk <= 0 || block % chunk != 0 || k_chunks < 0 || k_chunks > block / chunk)
+      return PA_ERR_INVALID;
+    if ((int64_t)k_chunks * chunk > block) return PA_ERR_INVALID;
+    if (sink % 16 != 0 || chunk % 16 != 0) return PA_ERR_UNSUPPORTED;
+    if (k_chunks > 0 && L / block > 1 && sel == nullptr) return PA_ERR_INVALID;
+  }
+  if (block % 16 != 0) return PA_ERR_UNSUPPORTED;
+  if (L > INT32_MAX) return PA_ERR_UNSUPPORTED;
+  const void* ptrs[] = {q, k, v, o, k_ret, v_ret};
+  for (const void* p : ptrs)
+    if (!aligned(p, 16)) return PA_ERR_UNSUPPORTED;
+  HostTable ht;
+  std::memset(&ht, 0, sizeof(ht));
+  int n = 0;
+  rc = layout(L, block, star ? 0 : sink, star ? 0 : k_chunks * chunk, star, ht.row_off, &n);
+  if (rc) return rc;
+  ht.n_hosts = n;
+  ht.star = star;
+  ht.block = block;
+  ht.sink = star ? 0 : sink;
+  ht.chunk = star ? 0 : chunk;
+  ht.k_chunks = star ? 0 : k_chunks;
+  ht.tile_off[0] = 0;
+  for (int i = 0; i < n; ++i) {
+    const int64_t ni = ht.row_off[i + 1] - ht.row_off[i];
+    ht.tile_off[i + 1] = ht.tile_off[i] + (int32_t)((ni + 127) / 128);
+  }
+  const int64_t R = ht.row_off[n];
+  const size_t need = phase1_workspace_bytes(L, hq, hkv, d, dtype, R);
+  rc = check_ws(ws, ws_bytes, need);
+  if (rc) return rc;
+  rc = clear_status(ws, s);
+  if (rc) return rc;
+  Phase1Args a;
+  a.dtype = dtype;
+  a.q = q; a.k = k; a.v = v;
+  a.L = L; a.hq = hq; a.hkv = hkv; a.d = d;
+  a.rope_theta = rope_theta;
+  a.sel = sel;
+  a.ht = ht;
+  a.o = o; a.lse = lse_opt; a.k_ret = k_ret; a.v_ret = v_ret;
+  char* w = static_cast<char*>(ws);
+  a.status = reinterpret_cast<DeviceStatus*>(w);
+  size_t off = kStatusBytes;
+  a.rowpos = reinterpret_cast<int32_t*>(w + off);
+  off += align_up(sizeof(int32_t) * (size_t)R);
+  const size_t qk_elem = dtype == PA_BF16 ? 2 : 4;
+  a.qr = w + off;
+  off += align_up(qk_elem * (size_t)L * hq * d);
+  a.kr = nullptr;
+  if (dtype == PA_BF16) a.kr = w + off;
+  return launch_phase1(a, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+int pa_abi_version(void) { return PA_ABI_VERSION; }
+
+int pa_set_profile_events(void* start, void* stop) {
+  if ((start == nullptr) != (stop == nullptr)) return PA_ERR_INVALID;
+  profile_events().start = static_cast<cudaEvent_t>(start);
+  profile_events().stop = static_cast<cudaEvent_t>(stop);
+  return PA_OK;
+}
+
+const char* pa_status_string(int status) {
+  switch (status) {
+    case PA_OK: return "ok";
+    case PA_ERR_INVALID: return "invalid argument";
+    case PA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case PA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case PA_ERR_CUDA: return "CUDA launch or copy failed";
+    case PA_ERR_TIMEOUT: return "bounded device wait expired";
+    case PA_ERR_RANGE: return "value outside the internal fp16 range";
+    default: return "unknown status";
+  }
+}
+
+int pa_workspace_status(const void* ws, void* stream) {
+  if (ws == nullptr) return PA_ERR_WORKSPACE;
+  int32_t code = 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&code, ws, sizeof(code), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return PA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return PA_ERR_CUDA;
+  return code;
+}
+
+size_t pa_select_workspace_size(int64_t L, int32_t vocab, int32_t block, int32_t chunk) {
+  if (L < 0 || vocab <= 0 || block <= 0 || chunk <= 0 || block % chunk || L % block) return 0;
+  size_t b = kStatusBytes;
+  b += align_up(sizeof(unsigned long long) * (size_t)vocab);
+  b += align_up(sizeof(int32_t) * (size_t)(L / chunk));
+  return b;
+}
+
+int pulsar_select_summaries(const int32_t* ids, int64_t L, int32_t vocab, int32_t block,
+                            int32_t chunk, int32_t k_chunks, int32_t* sel, int32_t* df_opt,
+                            int32_t* chunk_mindf_opt, void* ws, size_t ws_bytes, void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (L <= 0 || vocab <= 0 || block <= 0 || chunk <= 0) return PA_ERR_INVALID;
+  if (L % block != 0 || block % chunk != 0) return PA_ERR_INVALID;
+  if (k_chunks < 0 || k_chunks > block / chunk) return PA_ERR_INVALID;
+  if (ids == nullptr || (sel == nullptr && k_chunks > 0)) return PA_ERR_INVALID;
+  if (L / block > kMaxBlocks) return PA_ERR_UNSUPPORTED;
+  const size_t need = pa_select_workspace_size(L, vocab, block, chunk);
+  int rc = check_ws(ws, ws_bytes, need);
+  if (rc) return rc;
+  rc = clear_status(ws, s);
+  if (rc) return rc;
+  char* w = static_cast<char*>(ws);
+  SelectArgs a;
+  a.ids = ids; a.L = L; a.vocab = vocab; a.block = block; a.chunk = chunk; a.k = k_chunks;
+  a.sel = sel; a.df_out = df_opt;
+  a.status = reinterpret_cast<DeviceStatus*>(w);
+  size_t off = kStatusBytes;
+  a.mask = reinterpret_cast<unsigned long long*>(w + off);
+  off += align_up(sizeof(unsigned long long) * (size_t)vocab);
+  a.mindf = chunk_mindf_opt ? chunk_mindf_opt : reinterpret_cast<int32_t*>(w + off);
+  return launch_select(a, s);
+}
+
+int pa_phase1_layout(int64_t L, int32_t block, int32_t sink, int32_t summary_tokens, int star,
+                     int64_t* row_off) {
+  if (row_off == nullptr) return PA_ERR_INVALID;
+  int64_t tmp[kMaxBlocks + 1];
+  int n = 0;
+  const int rc = layout(L, block, sink, summary_tokens, star, tmp, &n);
+  if (rc) return rc;
+  std::memcpy(row_off, tmp, sizeof(int64_t) * (size_t)(n + 1));
+  return PA_OK;
+}
+
+size_t pa_phase1_workspace_size(int64_t L, int32_t hq, int32_t hkv, int32_t d, int dtype,
+                                int32_t block, int32_t sink, int32_t summary_tokens, int star) {
+  if (check_heads(hq, hkv, d, dtype)) return 0;
+  int64_t off[kMaxBlocks + 1];
+  int n = 0;
+  if (layout(L, block, star ? 0 : sink, star ? 0 : summary_tokens, star, off, &n)) return 0;
+  return phase1_workspace_bytes(L, hq, hkv, d, dtype, off[n]);
+}
+
+int pulsar_phase1_encode(const void* q, const void* k, const void* v, int dtype, int64_t L,
+                         int32_t hq, int32_t hkv, int32_t d, double rope_theta, int32_t block,
+                         int32_t sink, int32_t chunk, int32_t k_chunks, const int32_t* sel,
+                         void* o, float* lse_opt, void* k_ret, void* v_ret, void* ws,
+                         size_t ws_bytes, void* stream) {
+  return phase1_common(q, k, v, dtype, L, hq, hkv, d, rope_theta, block, sink, chunk, k_chunks,
+                       sel, 0, o, lse_opt, k_ret, v_ret, ws, ws_bytes,
+                       static_cast<cudaStream_t>(stream));
+}
+
+int star_phase1_encode(const void* q, const void* k, const void* v, int dtype, int64_t L,
+                       int32_t hq, int32_t hkv, int32_t d, double rope_theta, int32_t block,
+                       void* o, float* lse_opt, void* k_ret, void* v_ret, void* ws,
+                       size_t ws_bytes, void* stream) {
+  return phase1_common(q, k, v, dtype, L, hq, hkv, d, rope_theta, block, 0, 16, 0, nullptr, 1,
+                       o, lse_opt, k_ret, v_ret, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+size_t pa_phase2_workspace_size(int32_t B, int32_t Tq, int64_t T, int32_t n_shards, int32_t hq,
+                                int32_t hkv, int32_t d) {
+  if (B < 0 || Tq < 0 || T < 0 || n_shards < 1 || n_shards > 4096) return 0;
+  if (check_heads(hq, hkv, d, PA_F32)) return 0;
+  return phase2_workspace_bytes(B, Tq, T, n_shards, hq, hkv, d);
+}
+
+int star_phase2_attend(const void* q, int dtype, int32_t B, int32_t Tq, int64_t q_pos0,
+                       double rope_theta, const void* k_ret, const void* v_ret, int64_t T,
+                       int32_t n_shards, int32_t hq, int32_t hkv, int32_t d, void* o, float* lse,
+                       float* part_o_opt, float* part_lse_opt, void* ws, size_t ws_bytes,
+                       void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int rc = check_heads(hq, hkv, d, dtype);
+  if (rc) return rc;
+  if (B < 0 || Tq < 0 || T < 0 || n_shards < 1 || n_shards > 4096) return PA_ERR_INVALID;
+  if (!std::isfinite(rope_theta)) return PA_ERR_INVALID;
+  if (B > 0 && Tq > 0) {
+    if (!q || !o || !lse) return PA_ERR_INVALID;
+    if (T > 0 && (!k_ret || !v_ret)) return PA_ERR_INVALID;
+  }
+  const void* ptrs[] = {q, k_ret, v_ret, o, part_o_opt};
+  for (const void* p : ptrs)
+    if (p && !aligned(p, 16)) return PA_ERR_UNSUPPORTED;
+  const size_t need = phase2_workspace_bytes(B, Tq, T, n_shards, hq, hkv, d);
+  rc = check_ws(ws, ws_bytes, need);
+  if (rc) return rc;
+  rc = clear_status(ws, s);
+  if (rc) return rc;
+  Phase2Args a;
+  a.dtype = dtype;
+  a.q = q; a.B = B; a.Tq = Tq; a.q_pos0 = q_pos0; a.rope_theta = rope_theta;
+  a.k_ret = k_ret; a.v_ret = v_ret; a.T = T;
+  a.n_shards = n_shards;
+  a.n_split = phase2_split(B, Tq, T, n_shards, hq, hkv);
+  a.hq = hq; a.hkv = hkv; a.d = d;
+  a.o = o; a.lse = lse; a.part_o_opt = part_o_opt; a.part_lse_opt = part_lse_opt;
+  char* w = static_cast<char*>(ws);
+  a.status = reinterpret_cast<DeviceStatus*>(w);
+  const size_t rows = (size_t)B * Tq * hq;
+  const size_t units = (size_t)n_shards * a.n_split;
+  size_t off = kStatusBytes;
+  a.qr = reinterpret_cast<float*>(w + off);
+  off += align_up(sizeof(float) * rows * d);
+  a.unit_o = reinterpret_cast<float*>(w + off);
+  off += align_up(sizeof(float) * rows * units * d);
+  a.unit_lse = reinterpret_cast<float*>(w + off);
+  if (B == 0 || Tq == 0) return PA_OK;
+  return launch_phase2(a, s);
+}
+
+}  // extern "C"

@@ -1,0 +1,95 @@
+// Internal launcher interface between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include "pa_common.cuh"
+
+namespace pa {
+
+constexpr int kMaxBlocks = 64;   // per-token block mask is 64 bits
+constexpr int kMaxHalfDim = 64;  // d <= 128
+
+// Caller-provided events bracketing the dominant kernel (pa_set_profile_events).
+struct ProfileEvents {
+  cudaEvent_t start = nullptr, stop = nullptr;
+};
+ProfileEvents& profile_events();
+inline void profile_begin(cudaStream_t s) {
+  if (profile_events().start) cudaEventRecord(profile_events().start, s);
+}
+inline void profile_end(cudaStream_t s) {
+  if (profile_events().stop) cudaEventRecord(profile_events().stop, s);
+}
+
+struct SelectArgs {
+  const int32_t* ids;
+  int64_t L;
+  int32_t vocab, block, chunk, k;
+  int32_t* sel;
+  int32_t* df_out;              // may be null
+  int32_t* mindf;               // [L / chunk] (caller's or workspace)
+  unsigned long long* mask;     // [vocab] workspace
+  DeviceStatus* status;
+};
+int launch_select(const SelectArgs& a, cudaStream_t s);
+
+// Host-computed RoPE frequencies omega_m = theta^(-2m/d), fp64.
+struct RopeFreqs {
+  double omega[kMaxHalfDim];
+};
+
+// Phase-1 host layout shared by the kernels (small, passed by value).
+struct HostTable {
+  int32_t n_hosts;
+  int32_t star;
+  int32_t block, sink, chunk, k_chunks;
+  int64_t row_off[kMaxBlocks + 1];   // packed output row offsets
+  int32_t tile_off[kMaxBlocks + 1];  // cumulative 128-row tiles per host
+};
+
+struct Phase1Args {
+  int dtype;                    // PA_F32 / PA_BF16
+  const void *q, *k, *v;        // inputs [L][h][d]
+  int64_t L;
+  int32_t hq, hkv, d;
+  double rope_theta;
+  const int32_t* sel;           // [N][k] (Pulsar) or null (Star)
+  HostTable ht;
+  void* o;                      // [R][hq][d]
+  float* lse;                   // [R][hq] or null
+  void *k_ret, *v_ret;          // [L][hkv][d]
+  // workspace carve
+  int32_t* rowpos;              // [R] original position of every packed row
+  void* qr;                     // [L][hq][d] rotated, scaled Q (fp16 or fp32)
+  void* kr;                     // [L][hkv][d] rotated K in QK type (fp16) or == k_ret (fp32)
+  DeviceStatus* status;
+};
+size_t phase1_workspace_bytes(int64_t L, int32_t hq, int32_t hkv, int32_t d, int dtype,
+                              int64_t total_rows);
+int launch_phase1(const Phase1Args& a, cudaStream_t s);
+
+struct Phase2Args {
+  int dtype;
+  const void* q;                // [B][Tq][hq][d]
+  int32_t B, Tq;
+  int64_t q_pos0;
+  double rope_theta;
+  const void *k_ret, *v_ret;    // [B][T][hkv][d]
+  int64_t T;
+  int32_t n_shards, n_split;    // units = n_shards * n_split per batch element
+  int32_t hq, hkv, d;
+  void* o;                      // [B][Tq][hq][d]
+  float* lse;                   // [B][Tq][hq]
+  float* part_o_opt;            // [B][n_shards][Tq][hq][d]
+  float* part_lse_opt;          // [B][n_shards][Tq][hq]
+  float* qr;                    // workspace [B][Tq][hq][d]
+  float* unit_o;                // workspace [B][units][Tq][hq][d]
+  float* unit_lse;              // workspace [B][units][Tq][hq]
+  DeviceStatus* status;
+};
+int32_t phase2_split(int32_t B, int32_t Tq, int64_t T, int32_t n_shards, int32_t hq,
+                     int32_t hkv);
+size_t phase2_workspace_bytes(int32_t B, int32_t Tq, int64_t T, int32_t n_shards, int32_t hq,
+                              int32_t hkv, int32_t d);
+int launch_phase2(const Phase2Args& a, cudaStream_t s);
+
+}  // namespace pa

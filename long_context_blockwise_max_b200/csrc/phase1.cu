@@ -1,0 +1,272 @@
+// Phase-1 context encoding (Pulsar Attention page §2, §2.1; Dutch technical
+// summary "Fase 1"; Star Attention review, key_machinery).
+//
+// Layout idea: every Phase-1 row of every host is a token of the original
+// sequence carrying its original position id, and RoPE depends only on that
+// position.  So Q and K are rotated ONCE per token (rope_qk_kernel) and each
+// host's rows are read through `rowpos` (packed row -> position): the sink,
+// the summary chunks and the block itself are runs of contiguous tokens,
+// nothing is copied per host, and the retained cache (B_i's rotated K and V
+// for every host) is simply the whole sequence's rotated K and V.
+//
+//  rowpos_kernel     : packed row -> original position for every host.
+//  rope_qk_kernel    : Q -> Qr (scaled by log2(e)/sqrt(d)), K -> Kr (QK
+//                      operand type) and k_ret (input dtype).
+//  phase1_simt_kernel: causal attention over a host's rows, fp32 SIMT with an
+//                      online softmax (used for fp32 inputs, and for bf16
+//                      inputs when the tensor-core kernel is not selected).
+#include "pa_internal.h"
+
+namespace pa {
+
+__global__ void rowpos_kernel(HostTable ht, const int32_t* __restrict__ sel,
+                              int32_t* __restrict__ rowpos, DeviceStatus* st) {
+  const int64_t R = ht.row_off[ht.n_hosts];
+  const int64_t summ = (int64_t)ht.k_chunks * ht.chunk;
+  const int C = ht.chunk > 0 ? ht.block / ht.chunk : 0;
+  for (int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r < R;
+       r += (int64_t)gridDim.x * blockDim.x) {
+    int i = 0;
+    while (i + 1 < ht.n_hosts && r >= ht.row_off[i + 1]) ++i;
+    const int64_t u = r - ht.row_off[i];
+    int64_t p;
+    if (i == 0) {
+      p = u;                                         // host 0: B_0 alone
+    } else if (ht.star) {
+      p = (u < ht.block) ? u : (int64_t)i * ht.block + (u - ht.block);  // [B_0 || B_i]
+    } else if (u < ht.sink) {
+      p = u;                                         // attention sink
+    } else if (u < ht.sink + (int64_t)i * summ) {    // Sigma_0 .. Sigma_{i-1}
+      const int64_t w = u - ht.sink;
+      const int64_t j = w / summ, x = w % summ;
+      const int m = (int)(x / ht.chunk), t = (int)(x % ht.chunk);
+      int c = sel[j * ht.k_chunks + m];
+      if (c < 0 || c >= C) {
+        set_status(st, PA_ERR_INVALID, (int)(j * ht.k_chunks + m), c);
+        c = 0;
+      }
+      p = j * ht.block + (int64_t)c * ht.chunk + t;
+    } else {
+      p = (int64_t)i * ht.block + (u - ht.sink - (int64_t)i * summ);   // B_i
+    }
+    rowpos[r] = (int32_t)p;
+  }
+}
+
+template <typename T> __device__ __forceinline__ void check_range(float, DeviceStatus*) {}
+template <> __device__ __forceinline__ void check_range<__half>(float x, DeviceStatus* st) {
+  if (!(fabsf(x) <= 65504.f)) set_status(st, PA_ERR_RANGE, 0, 0);
+}
+
+// RoPE (rotate-half): for m < d/2, a = p * omega_m,
+//   x'[m] = x[m] cos a - x[m + d/2] sin a,  x'[m + d/2] = x[m + d/2] cos a + x[m] sin a.
+// The angle and its sine/cosine are evaluated in fp64, the rotation in fp32.
+template <typename IT, typename QT, int POS>
+__global__ void __launch_bounds__(256) rope_qk_kernel(
+    const IT* __restrict__ q, const IT* __restrict__ k, int64_t L, int hq, int hkv, int d,
+    RopeFreqs f, float qscale, QT* __restrict__ qr, QT* __restrict__ kr, IT* __restrict__ k_ret,
+    DeviceStatus* st) {
+  __shared__ float2 cs[POS][kMaxHalfDim];
+  const int half = d / 2;
+  const int64_t p0 = (int64_t)blockIdx.x * POS;
+  for (int e = threadIdx.x; e < POS * half; e += blockDim.x) {
+    const int pp = e / half, m = e % half;
+    double sn, cn;
+    sincos((double)(p0 + pp) * f.omega[m], &sn, &cn);
+    cs[pp][m] = make_float2((float)cn, (float)sn);
+  }
+  __syncthreads();
+  const int per_pos_q = hq * half, per_pos_k = hkv * half;
+  for (int e = threadIdx.x; e < POS * (per_pos_q + per_pos_k); e += blockDim.x) {
+    const int pp = e / (per_pos_q + per_pos_k);
+    const int64_t p = p0 + pp;
+    if (p >= L) continue;
+    int w = e % (per_pos_q + per_pos_k);
+    const bool is_q = w < per_pos_q;
+    if (!is_q) w -= per_pos_q;
+    const int h = w / half, m = w % half;
+    const int H = is_q ? hq : hkv;
+    const int64_t base = (p * H + h) * (int64_t)d;
+    const IT* src = is_q ? q : k;
+    const float x1 = to_f32(src[base + m]), x2 = to_f32(src[base + m + half]);
+    const float2 c = cs[pp][m];
+    const float y1 = x1 * c.x - x2 * c.y;
+    const float y2 = x2 * c.x + x1 * c.y;
+    if (is_q) {
+      const float a = y1 * qscale, b = y2 * qscale;
+      check_range<QT>(a, st);
+      check_range<QT>(b, st);
+      qr[base + m] = from_f32<QT>(a);
+      qr[base + m + half] = from_f32<QT>(b);
+    } else {
+      k_ret[base + m] = from_f32<IT>(y1);
+      k_ret[base + m + half] = from_f32<IT>(y2);
+      if (kr != nullptr) {
+        check_range<QT>(y1, st);
+        check_range<QT>(y2, st);
+        kr[base + m] = from_f32<QT>(y1);
+        kr[base + m + half] = from_f32<QT>(y2);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// SIMT causal attention.  CTA = 128 rows of one host x one query head; two
+// threads per row, each owning interleaved groups of 4 head-dim elements.
+// Scores are in log2 units (Q carries log2(e)/sqrt(d)).
+// ---------------------------------------------------------------------------
+template <int D, typename QT, typename VT, typename OT>
+__global__ void __launch_bounds__(256) phase1_simt_kernel(
+    const QT* __restrict__ qr, const QT* __restrict__ kr, const VT* __restrict__ v,
+    const int32_t* __restrict__ rowpos, HostTable ht, int hq, int hkv, OT* __restrict__ o,
+    float* __restrict__ lse) {
+  constexpr int BK = 32, HALF = D / 2, G4 = HALF / 4;
+  __shared__ __align__(16) float ks[BK][D];
+  __shared__ __align__(16) float vs[BK][D];
+  const int h = blockIdx.y, kvh = h / (hq / hkv);
+  int host = 0;
+  while (host + 1 < ht.n_hosts && (int)blockIdx.x >= ht.tile_off[host + 1]) ++host;
+  const int64_t row0 = ht.row_off[host];
+  const int n = (int)(ht.row_off[host + 1] - row0);
+  const int tile_r0 = ((int)blockIdx.x - ht.tile_off[host]) * 128;
+  const int r = tile_r0 + (threadIdx.x >> 1);
+  const int hf = threadIdx.x & 1;
+  const bool active = r < n;
+  // element index of group g, lane-half hf: 8*g + 4*hf + {0..3}
+  float qv[HALF], acc[HALF];
+  if (active) {
+    const int64_t pq = rowpos[row0 + r];
+    const QT* src = qr + (pq * hq + h) * (int64_t)D;
+#pragma unroll
+    for (int g = 0; g < G4; ++g)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) qv[4 * g + e] = to_f32(src[8 * g + 4 * hf + e]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < HALF; ++i) qv[i] = 0.f;
+  }
+#pragma unroll
+  for (int i = 0; i < HALF; ++i) acc[i] = 0.f;
+  float m_run = -INFINITY, l_run = 0.f;
+  const int last = min(n, tile_r0 + 128) - 1;
+  for (int c0 = 0; c0 <= last; c0 += BK) {
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < BK * D; idx += 256) {
+      const int kk = idx / D, mm = idx % D, c = c0 + kk;
+      float kx = 0.f, vx = 0.f;
+      if (c < n) {
+        const int64_t pk = rowpos[row0 + c];
+        const int64_t off = (pk * hkv + kvh) * (int64_t)D + mm;
+        kx = to_f32(kr[off]);
+        vx = to_f32(v[off]);
+      }
+      ks[kk][mm] = kx;
+      vs[kk][mm] = vx;
+    }
+    __syncthreads();
+    float s[BK];
+    float mt = m_run;
+#pragma unroll
+    for (int j = 0; j < BK; ++j) {
+      float a = 0.f;
+#pragma unroll
+      for (int g = 0; g < G4; ++g) {
+        const float4 kk4 = *reinterpret_cast<const float4*>(&ks[j][8 * g + 4 * hf]);
+        a = fmaf(qv[4 * g + 0], kk4.x, a);
+        a = fmaf(qv[4 * g + 1], kk4.y, a);
+        a = fmaf(qv[4 * g + 2], kk4.z, a);
+        a = fmaf(qv[4 * g + 3], kk4.w, a);
+      }
+      a += __shfl_xor_sync(0xffffffffu, a, 1);
+      s[j] = (c0 + j <= r) ? a : -INFINITY;
+      mt = fmaxf(mt, s[j]);
+    }
+    if (mt == -INFINITY) continue;   // row sees no key of this tile (uniform per pair)
+    const float alpha = fast_exp2(m_run - mt);   // exp2(-inf) = 0 on the first tile
+    l_run *= alpha;
+#pragma unroll
+    for (int i = 0; i < HALF; ++i) acc[i] *= alpha;
+#pragma unroll
+    for (int j = 0; j < BK; ++j) {
+      const float pj = fast_exp2(s[j] - mt);
+      l_run += pj;
+#pragma unroll
+      for (int g = 0; g < G4; ++g) {
+        const float4 vv4 = *reinterpret_cast<const float4*>(&vs[j][8 * g + 4 * hf]);
+        acc[4 * g + 0] = fmaf(pj, vv4.x, acc[4 * g + 0]);
+        acc[4 * g + 1] = fmaf(pj, vv4.y, acc[4 * g + 1]);
+        acc[4 * g + 2] = fmaf(pj, vv4.z, acc[4 * g + 2]);
+        acc[4 * g + 3] = fmaf(pj, vv4.w, acc[4 * g + 3]);
+      }
+    }
+    m_run = mt;
+  }
+  if (!active) return;
+  const float inv = 1.f / l_run;
+  OT* dst = o + ((row0 + r) * hq + h) * (int64_t)D;
+#pragma unroll
+  for (int g = 0; g < G4; ++g)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) dst[8 * g + 4 * hf + e] = from_f32<OT>(acc[4 * g + e] * inv);
+  if (lse != nullptr && hf == 0) lse[(row0 + r) * hq + h] = (m_run + __log2f(l_run)) * kLn2f;
+}
+
+size_t phase1_workspace_bytes(int64_t L, int32_t hq, int32_t hkv, int32_t d, int dtype,
+                              int64_t total_rows) {
+  const size_t qk_elem = dtype == PA_BF16 ? 2 : 4;
+  size_t b = kStatusBytes;
+  b += align_up(sizeof(int32_t) * (size_t)total_rows);
+  b += align_up(qk_elem * (size_t)L * hq * d);
+  if (dtype == PA_BF16) b += align_up(qk_elem * (size_t)L * hkv * d);
+  return b;
+}
+
+template <typename IT, typename QT, typename VT, typename OT>
+static int launch_phase1_t(const Phase1Args& a, cudaStream_t s) {
+  const int64_t R = a.ht.row_off[a.ht.n_hosts];
+  {
+    const int threads = 256;
+    const int64_t want = (R + threads - 1) / threads;
+    rowpos_kernel<<<(int)(want < 148 * 8 ? want : 148 * 8), threads, 0, s>>>(a.ht, a.sel,
+                                                                             a.rowpos, a.status);
+  }
+  RopeFreqs f;
+  for (int m = 0; m < kMaxHalfDim; ++m)
+    f.omega[m] = (m < a.d / 2) ? pow(a.rope_theta, -2.0 * m / a.d) : 0.0;
+  const float qscale = (float)(kLog2e / sqrt((double)a.d));
+  constexpr int POS = 4;
+  if (a.L > 0) {
+    rope_qk_kernel<IT, QT, POS><<<(unsigned)((a.L + POS - 1) / POS), 256, 0, s>>>(
+        static_cast<const IT*>(a.q), static_cast<const IT*>(a.k), a.L, a.hq, a.hkv, a.d, f,
+        qscale, static_cast<QT*>(a.qr), static_cast<QT*>(a.kr), static_cast<IT*>(a.k_ret),
+        a.status);
+  }
+  if (a.v_ret != a.v && a.L > 0) {
+    if (cudaMemcpyAsync(a.v_ret, a.v, sizeof(IT) * (size_t)a.L * a.hkv * a.d,
+                        cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+      return PA_ERR_CUDA;
+  }
+  const QT* kq = a.kr ? static_cast<const QT*>(a.kr) : static_cast<const QT*>(a.k_ret);
+  const dim3 grid(a.ht.tile_off[a.ht.n_hosts], a.hq);
+  profile_begin(s);
+  if (grid.x > 0) {
+    if (a.d == 128)
+      phase1_simt_kernel<128, QT, VT, OT><<<grid, 256, 0, s>>>(
+          static_cast<const QT*>(a.qr), kq, static_cast<const VT*>(a.v), a.rowpos, a.ht, a.hq,
+          a.hkv, static_cast<OT*>(a.o), a.lse);
+    else
+      phase1_simt_kernel<64, QT, VT, OT><<<grid, 256, 0, s>>>(
+          static_cast<const QT*>(a.qr), kq, static_cast<const VT*>(a.v), a.rowpos, a.ht, a.hq,
+          a.hkv, static_cast<OT*>(a.o), a.lse);
+  }
+  profile_end(s);
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+int launch_phase1(const Phase1Args& a, cudaStream_t s) {
+  if (a.dtype == PA_F32) return launch_phase1_t<float, float, float, float>(a, s);
+  return launch_phase1_t<__nv_bfloat16, __half, __nv_bfloat16, __nv_bfloat16>(a, s);
+}
+
+}  // namespace pa

@@ -1,0 +1,253 @@
+// Phase-2 global query attention: split-KV partial attention per shard and
+// the exact log-sum-exp merge (Pulsar Attention page §2.2; Dutch technical
+// summary "Fase 2"; Star Attention review, key_machinery and the referee's
+// correction of Algorithm 2: O = sum_h exp(s_h - s_global) A_h).
+//
+// Work unit = (batch element, shard, split, kv head, tile of 128 query rows).
+// A shard may be cut into `n_split` contiguous splits so that small batches
+// still fill the GPU; the merge is associative, so splits and shards merge
+// with the same algebra.
+#include "pa_internal.h"
+
+namespace pa {
+
+// q [B][Tq][hq][d] -> qr fp32, rotated at q_pos0 + t (theta > 0) and scaled
+// by log2(e)/sqrt(d) so that scores come out in log2 units.
+template <typename IT>
+__global__ void rope_query_kernel(const IT* __restrict__ q, int B, int Tq, int hq, int d,
+                                  int64_t q_pos0, int use_rope, RopeFreqs f, float qscale,
+                                  float* __restrict__ qr) {
+  const int half = d / 2;
+  const int64_t n = (int64_t)B * Tq * hq * half;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int m = (int)(e % half);
+    const int64_t row = e / half;                 // (b, t, h)
+    const int t = (int)((row / hq) % Tq);
+    const int64_t base = row * d;
+    const float x1 = to_f32(q[base + m]), x2 = to_f32(q[base + m + half]);
+    float y1 = x1, y2 = x2;
+    if (use_rope) {
+      double sn, cn;
+      sincos((double)(q_pos0 + t) * f.omega[m], &sn, &cn);
+      const float c = (float)cn, s = (float)sn;
+      y1 = x1 * c - x2 * s;
+      y2 = x2 * c + x1 * s;
+    }
+    qr[base + m] = y1 * qscale;
+    qr[base + m + half] = y2 * qscale;
+  }
+}
+
+__host__ __device__ inline void unit_range(int64_t T, int n_shards, int n_split, int u,
+                                           int64_t* k0, int64_t* k1) {
+  const int64_t step = (T + n_shards - 1) / n_shards;
+  const int sh = u / n_split, sp = u % n_split;
+  const int64_t lo = min((int64_t)sh * step, T), hi = min((int64_t)(sh + 1) * step, T);
+  const int64_t len = (hi - lo + n_split - 1) / n_split;
+  *k0 = min(lo + (int64_t)sp * len, hi);
+  *k1 = min(lo + (int64_t)(sp + 1) * len, hi);
+}
+
+template <int D, typename VT>
+__global__ void __launch_bounds__(256) phase2_simt_kernel(Phase2Args a) {
+  constexpr int BK = 32, HALF = D / 2, G4 = HALF / 4;
+  __shared__ __align__(16) float ks[BK][D];
+  __shared__ __align__(16) float vs[BK][D];
+  const int units = a.n_shards * a.n_split;
+  const int b = blockIdx.x / units, u = blockIdx.x % units;
+  const int kvh = blockIdx.y, g = a.hq / a.hkv;
+  const int idx = blockIdx.z * 128 + (threadIdx.x >> 1);
+  const int hf = threadIdx.x & 1;
+  const bool active = idx < a.Tq * g;
+  const int t = active ? idx / g : 0, head = kvh * g + (active ? idx % g : 0);
+  int64_t k0, k1;
+  unit_range(a.T, a.n_shards, a.n_split, u, &k0, &k1);
+  const VT* K = static_cast<const VT*>(a.k_ret) + (int64_t)b * a.T * a.hkv * D;
+  const VT* V = static_cast<const VT*>(a.v_ret) + (int64_t)b * a.T * a.hkv * D;
+  float qv[HALF], acc[HALF];
+  {
+    const float* src = a.qr + (((int64_t)b * a.Tq + t) * a.hq + head) * D;
+#pragma unroll
+    for (int gg = 0; gg < G4; ++gg)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) qv[4 * gg + e] = active ? src[8 * gg + 4 * hf + e] : 0.f;
+  }
+#pragma unroll
+  for (int i = 0; i < HALF; ++i) acc[i] = 0.f;
+  float m_run = -INFINITY, l_run = 0.f;
+  for (int64_t c0 = k0; c0 < k1; c0 += BK) {
+    __syncthreads();
+    for (int id = threadIdx.x; id < BK * D; id += 256) {
+      const int kk = id / D, mm = id % D;
+      const int64_t c = c0 + kk;
+      float kx = 0.f, vx = 0.f;
+      if (c < k1) {
+        const int64_t off = (c * a.hkv + kvh) * (int64_t)D + mm;
+        kx = to_f32(K[off]);
+        vx = to_f32(V[off]);
+      }
+      ks[kk][mm] = kx;
+      vs[kk][mm] = vx;
+    }
+    __syncthreads();
+    float s[BK];
+    float mt = m_run;
+#pragma unroll
+    for (int j = 0; j < BK; ++j) {
+      float acc_s = 0.f;
+#pragma unroll
+      for (int gg = 0; gg < G4; ++gg) {
+        const float4 kk4 = *reinterpret_cast<const float4*>(&ks[j][8 * gg + 4 * hf]);
+        acc_s = fmaf(qv[4 * gg + 0], kk4.x, acc_s);
+        acc_s = fmaf(qv[4 * gg + 1], kk4.y, acc_s);
+        acc_s = fmaf(qv[4 * gg + 2], kk4.z, acc_s);
+        acc_s = fmaf(qv[4 * gg + 3], kk4.w, acc_s);
+      }
+      acc_s += __shfl_xor_sync(0xffffffffu, acc_s, 1);
+      s[j] = (c0 + j < k1) ? acc_s : -INFINITY;
+      mt = fmaxf(mt, s[j]);
+    }
+    const float alpha = fast_exp2(m_run - mt);
+    l_run *= alpha;
+#pragma unroll
+    for (int i = 0; i < HALF; ++i) acc[i] *= alpha;
+#pragma unroll
+    for (int j = 0; j < BK; ++j) {
+      const float pj = fast_exp2(s[j] - mt);
+      l_run += pj;
+#pragma unroll
+      for (int gg = 0; gg < G4; ++gg) {
+        const float4 vv4 = *reinterpret_cast<const float4*>(&vs[j][8 * gg + 4 * hf]);
+        acc[4 * gg + 0] = fmaf(pj, vv4.x, acc[4 * gg + 0]);
+        acc[4 * gg + 1] = fmaf(pj, vv4.y, acc[4 * gg + 1]);
+        acc[4 * gg + 2] = fmaf(pj, vv4.z, acc[4 * gg + 2]);
+        acc[4 * gg + 3] = fmaf(pj, vv4.w, acc[4 * gg + 3]);
+      }
+    }
+    m_run = mt;
+  }
+  if (!active) return;
+  const int64_t orow = (((int64_t)b * units + u) * a.Tq + t) * a.hq + head;
+  float* dst = a.unit_o + orow * D;
+  const bool empty = k1 <= k0;
+  const float inv = empty ? 0.f : 1.f / l_run;
+#pragma unroll
+  for (int gg = 0; gg < G4; ++gg)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) dst[8 * gg + 4 * hf + e] = acc[4 * gg + e] * inv;
+  if (hf == 0) a.unit_lse[orow] = empty ? -INFINITY : (m_run + __log2f(l_run)) * kLn2f;
+}
+
+// One warp per (b, t, head): merge splits into shard partials, shards into
+// the global result.  s = ln sum exp(s_h) ; O = sum_h exp(s_h - s) A_h.
+template <typename OT>
+__global__ void merge_kernel(Phase2Args a) {
+  const int lane = threadIdx.x & 31;
+  const int64_t nrows = (int64_t)a.B * a.Tq * a.hq;
+  const int units = a.n_shards * a.n_split;
+  const int per_lane = a.d / 32;   // 2 or 4
+  for (int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < nrows;
+       row += ((int64_t)gridDim.x * blockDim.x) >> 5) {
+    const int64_t b = row / ((int64_t)a.Tq * a.hq), th = row % ((int64_t)a.Tq * a.hq);
+    float gm = -INFINITY, gz = 0.f, gacc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int sh = 0; sh < a.n_shards; ++sh) {
+      float sm = -INFINITY, sz = 0.f, sacc[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int sp = 0; sp < a.n_split; ++sp) {
+        const int u = sh * a.n_split + sp;
+        const int64_t urow = (b * units + u) * (int64_t)a.Tq * a.hq + th;
+        const float s = a.unit_lse[urow];
+        if (s == -INFINITY) continue;
+        const float mn = fmaxf(sm, s);
+        const float c_old = expf(sm - mn), c_new = expf(s - mn);
+        sz = sz * c_old + c_new;
+        const float* A = a.unit_o + urow * a.d;
+        for (int e = 0; e < per_lane; ++e) sacc[e] = sacc[e] * c_old + c_new * A[lane + 32 * e];
+        sm = mn;
+      }
+      const float s_h = (sm == -INFINITY) ? -INFINITY : sm + logf(sz);
+      if (a.part_o_opt != nullptr) {
+        const int64_t prow = (b * a.n_shards + sh) * (int64_t)a.Tq * a.hq + th;
+        const float inv = (sm == -INFINITY) ? 0.f : 1.f / sz;
+        for (int e = 0; e < per_lane; ++e) a.part_o_opt[prow * a.d + lane + 32 * e] = sacc[e] * inv;
+        if (lane == 0 && a.part_lse_opt != nullptr) a.part_lse_opt[prow] = s_h;
+      } else if (a.part_lse_opt != nullptr && lane == 0) {
+        a.part_lse_opt[(b * a.n_shards + sh) * (int64_t)a.Tq * a.hq + th] = s_h;
+      }
+      if (s_h == -INFINITY) continue;
+      // fold the shard's (unnormalised) sums into the global accumulator
+      const float mn = fmaxf(gm, sm);
+      const float c_old = expf(gm - mn), c_new = expf(sm - mn);
+      gz = gz * c_old + sz * c_new;
+      for (int e = 0; e < per_lane; ++e) gacc[e] = gacc[e] * c_old + sacc[e] * c_new;
+      gm = mn;
+    }
+    OT* O = static_cast<OT*>(a.o) + row * a.d;
+    const float inv = (gm == -INFINITY) ? 0.f : 1.f / gz;
+    for (int e = 0; e < per_lane; ++e) O[lane + 32 * e] = from_f32<OT>(gacc[e] * inv);
+    if (lane == 0) a.lse[row] = (gm == -INFINITY) ? -INFINITY : gm + logf(gz);
+  }
+}
+
+int32_t phase2_split(int32_t B, int32_t Tq, int64_t T, int32_t n_shards, int32_t hq,
+                     int32_t hkv) {
+  const int g = hq / hkv;
+  const int64_t row_tiles = ((int64_t)Tq * g + 127) / 128;
+  const int64_t base = (int64_t)B * n_shards * hkv * row_tiles;
+  const int64_t shard_len = (T + n_shards - 1) / n_shards;
+  int64_t want = base > 0 ? (4 * 148 + base - 1) / base : 1;
+  const int64_t cap = shard_len / 512;
+  if (want > cap) want = cap;
+  if (want > 64) want = 64;
+  if (want < 1) want = 1;
+  return (int32_t)want;
+}
+
+size_t phase2_workspace_bytes(int32_t B, int32_t Tq, int64_t T, int32_t n_shards, int32_t hq,
+                              int32_t hkv, int32_t d) {
+  const int32_t ns = phase2_split(B, Tq, T, n_shards, hq, hkv);
+  const size_t units = (size_t)n_shards * ns;
+  const size_t rows = (size_t)B * Tq * hq;
+  size_t b = kStatusBytes;
+  b += align_up(sizeof(float) * rows * d);          // rotated query
+  b += align_up(sizeof(float) * rows * units * d);  // unit partial outputs
+  b += align_up(sizeof(float) * rows * units);      // unit partial lse
+  return b;
+}
+
+template <typename IT>
+static int launch_phase2_t(const Phase2Args& a, cudaStream_t s) {
+  RopeFreqs f;
+  for (int m = 0; m < kMaxHalfDim; ++m)
+    f.omega[m] = (m < a.d / 2 && a.rope_theta > 0) ? pow(a.rope_theta, -2.0 * m / a.d) : 0.0;
+  const float qscale = (float)(kLog2e / sqrt((double)a.d));
+  const int64_t nq = (int64_t)a.B * a.Tq * a.hq * (a.d / 2);
+  if (nq > 0) {
+    const int64_t want = (nq + 255) / 256;
+    rope_query_kernel<IT><<<(int)(want < 148 * 8 ? want : 148 * 8), 256, 0, s>>>(
+        static_cast<const IT*>(a.q), a.B, a.Tq, a.hq, a.d, a.q_pos0, a.rope_theta > 0, f, qscale,
+        a.qr);
+  }
+  const int units = a.n_shards * a.n_split;
+  const int g = a.hq / a.hkv;
+  const dim3 grid((unsigned)(a.B * units), a.hkv, (unsigned)((a.Tq * g + 127) / 128));
+  profile_begin(s);
+  if (grid.x > 0 && grid.z > 0) {
+    if (a.d == 128) phase2_simt_kernel<128, IT><<<grid, 256, 0, s>>>(a);
+    else phase2_simt_kernel<64, IT><<<grid, 256, 0, s>>>(a);
+  }
+  profile_end(s);
+  const int64_t nrows = (int64_t)a.B * a.Tq * a.hq;
+  if (nrows > 0) {
+    const int64_t want = (nrows * 32 + 255) / 256;
+    merge_kernel<IT><<<(int)(want < 148 * 16 ? want : 148 * 16), 256, 0, s>>>(a);
+  }
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+int launch_phase2(const Phase2Args& a, cudaStream_t s) {
+  if (a.dtype == PA_F32) return launch_phase2_t<float>(a, s);
+  return launch_phase2_t<__nv_bfloat16>(a, s);
+}
+
+}  // namespace pa

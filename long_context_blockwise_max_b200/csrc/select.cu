@@ -1,0 +1,170 @@
+// Max-IDF summary selection kernels (Pulsar Attention page, §2.1 and
+// Figure 2; Dutch technical summary, "Fase 1").
+//
+// Integer formulation: the chunk score max_t ln(N / df(t)) is strictly
+// decreasing in df, so ranking chunks by score equals ranking them by their
+// minimum document frequency, with identical ties.  Everything here is
+// integer arithmetic and bit-exact.
+//
+//  presence_mask_kernel : mask[t] |= 1 << j for every token t of block j
+//                         (blocks are the documents); df(t) = popc(mask[t]).
+//  chunk_mindf_kernel   : one warp per chunk, min over its tokens of df.
+//  topk_kernel          : one CTA per block; histogram of min-df values
+//                         (1..N) -> threshold -> ordered compaction that keeps
+//                         the lowest-index chunks among equal scores.
+#include "pa_internal.h"
+
+namespace pa {
+
+__global__ void presence_mask_kernel(const int32_t* __restrict__ ids, int64_t L, int32_t vocab,
+                                     int32_t block, unsigned long long* __restrict__ mask,
+                                     DeviceStatus* st) {
+  const int lane = threadIdx.x & 31;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  // Warp-uniform loop so that every lane takes part in __match_any_sync.
+  for (int64_t base = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); base < L;
+       base += stride) {
+    const int64_t i = base + lane;
+    const bool valid = i < L;
+    const int t = valid ? ids[i] : 0;
+    const int j = valid ? (int)(i / block) : 0;
+    const bool ok = valid && t >= 0 && t < vocab;
+    if (valid && !ok) set_status(st, PA_ERR_INVALID, (int)(i & 0x7fffffff), t);
+    // Lanes holding the same (token, block) pair elect one leader, which
+    // sets the block's bit unless it is already visible in L2.
+    const unsigned long long key = ok ? (((unsigned long long)(unsigned)t << 6) | (unsigned)j)
+                                      : ~0ull;
+    const unsigned peers = __match_any_sync(0xffffffffu, key);
+    if (ok && lane == __ffs(peers) - 1) {
+      const unsigned long long bit = 1ull << j;
+      if (!(ld_cg_u64(mask + t) & bit)) atomicOr(mask + t, bit);
+    }
+  }
+}
+
+__global__ void df_from_mask_kernel(const unsigned long long* __restrict__ mask, int32_t vocab,
+                                    int32_t* __restrict__ df) {
+  for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < vocab;
+       t += (int64_t)gridDim.x * blockDim.x)
+    df[t] = __popcll(mask[t]);
+}
+
+__global__ void chunk_mindf_kernel(const int32_t* __restrict__ ids, int64_t n_chunks,
+                                   int32_t chunk, int32_t vocab,
+                                   const unsigned long long* __restrict__ mask,
+                                   int32_t* __restrict__ mindf) {
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t c = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; c < n_chunks;
+       c += nwarps) {
+    unsigned best = 0xffffffffu;
+    const int32_t* tok = ids + c * chunk;
+    for (int u = lane; u < chunk; u += 32) {
+      const int t = tok[u];
+      if (t >= 0 && t < vocab) best = min(best, (unsigned)__popcll(mask[t]));
+    }
+    best = __reduce_min_sync(0xffffffffu, best);
+    if (lane == 0) mindf[c] = (int32_t)best;  // all-invalid chunk -> -1 (status already set)
+  }
+}
+
+// Exclusive block-wide prefix count of `flag`; also returns the tile total.
+template <int THREADS>
+__device__ __forceinline__ int block_exclusive_count(bool flag, int* warp_tot, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const unsigned b = __ballot_sync(0xffffffffu, flag);
+  const int in_warp = __popc(b & ((1u << lane) - 1u));
+  if (lane == 0) warp_tot[warp] = __popc(b);
+  __syncthreads();
+  int before = 0, sum = 0;
+#pragma unroll
+  for (int w = 0; w < THREADS / 32; ++w) {
+    const int x = warp_tot[w];
+    before += (w < warp) ? x : 0;
+    sum += x;
+  }
+  __syncthreads();  // warp_tot is reused by the next call
+  *total = sum;
+  return before + in_warp;
+}
+
+template <int THREADS>
+__global__ void __launch_bounds__(THREADS) topk_kernel(const int32_t* __restrict__ mindf,
+                                                       int32_t C, int32_t k, int32_t n_blocks,
+                                                       int32_t* __restrict__ sel) {
+  constexpr int kBins = 66;  // 1..64 valid df values, 65 = invalid entry
+  __shared__ int hist[kBins];
+  __shared__ int warp_tot[THREADS / 32];
+  __shared__ int s_tau, s_need;
+  const int j = blockIdx.x;
+  const int32_t* md = mindf + (int64_t)j * C;
+  for (int i = threadIdx.x; i < kBins; i += THREADS) hist[i] = 0;
+  __syncthreads();
+  for (int c = threadIdx.x; c < C; c += THREADS) {
+    int v = md[c];
+    if (v < 1 || v > n_blocks) v = 65;
+    atomicAdd(&hist[v], 1);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // Threshold tau: the smallest df value at which the k-th best chunk sits;
+    // every chunk below tau is kept, plus the first `need` chunks equal to tau.
+    int tau = 0, need = 0, cum = 0;
+    if (k > 0) {
+      for (int v = 1; v < kBins; ++v) {
+        if (cum + hist[v] >= k) { tau = v; need = k - cum; break; }
+        cum += hist[v];
+      }
+    }
+    s_tau = tau;
+    s_need = need;
+  }
+  __syncthreads();
+  const int tau = s_tau, need = s_need;
+  int base_eq = 0, base_sel = 0;
+  for (int base = 0; base < C; base += THREADS) {
+    const int c = base + threadIdx.x;
+    int v = kBins;
+    if (c < C) {
+      v = md[c];
+      if (v < 1 || v > n_blocks) v = 65;
+    }
+    const bool eq = (c < C) && v == tau;
+    const bool less = (c < C) && v < tau;
+    int tot_eq, tot_sel;
+    const int eq_rank = base_eq + block_exclusive_count<THREADS>(eq, warp_tot, &tot_eq);
+    const bool take = less || (eq && eq_rank < need);
+    const int pos = base_sel + block_exclusive_count<THREADS>(take, warp_tot, &tot_sel);
+    if (take) sel[(int64_t)j * k + pos] = c;
+    base_eq += tot_eq;
+    base_sel += tot_sel;
+  }
+}
+
+int launch_select(const SelectArgs& a, cudaStream_t s) {
+  const int64_t n_chunks = a.L / a.chunk;
+  const int C = a.block / a.chunk;
+  const int n_blocks = (int)(a.L / a.block);
+  if (cudaMemsetAsync(a.mask, 0, sizeof(unsigned long long) * (size_t)a.vocab, s) != cudaSuccess)
+    return PA_ERR_CUDA;
+  if (a.L > 0) {
+    const int threads = 256;
+    const int64_t want = (a.L + threads - 1) / threads;
+    const int grid = (int)(want < 148 * 16 ? want : 148 * 16);
+    presence_mask_kernel<<<grid, threads, 0, s>>>(a.ids, a.L, a.vocab, a.block, a.mask, a.status);
+    const int64_t wwarps = n_chunks;
+    const int64_t wgrid = (wwarps * 32 + threads - 1) / threads;
+    chunk_mindf_kernel<<<(int)(wgrid < 148 * 32 ? wgrid : 148 * 32), threads, 0, s>>>(
+        a.ids, n_chunks, a.chunk, a.vocab, a.mask, a.mindf);
+    if (a.k > 0) topk_kernel<1024><<<n_blocks, 1024, 0, s>>>(a.mindf, C, a.k, n_blocks, a.sel);
+  }
+  if (a.df_out) {
+    const int threads = 256;
+    const int64_t want = ((int64_t)a.vocab + threads - 1) / threads;
+    df_from_mask_kernel<<<(int)(want < 148 * 8 ? want : 148 * 8), threads, 0, s>>>(
+        a.mask, a.vocab, a.df_out);
+  }
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+}  // namespace pa

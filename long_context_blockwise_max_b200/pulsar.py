@@ -1,0 +1,242 @@
+"""Python binding of ``libpulsar_b200.so`` (C ABI in ``include/pulsar.h``).
+
+Argument marshalling only: every function checks shapes, dtypes and devices
+of torch tensors, allocates missing outputs and workspaces with torch (the
+library itself never allocates), and passes raw device pointers and the
+current CUDA stream to the C entry point of the same name.  Every step of the
+computation runs in the library's CUDA kernels; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libpulsar_b200.so")
+
+PA_F32, PA_BF16 = 0, 1
+_STATUS = {0: "PA_OK", -1: "PA_ERR_INVALID", -2: "PA_ERR_UNSUPPORTED", -3: "PA_ERR_WORKSPACE",
+           -4: "PA_ERR_CUDA", -5: "PA_ERR_TIMEOUT", -6: "PA_ERR_RANGE"}
+
+# Every symbol declared in include/pulsar.h.
+ABI_SYMBOLS = (
+    "pa_abi_version", "pa_status_string", "pa_workspace_status", "pa_set_profile_events",
+    "pa_select_workspace_size", "pulsar_select_summaries",
+    "pa_phase1_layout", "pa_phase1_workspace_size", "pulsar_phase1_encode", "star_phase1_encode",
+    "pa_phase2_workspace_size", "star_phase2_attend",
+)
+
+
+class PulsarError(RuntimeError):
+    """A library call returned a negative pa_status."""
+
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {_STATUS.get(code, code)} ({status_string(code)})")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built; run `python -m long_context_blockwise_max_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I32, I64, SZ, D = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_double
+    sig = {
+        "pa_abi_version": (ctypes.c_int, []),
+        "pa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "pa_workspace_status": (ctypes.c_int, [P, P]),
+        "pa_set_profile_events": (ctypes.c_int, [P, P]),
+        "pa_select_workspace_size": (SZ, [I64, I32, I32, I32]),
+        "pulsar_select_summaries": (ctypes.c_int, [P, I64, I32, I32, I32, I32, P, P, P, P, SZ, P]),
+        "pa_phase1_layout": (ctypes.c_int, [I64, I32, I32, I32, ctypes.c_int, P]),
+        "pa_phase1_workspace_size": (SZ, [I64, I32, I32, I32, ctypes.c_int, I32, I32, I32, ctypes.c_int]),
+        "pulsar_phase1_encode": (ctypes.c_int, [P, P, P, ctypes.c_int, I64, I32, I32, I32, D, I32, I32, I32,
+                                                I32, P, P, P, P, P, P, SZ, P]),
+        "star_phase1_encode": (ctypes.c_int, [P, P, P, ctypes.c_int, I64, I32, I32, I32, D, I32, P, P, P, P,
+                                              P, SZ, P]),
+        "pa_phase2_workspace_size": (SZ, [I32, I32, I64, I32, I32, I32, I32]),
+        "star_phase2_attend": (ctypes.c_int, [P, ctypes.c_int, I32, I32, I64, D, P, P, I64, I32, I32, I32,
+                                              I32, P, P, P, P, P, SZ, P]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype, fn.argtypes = res, args
+    return lib
+
+
+_lib = _load()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _check(rc: int, where: str):
+    if rc != 0:
+        raise PulsarError(rc, where)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return PA_F32
+    if t.dtype == torch.bfloat16:
+        return PA_BF16
+    raise PulsarError(-2, f"dtype {t.dtype}")
+
+
+def _dev(*ts):
+    for t in ts:
+        if t is not None:
+            if not t.is_cuda:
+                raise ValueError("tensors must be on a CUDA device")
+            if not t.is_contiguous():
+                raise ValueError("tensors must be contiguous")
+
+
+def _workspace(nbytes: int, device, ws=None):
+    if ws is not None:
+        return ws
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def pa_abi_version() -> int:
+    return _lib.pa_abi_version()
+
+
+def status_string(code: int) -> str:
+    return _lib.pa_status_string(code).decode()
+
+
+def pa_workspace_status(ws: torch.Tensor) -> int:
+    """Device status recorded in ``ws`` by the last call that used it (synchronises)."""
+    return _lib.pa_workspace_status(_ptr(ws), _stream())
+
+
+def pa_set_profile_events(start=None, stop=None) -> None:
+    """Record torch.cuda.Event pair around the dominant kernel of later calls
+    (None, None: off)."""
+    h = lambda e: None if e is None else ctypes.c_void_p(e.cuda_event)
+    _check(_lib.pa_set_profile_events(h(start), h(stop)), "pa_set_profile_events")
+
+
+def pa_select_workspace_size(L, vocab, block, chunk) -> int:
+    return _lib.pa_select_workspace_size(L, vocab, block, chunk)
+
+
+def pulsar_select_summaries(ids: torch.Tensor, vocab: int, block: int, chunk: int, k_chunks: int,
+                            sel=None, df=None, chunk_mindf=None, ws=None, want_df=False,
+                            want_mindf=False):
+    """Max-IDF summary selection. Returns (sel [N][k] int32, df or None, mindf or None, ws)."""
+    _dev(ids)
+    L = ids.numel()
+    n = L // block if block > 0 else 0
+    dev = ids.device
+    if sel is None:
+        sel = torch.empty((n, k_chunks), dtype=torch.int32, device=dev)
+    if want_df and df is None:
+        df = torch.empty(vocab, dtype=torch.int32, device=dev)
+    if want_mindf and chunk_mindf is None:
+        chunk_mindf = torch.empty(L // chunk, dtype=torch.int32, device=dev)
+    need = pa_select_workspace_size(L, vocab, block, chunk)
+    ws = _workspace(need, dev, ws)
+    rc = _lib.pulsar_select_summaries(_ptr(ids), L, vocab, block, chunk, k_chunks, _ptr(sel),
+                                      _ptr(df), _ptr(chunk_mindf), _ptr(ws), ws.numel() * ws.element_size(), _stream())
+    _check(rc, "pulsar_select_summaries")
+    return sel, df, chunk_mindf, ws
+
+
+def pa_phase1_layout(L, block, sink, summary_tokens, star) -> list[int]:
+    n = L // block if block > 0 else 0
+    buf = (ctypes.c_int64 * (max(n, 0) + 1))()
+    _check(_lib.pa_phase1_layout(L, block, sink, summary_tokens, int(star), ctypes.cast(buf, ctypes.c_void_p)),
+           "pa_phase1_layout")
+    return list(buf)
+
+
+def pa_phase1_workspace_size(L, hq, hkv, d, dtype, block, sink, summary_tokens, star) -> int:
+    return _lib.pa_phase1_workspace_size(L, hq, hkv, d, dtype, block, sink, summary_tokens, int(star))
+
+
+def _phase1_outputs(q, k, rows, o, lse, k_ret, v_ret, want_lse):
+    L, hq, d = q.shape
+    hkv = k.shape[1]
+    if o is None:
+        o = torch.empty((rows, hq, d), dtype=q.dtype, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((rows, hq), dtype=torch.float32, device=q.device)
+    if k_ret is None:
+        k_ret = torch.empty((L, hkv, d), dtype=q.dtype, device=q.device)
+    if v_ret is None:
+        v_ret = torch.empty((L, hkv, d), dtype=q.dtype, device=q.device)
+    return o, lse, k_ret, v_ret
+
+
+def pulsar_phase1_encode(q, k, v, rope_theta, block, sink, chunk, k_chunks, sel, o=None, lse=None,
+                         k_ret=None, v_ret=None, ws=None, want_lse=True):
+    """Pulsar Phase 1 for all hosts. Returns (o, lse, k_ret, v_ret, row_off, ws)."""
+    _dev(q, k, v, sel, o, lse, k_ret, v_ret)
+    L, hq, d = q.shape
+    hkv = k.shape[1]
+    dt = _dtype_code(q)
+    row_off = pa_phase1_layout(L, block, sink, k_chunks * chunk, False)
+    o, lse, k_ret, v_ret = _phase1_outputs(q, k, row_off[-1], o, lse, k_ret, v_ret, want_lse)
+    need = pa_phase1_workspace_size(L, hq, hkv, d, dt, block, sink, k_chunks * chunk, False)
+    ws = _workspace(need, q.device, ws)
+    rc = _lib.pulsar_phase1_encode(_ptr(q), _ptr(k), _ptr(v), dt, L, hq, hkv, d, float(rope_theta), block,
+                                   sink, chunk, k_chunks, _ptr(sel), _ptr(o), _ptr(lse), _ptr(k_ret),
+                                   _ptr(v_ret), _ptr(ws), ws.numel() * ws.element_size(), _stream())
+    _check(rc, "pulsar_phase1_encode")
+    return o, lse, k_ret, v_ret, row_off, ws
+
+
+def star_phase1_encode(q, k, v, rope_theta, block, o=None, lse=None, k_ret=None, v_ret=None,
+                       ws=None, want_lse=True):
+    """Star anchor-variant Phase 1. Returns (o, lse, k_ret, v_ret, row_off, ws)."""
+    _dev(q, k, v, o, lse, k_ret, v_ret)
+    L, hq, d = q.shape
+    hkv = k.shape[1]
+    dt = _dtype_code(q)
+    row_off = pa_phase1_layout(L, block, 0, 0, True)
+    o, lse, k_ret, v_ret = _phase1_outputs(q, k, row_off[-1], o, lse, k_ret, v_ret, want_lse)
+    need = pa_phase1_workspace_size(L, hq, hkv, d, dt, block, 0, 0, True)
+    ws = _workspace(need, q.device, ws)
+    rc = _lib.star_phase1_encode(_ptr(q), _ptr(k), _ptr(v), dt, L, hq, hkv, d, float(rope_theta), block,
+                                 _ptr(o), _ptr(lse), _ptr(k_ret), _ptr(v_ret), _ptr(ws), ws.numel(),
+                                 _stream())
+    _check(rc, "star_phase1_encode")
+    return o, lse, k_ret, v_ret, row_off, ws
+
+
+def pa_phase2_workspace_size(B, Tq, T, n_shards, hq, hkv, d) -> int:
+    return _lib.pa_phase2_workspace_size(B, Tq, T, n_shards, hq, hkv, d)
+
+
+def star_phase2_attend(q, k_ret, v_ret, n_shards, q_pos0=0, rope_theta=0.0, o=None, lse=None,
+                       want_partials=False, part_o=None, part_lse=None, ws=None):
+    """Phase-2 split-KV attention + exact merge. q [B][Tq][hq][d]; caches [B][T][hkv][d].
+    Returns (o, lse, part_o, part_lse, ws)."""
+    _dev(q, k_ret, v_ret, o, lse, part_o, part_lse)
+    B, Tq, hq, d = q.shape
+    T, hkv = k_ret.shape[1], k_ret.shape[2]
+    dt = _dtype_code(q)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Tq, hq), dtype=torch.float32, device=q.device)
+    if want_partials:
+        if part_o is None:
+            part_o = torch.empty((B, n_shards, Tq, hq, d), dtype=torch.float32, device=q.device)
+        if part_lse is None:
+            part_lse = torch.empty((B, n_shards, Tq, hq), dtype=torch.float32, device=q.device)
+    need = pa_phase2_workspace_size(B, Tq, T, n_shards, hq, hkv, d)
+    ws = _workspace(need, q.device, ws)
+    rc = _lib.star_phase2_attend(_ptr(q), dt, B, Tq, int(q_pos0), float(rope_theta), _ptr(k_ret), _ptr(v_ret),
+                                 T, n_shards, hq, hkv, d, _ptr(o), _ptr(lse), _ptr(part_o), _ptr(part_lse),
+                                 _ptr(ws), ws.numel() * ws.element_size(), _stream())
+    _check(rc, "star_phase2_attend")
+    return o, lse, part_o, part_lse, ws

@@ -1,0 +1,88 @@
+"""Host-side checks of the C ABI (no GPU needed): the shared library loads,
+exports every function include/pulsar.h declares, and rejects invalid
+arguments on the host before any launch."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from long_context_blockwise_max_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    from long_context_blockwise_max_b200 import pulsar
+    return pulsar
+
+
+def _header_functions():
+    src = open(os.path.join(ROOT, "include", "pulsar.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:int|size_t|const char\*)\s+(\w+)\s*\(", src, flags=re.M)))
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = _header_functions()
+    assert len(names) == 12
+    assert sorted(lib.ABI_SYMBOLS) == names
+    so = ctypes.CDLL(lib.LIB_PATH)
+    for n in names:
+        assert hasattr(so, n), n
+    assert lib.pa_abi_version() == 1
+    assert lib.status_string(-3).startswith("workspace")
+
+
+def test_phase1_layout_matches_oracle(lib):
+    L, b, sink, chunk, k = 8 * 16384, 16384, 64, 32, 64
+    sel = np.zeros((8, k), dtype=np.int64)
+    for star in (False, True):
+        want = oracle.host_row_offsets(oracle.host_positions(L, b, sink, chunk, sel, star=star))
+        got = lib.pa_phase1_layout(L, b, sink, k * chunk, star)
+        assert got == want.tolist()
+
+
+def test_workspace_sizes(lib):
+    assert lib.pa_select_workspace_size(2048, 1000, 512, 32) >= 256 + 8 * 1000
+    assert lib.pa_select_workspace_size(2047, 1000, 512, 32) == 0
+    assert lib.pa_phase1_workspace_size(2048, 4, 2, 64, 0, 512, 64, 64, False) > 0
+    assert lib.pa_phase1_workspace_size(2048, 4, 2, 96, 0, 512, 64, 64, False) == 0
+    assert lib.pa_phase2_workspace_size(16, 1, 131072, 8, 32, 8, 128) > 0
+    assert lib.pa_phase2_workspace_size(16, 1, 131072, 0, 32, 8, 128) == 0
+
+
+def test_host_validation_rejects_before_launch(lib):
+    so = lib._lib
+    ws = ctypes.c_void_p(256)   # never dereferenced: validation fails first
+    dummy = ctypes.c_void_p(4096)
+    # L not a multiple of the block
+    assert so.pulsar_select_summaries(dummy, 1000, 100, 512, 32, 2, dummy, None, None, ws, 1 << 20, None) == -1
+    # k larger than the chunk count
+    assert so.pulsar_select_summaries(dummy, 1024, 100, 512, 32, 17, dummy, None, None, ws, 1 << 20, None) == -1
+    # more than 64 blocks
+    assert so.pulsar_select_summaries(dummy, 65 * 16, 100, 16, 16, 1, dummy, None, None, ws, 1 << 20, None) == -2
+    # workspace too small
+    assert so.pulsar_select_summaries(dummy, 1024, 100, 512, 32, 2, dummy, None, None, ws, 16, None) == -3
+    # head_dim 96 unsupported; hq not a multiple of hkv invalid
+    args = (dummy, dummy, dummy, 0, 2048, 4, 2, 96, 10000.0, 512, 64, 32, 2, dummy, dummy, None, dummy, dummy,
+            ws, 1 << 30, None)
+    assert so.pulsar_phase1_encode(*args) == -2
+    args = (dummy, dummy, dummy, 0, 2048, 3, 2, 64, 10000.0, 512, 64, 32, 2, dummy, dummy, None, dummy, dummy,
+            ws, 1 << 30, None)
+    assert so.pulsar_phase1_encode(*args) == -1
+    # sink not a multiple of 16
+    args = (dummy, dummy, dummy, 0, 2048, 4, 2, 64, 10000.0, 512, 40, 32, 2, dummy, dummy, None, dummy, dummy,
+            ws, 1 << 30, None)
+    assert so.pulsar_phase1_encode(*args) == -2
+    # misaligned output pointer
+    args = (dummy, dummy, dummy, 0, 2048, 4, 2, 64, 10000.0, 512, dummy, None, ctypes.c_void_p(4098), dummy,
+            ws, 1 << 30, None)
+    assert so.star_phase1_encode(*args) == -2
+    # phase 2: zero shards
+    assert so.star_phase2_attend(dummy, 1, 1, 1, 0, 0.0, dummy, dummy, 100, 0, 32, 8, 128, dummy, dummy, None,
+                                 None, ws, 1 << 30, None) == -1

@@ -1,0 +1,101 @@
+"""GPU parity of Phase-2 split-KV attention and the exact LSE merge against
+the fp64 oracle (Pulsar Attention page §2.2; Star Attention review,
+Algorithm 2 as corrected): per-shard partials and merged outputs at small
+sizes, and sampled (batch, kv-head) groups of the 128K decode, the 128K
+64-token query and the 1M-token decode."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from helpers import LSE_TOL, O_TOL, assert_close, f64
+from long_context_blockwise_max_b200 import workloads
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda:0")
+
+
+@pytest.fixture(scope="module")
+def P():
+    from long_context_blockwise_max_b200 import pulsar
+    return pulsar
+
+
+def _oracle_group(q, kc, vc, b, kvh, g, n_shards, q_pos0, theta):
+    """Oracle for one (batch, kv head) group: its g query heads only."""
+    qs = f64(q[b:b + 1, :, kvh * g:(kvh + 1) * g, :])
+    ks = f64(kc[b:b + 1, :, kvh:kvh + 1, :])
+    vs = f64(vc[b:b + 1, :, kvh:kvh + 1, :])
+    return oracle.phase2_attend(qs, ks, vs, n_shards, q_pos0, theta)
+
+
+def test_tiny_fp32_full(P):
+    w = workloads.TINY
+    B, T, S = 2, w.L, w.n_blocks
+    q = workloads.normal((B, w.q_tokens, w.hq, w.d), 50, torch.float32)
+    kc = workloads.normal((B, T, w.hkv, w.d), 51, torch.float32)
+    vc = workloads.normal((B, T, w.hkv, w.d), 52, torch.float32)
+    o, lse, po, pl, ws = P.star_phase2_attend(q.to(DEV), kc.to(DEV), vc.to(DEV), S, q_pos0=T,
+                                              rope_theta=w.rope_theta, want_partials=True)
+    assert P.pa_workspace_status(ws) == 0
+    ro, rl, ra, rs = oracle.phase2_attend(f64(q), f64(kc), f64(vc), S, T, w.rope_theta)
+    assert_close(f64(o.cpu()), ro, O_TOL[torch.float32], "O")
+    assert_close(lse.cpu().double().numpy(), rl, LSE_TOL, "lse")
+    assert_close(po.cpu().double().numpy(), ra, O_TOL[torch.float32], "A_h")
+    assert_close(pl.cpu().double().numpy(), rs, LSE_TOL, "s_h")
+
+
+@pytest.mark.parametrize("case", [
+    # (B, Tq, T, S, hq, hkv, d, theta)
+    (1, 64, 3000, 5, 8, 2, 128, 500000.0),     # ragged shards, a 64-token query
+    (3, 1, 999, 4, 32, 8, 128, 500000.0),      # decode rows, ragged cache
+    (2, 7, 10, 16, 4, 4, 64, 0.0),             # more shards than keys: empty shards, no RoPE
+    (1, 3, 0, 2, 4, 2, 64, 10000.0),           # empty cache: O = 0, lse = -inf
+])
+def test_bf16_small_full(P, case):
+    B, Tq, T, S, hq, hkv, d, theta = case
+    q = workloads.normal((B, Tq, hq, d), 60, torch.bfloat16)
+    kc = workloads.normal((B, T, hkv, d), 61, torch.bfloat16)
+    vc = workloads.normal((B, T, hkv, d), 62, torch.bfloat16)
+    o, lse, po, pl, ws = P.star_phase2_attend(q.to(DEV), kc.to(DEV), vc.to(DEV), S, q_pos0=T,
+                                              rope_theta=theta, want_partials=True)
+    assert P.pa_workspace_status(ws) == 0
+    ro, rl, ra, rs = oracle.phase2_attend(f64(q), f64(kc), f64(vc), S, T, theta)
+    assert_close(f64(o.cpu()), ro, O_TOL[torch.bfloat16], "O")
+    assert_close(lse.cpu().double().numpy(), rl, LSE_TOL, "lse")
+    assert_close(po.cpu().double().numpy(), ra, O_TOL[torch.bfloat16], "A_h")
+    assert_close(pl.cpu().double().numpy(), rs, LSE_TOL, "s_h")
+
+
+@pytest.mark.parametrize("wname,groups", [
+    ("decode_128k_b16", [(0, 0), (9, 5), (15, 7)]),
+    ("scale_1m", [(0, 3), (3, 7)]),
+])
+def test_decode_sampled_groups(P, wname, groups):
+    w = workloads.WORKLOADS[wname]
+    q, kc, vc = w.decode_inputs(device=DEV)
+    T, S, g = w.decode_T, w.decode_shards, w.hq // w.hkv
+    o, lse, po, pl, ws = P.star_phase2_attend(q, kc, vc, S, q_pos0=T, rope_theta=w.rope_theta,
+                                              want_partials=True)
+    assert P.pa_workspace_status(ws) == 0
+    for b, kvh in groups:
+        ro, rl, ra, rs = _oracle_group(q, kc, vc, b, kvh, g, S, T, w.rope_theta)
+        hs = slice(kvh * g, (kvh + 1) * g)
+        assert_close(f64(o[b:b + 1, :, hs].cpu()), ro, O_TOL[torch.bfloat16], "O")
+        assert_close(lse[b:b + 1, :, hs].cpu().double().numpy(), rl, LSE_TOL, "lse")
+        assert_close(pl[b:b + 1, :, :, hs].cpu().double().numpy(), rs, LSE_TOL, "s_h")
+
+
+def test_query_128k_sampled_groups(P):
+    w = workloads.LLAMA_128K
+    q = w.query(device=DEV)
+    kc = workloads.normal((1, w.L, w.hkv, w.d), workloads.SEED_KC, w.dtype, DEV)
+    vc = workloads.normal((1, w.L, w.hkv, w.d), workloads.SEED_VC, w.dtype, DEV)
+    o, lse, _, _, ws = P.star_phase2_attend(q, kc, vc, w.n_blocks, q_pos0=w.L, rope_theta=w.rope_theta)
+    assert P.pa_workspace_status(ws) == 0
+    g = w.hq // w.hkv
+    for kvh in (0, 6):
+        ro, rl, _, _ = _oracle_group(q, kc, vc, 0, kvh, g, w.n_blocks, w.L, w.rope_theta)
+        hs = slice(kvh * g, (kvh + 1) * g)
+        assert_close(f64(o[:, :, hs].cpu()), ro, O_TOL[torch.bfloat16], "O")
+        assert_close(lse[:, :, hs].cpu().double().numpy(), rl, LSE_TOL, "lse")
