@@ -63,6 +63,8 @@ struct Phase1Args {
   void* kr;                     // [L][hkv][d] rotated K in QK type (fp16) or == k_ret (fp32)
   DeviceStatus* status;
 };
+bool phase1_tc_supported(const Phase1Args& a);
+int launch_phase1_tc(const Phase1Args& a, cudaStream_t s);
 size_t phase1_workspace_bytes(int64_t L, int32_t hq, int32_t hkv, int32_t d, int dtype,
                               int64_t total_rows);
 int launch_phase1(const Phase1Args& a, cudaStream_t s);

@@ -249,8 +249,11 @@ static int launch_phase1_t(const Phase1Args& a, cudaStream_t s) {
   }
   const QT* kq = a.kr ? static_cast<const QT*>(a.kr) : static_cast<const QT*>(a.k_ret);
   const dim3 grid(a.ht.tile_off[a.ht.n_hosts], a.hq);
+  int rc = PA_OK;
   profile_begin(s);
-  if (grid.x > 0) {
+  if (phase1_tc_supported(a)) {
+    rc = launch_phase1_tc(a, s);
+  } else if (grid.x > 0) {
     if (a.d == 128)
       phase1_simt_kernel<128, QT, VT, OT><<<grid, 256, 0, s>>>(
           static_cast<const QT*>(a.qr), kq, static_cast<const VT*>(a.v), a.rowpos, a.ht, a.hq,
@@ -261,6 +264,7 @@ static int launch_phase1_t(const Phase1Args& a, cudaStream_t s) {
           a.hkv, static_cast<OT*>(a.o), a.lse);
   }
   profile_end(s);
+  if (rc != PA_OK) return rc;
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
