@@ -88,6 +88,7 @@ struct Phase2Args {
   float* unit_lse;              // workspace [B][units][Tq][hq]
   DeviceStatus* status;
 };
+int launch_phase2_mma(const Phase2Args& a, cudaStream_t s);
 int32_t phase2_split(int32_t B, int32_t Tq, int64_t T, int32_t n_shards, int32_t hq,
                      int32_t hkv);
 size_t phase2_workspace_bytes(int32_t B, int32_t Tq, int64_t T, int32_t n_shards, int32_t hq,

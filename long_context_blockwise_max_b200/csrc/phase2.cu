@@ -189,11 +189,15 @@ __global__ void merge_kernel(Phase2Args a) {
   }
 }
 
+// Splits per shard so that small batches still fill the GPU: work units are
+// (batch, shard split, kv head, group of 8 query rows); aim for 4 units per
+// SM, with at least 512 keys per split.  Independent of the dtype, so that
+// the workspace size does not depend on it.
 int32_t phase2_split(int32_t B, int32_t Tq, int64_t T, int32_t n_shards, int32_t hq,
                      int32_t hkv) {
   const int g = hq / hkv;
-  const int64_t row_tiles = ((int64_t)Tq * g + 127) / 128;
-  const int64_t base = (int64_t)B * n_shards * hkv * row_tiles;
+  const int64_t row_groups = ((int64_t)Tq * g + 7) / 8;
+  const int64_t base = (int64_t)B * n_shards * hkv * row_groups;
   const int64_t shard_len = (T + n_shards - 1) / n_shards;
   int64_t want = base > 0 ? (4 * 148 + base - 1) / base : 1;
   const int64_t cap = shard_len / 512;
@@ -231,12 +235,16 @@ static int launch_phase2_t(const Phase2Args& a, cudaStream_t s) {
   const int units = a.n_shards * a.n_split;
   const int g = a.hq / a.hkv;
   const dim3 grid((unsigned)(a.B * units), a.hkv, (unsigned)((a.Tq * g + 127) / 128));
+  int rc = PA_OK;
   profile_begin(s);
-  if (grid.x > 0 && grid.z > 0) {
+  if (a.dtype == PA_BF16) {
+    rc = launch_phase2_mma(a, s);
+  } else if (grid.x > 0 && grid.z > 0) {
     if (a.d == 128) phase2_simt_kernel<128, IT><<<grid, 256, 0, s>>>(a);
     else phase2_simt_kernel<64, IT><<<grid, 256, 0, s>>>(a);
   }
   profile_end(s);
+  if (rc != PA_OK) return rc;
   const int64_t nrows = (int64_t)a.B * a.Tq * a.hq;
   if (nrows > 0) {
     const int64_t want = (nrows * 32 + 255) / 256;
