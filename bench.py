@@ -140,19 +140,19 @@ class Step:
         self.ws2 = torch.empty(P.pa_phase2_workspace_size(1, w.q_tokens, w.L, n, w.hq, w.hkv, w.d),
                                dtype=torch.uint8, device=dev)
         self.attn_events = None
+        self.p2_events = None
 
     def run(self):
         P, w = self.P, self.w
         P.pulsar_select_summaries(self.ids, w.vocab, w.block, w.chunk, w.k_chunks, sel=self.sel, ws=self.ws_sel)
-        if self.attn_events is not None:
-            P.pa_set_profile_events(*self.attn_events)
+        P.pa_set_profile_events(*(self.attn_events or (None, None)))
         P.pulsar_phase1_encode(self.q, self.k, self.v, w.rope_theta, w.block, w.sink, w.chunk, w.k_chunks,
                                self.sel, o=self.o1, lse=self.lse1, k_ret=self.k_ret, v_ret=self.v_ret,
                                ws=self.ws1)
-        if self.attn_events is not None:
-            P.pa_set_profile_events(None, None)
+        P.pa_set_profile_events(*(self.p2_events or (None, None)))
         P.star_phase2_attend(self.query, self.k_ret[None], self.v_ret[None], w.n_blocks, q_pos0=w.L,
                              rope_theta=w.rope_theta, o=self.o2, lse=self.lse2, ws=self.ws2)
+        P.pa_set_profile_events(None, None)
 
     # kernels of ours launched by one step (selection 3, Phase 1 3, Phase 2 3)
     LAUNCHES = 9
@@ -200,7 +200,8 @@ def run_ours(args, rank, world, local_rank, dist_on):
     # ---- timed region: K steps -----------------------------------------
     K = args.steps
     ev_attn = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    for a, b in ev_attn:      # torch creates the CUDA event on its first record
+    ev_p2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for a, b in ev_attn + ev_p2:      # torch creates the CUDA event on its first record
         a.record()
         b.record()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -209,13 +210,16 @@ def run_ours(args, rank, world, local_rank, dist_on):
         t0.record()
         for i in range(K):
             step.attn_events = ev_attn[i]
+            step.p2_events = ev_p2[i]
             step.run()
         t1.record()
         torch.cuda.synchronize()
     step.attn_events = None
+    step.p2_events = None
     sync_all(dist_on)
     ms = max_over_ranks(t0.elapsed_time(t1), dist_on) / K
     attn_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_attn)
+    p2_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_p2)
 
     flops = attn_flops(w)
     tokens_per_s = w.L * world / (ms * 1e-3)
@@ -342,7 +346,10 @@ def run_ours(args, rank, world, local_rank, dist_on):
                      "kernel_ms": round(attn_ms, 3), "flop_per_launch": flops},
         "phase1": {"attn_ms": round(attn_ms, 3), "tflop": round(flops / 1e12, 3),
                    "tflop_s": round(attn_tf, 1)},
-        "phase2_query": {"kv_bytes": q2_bytes},
+        "phase2_query": {"kernel_ms": round(p2_ms, 4), "kv_bytes": q2_bytes,
+                         "gb_s": round(q2_bytes / (p2_ms * 1e-3) / 1e9, 1),
+                         "frac_hbm": round(q2_bytes / (p2_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                         "tflop_s": round(4.0 * w.d * w.hq * w.q_tokens * w.L / (p2_ms * 1e-3) / 1e12, 1)},
     }
     line.update(extra)
     return line
