@@ -122,6 +122,33 @@ int pulsar_select_summaries(const int32_t* ids, int64_t L, int32_t vocab, int32_
                             int32_t chunk, int32_t k_chunks, int32_t* sel, int32_t* df_opt,
                             int32_t* chunk_mindf_opt, void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * Allocation-free variant of pulsar_select_summaries.  The paper has no
+ * counterpart to this call: it exists for callers that cannot allocate
+ * device memory -- e.g. a plugin inside a host application that owns every
+ * device allocation, or a latency-critical serving thread that must never
+ * call cudaMalloc (which may synchronise the whole device).  The caller
+ * passes inputs and outputs only (same meaning, layout and results as
+ * pulsar_select_summaries); the scratch lives in a fixed array inside this
+ * library's device memory, which every GPU that loads the library keeps
+ * until the process exits.
+ *
+ * Limits: vocab <= 262144 and L / chunk <= 65536 (PA_ERR_UNSUPPORTED
+ * beyond), plus every rule of pulsar_select_summaries.  No cudaMalloc,
+ * cudaFree or other allocating routine is called.
+ * Set-up: the first call on a device looks up the array's device address
+ * (with that device current) and caches it; make that first call before any
+ * stream capture.  Every call reuses the same array and clears what must
+ * start at zero, so calls that may overlap on the GPU (different streams, or
+ * different host threads, without ordering between them) race with each
+ * other and must be serialised by the caller.  Device-detected invalid ids
+ * are skipped as in pulsar_select_summaries, but this call has no workspace
+ * whose status could be read back: pass ids in [0, vocab).
+ */
+int pulsar_select_summaries_noalloc(const int32_t* ids, int64_t L, int32_t vocab, int32_t block,
+                                    int32_t chunk, int32_t k_chunks, int32_t* sel, int32_t* df_opt,
+                                    int32_t* chunk_mindf_opt, void* stream);
+
 /* ------------------------------------------------------------------------ */
 /* (a4-a5) Phase-1 context encoding   [PS] Fase 1; [P] §2, §2.1; [S] summary */
 /* ------------------------------------------------------------------------ */

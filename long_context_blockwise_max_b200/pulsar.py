@@ -23,7 +23,7 @@ _STATUS = {0: "PA_OK", -1: "PA_ERR_INVALID", -2: "PA_ERR_UNSUPPORTED", -3: "PA_E
 # Every symbol declared in include/pulsar.h.
 ABI_SYMBOLS = (
     "pa_abi_version", "pa_status_string", "pa_workspace_status", "pa_set_profile_events",
-    "pa_select_workspace_size", "pulsar_select_summaries",
+    "pa_select_workspace_size", "pulsar_select_summaries", "pulsar_select_summaries_noalloc",
     "pa_phase1_layout", "pa_phase1_workspace_size", "pulsar_phase1_encode", "star_phase1_encode",
     "pa_phase2_workspace_size", "star_phase2_attend",
 )
@@ -49,6 +49,7 @@ def _load() -> ctypes.CDLL:
         "pa_set_profile_events": (ctypes.c_int, [P, P]),
         "pa_select_workspace_size": (SZ, [I64, I32, I32, I32]),
         "pulsar_select_summaries": (ctypes.c_int, [P, I64, I32, I32, I32, I32, P, P, P, P, SZ, P]),
+        "pulsar_select_summaries_noalloc": (ctypes.c_int, [P, I64, I32, I32, I32, I32, P, P, P, P]),
         "pa_phase1_layout": (ctypes.c_int, [I64, I32, I32, I32, ctypes.c_int, P]),
         "pa_phase1_workspace_size": (SZ, [I64, I32, I32, I32, ctypes.c_int, I32, I32, I32, ctypes.c_int]),
         "pulsar_phase1_encode": (ctypes.c_int, [P, P, P, ctypes.c_int, I64, I32, I32, I32, D, I32, I32, I32,
@@ -148,6 +149,18 @@ def pulsar_select_summaries(ids: torch.Tensor, vocab: int, block: int, chunk: in
                                       _ptr(df), _ptr(chunk_mindf), _ptr(ws), ws.numel() * ws.element_size(), _stream())
     _check(rc, "pulsar_select_summaries")
     return sel, df, chunk_mindf, ws
+
+
+def pulsar_select_summaries_noalloc(ids: torch.Tensor, vocab: int, block: int, chunk: int, k_chunks: int,
+                                    sel: torch.Tensor, df=None, chunk_mindf=None):
+    """Selection with no workspace, for callers that cannot allocate device
+    memory: writes into the caller's preallocated ``sel`` (and optional
+    ``df`` / ``chunk_mindf``) and allocates nothing.  Returns ``sel``."""
+    _dev(ids, sel, df, chunk_mindf)
+    rc = _lib.pulsar_select_summaries_noalloc(_ptr(ids), ids.numel(), vocab, block, chunk, k_chunks, _ptr(sel),
+                                              _ptr(df), _ptr(chunk_mindf), _stream())
+    _check(rc, "pulsar_select_summaries_noalloc")
+    return sel
 
 
 def pa_phase1_layout(L, block, sink, summary_tokens, star) -> list[int]:
