@@ -426,6 +426,54 @@ def run_reference(args):
                     "d2h_bytes_per_step": 0}}
 
 
+def run_profile_case(name, steps, warmup):
+    """A single kernel family on a small workload, for ncu captures:
+    phase1-32k (Pulsar Phase 1, 32K shape), decode-128k (Phase-2 decode),
+    query-128k (Phase-2 64-token query), rope-32k (the RoPE prepass alone is
+    part of phase1-32k).  Prints one JSON line with the mean call time."""
+    from long_context_blockwise_max_b200 import pulsar as P
+    dev = torch.device("cuda", 0)
+    if name == "phase1-32k":
+        w = workloads.LLAMA_32K
+        q, k, v = w.qkv(device=dev)
+        sel, _, _, _ = P.pulsar_select_summaries(torch.from_numpy(w.token_ids()).to(dev), w.vocab, w.block,
+                                                 w.chunk, w.k_chunks)
+        out = P.pulsar_phase1_encode(q, k, v, w.rope_theta, w.block, w.sink, w.chunk, w.k_chunks, sel)
+        o, lse, kr, vr, _, ws = out
+
+        def call():
+            P.pulsar_phase1_encode(q, k, v, w.rope_theta, w.block, w.sink, w.chunk, w.k_chunks, sel, o=o, lse=lse,
+                                   k_ret=kr, v_ret=vr, ws=ws)
+    elif name == "decode-128k":
+        w = DECODE
+        q, kc, vc = w.decode_inputs(device=dev)
+        o, lse, _, _, ws = P.star_phase2_attend(q, kc, vc, w.decode_shards, w.decode_T, w.rope_theta)
+
+        def call():
+            P.star_phase2_attend(q, kc, vc, w.decode_shards, w.decode_T, w.rope_theta, o=o, lse=lse, ws=ws)
+    elif name == "query-128k":
+        w = WORKLOAD
+        q = w.query(device=dev)
+        kc = workloads.normal((1, w.L, w.hkv, w.d), workloads.SEED_KC, w.dtype, dev)
+        vc = workloads.normal((1, w.L, w.hkv, w.d), workloads.SEED_VC, w.dtype, dev)
+        o, lse, _, _, ws = P.star_phase2_attend(q, kc, vc, w.n_blocks, w.L, w.rope_theta)
+
+        def call():
+            P.star_phase2_attend(q, kc, vc, w.n_blocks, w.L, w.rope_theta, o=o, lse=lse, ws=ws)
+    else:
+        raise SystemExit(f"unknown profile case {name}")
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        call()
+    e1.record()
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_case": name, "steps": steps, "ms_per_call": e0.elapsed_time(e1) / max(steps, 1)}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -434,7 +482,12 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--headline-only", action="store_true", help="skip the side measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", default=None,
+                    help="run one kernel family on a small workload (phase1-32k, decode-128k, query-128k)")
     args = ap.parse_args()
+    if args.profile_case:
+        run_profile_case(args.profile_case, args.steps, args.warmup)
+        return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
