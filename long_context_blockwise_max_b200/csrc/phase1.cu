@@ -53,19 +53,22 @@ __global__ void rowpos_kernel(HostTable ht, const int32_t* __restrict__ sel,
   }
 }
 
-template <typename T> __device__ __forceinline__ void check_range(float, DeviceStatus*) {}
-template <> __device__ __forceinline__ void check_range<__half>(float x, DeviceStatus* st) {
-  if (!(fabsf(x) <= 65504.f)) set_status(st, PA_ERR_RANGE, 0, 0);
-}
-
 // RoPE (rotate-half): for m < d/2, a = p * omega_m,
 //   x'[m] = x[m] cos a - x[m + d/2] sin a,  x'[m + d/2] = x[m + d/2] cos a + x[m] sin a.
 // The angle and its sine/cosine are evaluated in fp64, the rotation in fp32.
+// Each thread rotates one 16-byte vector of x[m..] together with the
+// matching vector of x[m + d/2 ..]; a CTA covers POS positions, all heads.
+template <typename T, int N>
+struct alignas(16) Vec {
+  T v[N];
+};
+
 template <typename IT, typename QT, int POS>
 __global__ void __launch_bounds__(256) rope_qk_kernel(
     const IT* __restrict__ q, const IT* __restrict__ k, int64_t L, int hq, int hkv, int d,
     RopeFreqs f, float qscale, QT* __restrict__ qr, QT* __restrict__ kr, IT* __restrict__ k_ret,
     DeviceStatus* st) {
+  constexpr int VEC = 16 / sizeof(IT);          // input elements per 16-byte vector
   __shared__ float2 cs[POS][kMaxHalfDim];
   const int half = d / 2;
   const int64_t p0 = (int64_t)blockIdx.x * POS;
@@ -76,39 +79,63 @@ __global__ void __launch_bounds__(256) rope_qk_kernel(
     cs[pp][m] = make_float2((float)cn, (float)sn);
   }
   __syncthreads();
-  const int per_pos_q = hq * half, per_pos_k = hkv * half;
-  for (int e = threadIdx.x; e < POS * (per_pos_q + per_pos_k); e += blockDim.x) {
-    const int pp = e / (per_pos_q + per_pos_k);
+  const int vpr = half / VEC;                         // vectors per half row
+  const int per_pos = (hq + hkv) * vpr;
+  bool bad = false;
+  for (int e = threadIdx.x; e < POS * per_pos; e += blockDim.x) {
+    const int pp = e / per_pos;
     const int64_t p = p0 + pp;
     if (p >= L) continue;
-    int w = e % (per_pos_q + per_pos_k);
-    const bool is_q = w < per_pos_q;
-    if (!is_q) w -= per_pos_q;
-    const int h = w / half, m = w % half;
-    const int H = is_q ? hq : hkv;
-    const int64_t base = (p * H + h) * (int64_t)d;
+    const int w = e % per_pos;
+    const int row = w / vpr, m0 = (w % vpr) * VEC;
+    const bool is_q = row < hq;
+    const int h = is_q ? row : row - hq;
+    const int64_t base = (p * (is_q ? hq : hkv) + h) * (int64_t)d;
     const IT* src = is_q ? q : k;
-    const float x1 = to_f32(src[base + m]), x2 = to_f32(src[base + m + half]);
-    const float2 c = cs[pp][m];
-    const float y1 = x1 * c.x - x2 * c.y;
-    const float y2 = x2 * c.x + x1 * c.y;
+    const Vec<IT, VEC> a = *reinterpret_cast<const Vec<IT, VEC>*>(src + base + m0);
+    const Vec<IT, VEC> b = *reinterpret_cast<const Vec<IT, VEC>*>(src + base + m0 + half);
+    float y1[VEC], y2[VEC];
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) {
+      const float2 c = cs[pp][m0 + i];
+      const float x1 = to_f32(a.v[i]), x2 = to_f32(b.v[i]);
+      y1[i] = x1 * c.x - x2 * c.y;
+      y2[i] = x2 * c.x + x1 * c.y;
+    }
     if (is_q) {
-      const float a = y1 * qscale, b = y2 * qscale;
-      check_range<QT>(a, st);
-      check_range<QT>(b, st);
-      qr[base + m] = from_f32<QT>(a);
-      qr[base + m + half] = from_f32<QT>(b);
+      Vec<QT, VEC> o1, o2;
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) {
+        const float u1 = y1[i] * qscale, u2 = y2[i] * qscale;
+        if (sizeof(QT) == 2) bad |= !(fabsf(u1) <= 65504.f) || !(fabsf(u2) <= 65504.f);
+        o1.v[i] = from_f32<QT>(u1);
+        o2.v[i] = from_f32<QT>(u2);
+      }
+      *reinterpret_cast<Vec<QT, VEC>*>(qr + base + m0) = o1;
+      *reinterpret_cast<Vec<QT, VEC>*>(qr + base + m0 + half) = o2;
     } else {
-      k_ret[base + m] = from_f32<IT>(y1);
-      k_ret[base + m + half] = from_f32<IT>(y2);
+      Vec<IT, VEC> r1, r2;
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) {
+        r1.v[i] = from_f32<IT>(y1[i]);
+        r2.v[i] = from_f32<IT>(y2[i]);
+      }
+      *reinterpret_cast<Vec<IT, VEC>*>(k_ret + base + m0) = r1;
+      *reinterpret_cast<Vec<IT, VEC>*>(k_ret + base + m0 + half) = r2;
       if (kr != nullptr) {
-        check_range<QT>(y1, st);
-        check_range<QT>(y2, st);
-        kr[base + m] = from_f32<QT>(y1);
-        kr[base + m + half] = from_f32<QT>(y2);
+        Vec<QT, VEC> o1, o2;
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) {
+          if (sizeof(QT) == 2) bad |= !(fabsf(y1[i]) <= 65504.f) || !(fabsf(y2[i]) <= 65504.f);
+          o1.v[i] = from_f32<QT>(y1[i]);
+          o2.v[i] = from_f32<QT>(y2[i]);
+        }
+        *reinterpret_cast<Vec<QT, VEC>*>(kr + base + m0) = o1;
+        *reinterpret_cast<Vec<QT, VEC>*>(kr + base + m0 + half) = o2;
       }
     }
   }
+  if (bad) set_status(st, PA_ERR_RANGE, 0, 0);
 }
 
 // ---------------------------------------------------------------------------
@@ -235,7 +262,7 @@ static int launch_phase1_t(const Phase1Args& a, cudaStream_t s) {
   for (int m = 0; m < kMaxHalfDim; ++m)
     f.omega[m] = (m < a.d / 2) ? pow(a.rope_theta, -2.0 * m / a.d) : 0.0;
   const float qscale = (float)(kLog2e / sqrt((double)a.d));
-  constexpr int POS = 4;
+  constexpr int POS = 8;
   if (a.L > 0) {
     rope_qk_kernel<IT, QT, POS><<<(unsigned)((a.L + POS - 1) / POS), 256, 0, s>>>(
         static_cast<const IT*>(a.q), static_cast<const IT*>(a.k), a.L, a.hq, a.hkv, a.d, f,

@@ -296,21 +296,27 @@ __global__ void __launch_bounds__(384, 1) phase1_tc_kernel(const __grid_constant
     for (int j = 0; j < nkv; ++j) {
       if (!mbar_wait(&bars->s_full[t], j & 1, abort, kWaitLimitNs, gabort)) { fail(9); ok = false; break; }
       tc_fence_after();
-      uint32_t sr[4][32];
+      uint32_t sr[128];
+      tmem_ld_x128(s_tmem, sr);
+      // row max with 8 independent partial maxima (short dependency chains);
+      // only the diagonal tile needs the causal / ragged-end mask
+      float mx[8];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld_x32(s_tmem + 32 * c, sr[c]);
-      const bool diag = (j == nkv - 1);
-      const int lim = min(r, n - 1) - j * 128;   // columns <= lim are visible
-      float mt = -INFINITY;
+      for (int e = 0; e < 8; ++e) mx[e] = -INFINITY;
+      if (j == nkv - 1) {
+        const int lim = min(r, n - 1) - j * 128;   // columns <= lim are visible
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          float x = __uint_as_float(sr[c][i]);
-          if (diag && (32 * c + i) > lim) x = -INFINITY;
-          sr[c][i] = __float_as_uint(x);
-          mt = fmaxf(mt, x);
+        for (int i = 0; i < 128; ++i) {
+          const float x = (i > lim) ? -INFINITY : __uint_as_float(sr[i]);
+          sr[i] = __float_as_uint(x);
+          mx[i & 7] = fmaxf(mx[i & 7], x);
         }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 128; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(sr[i]));
+      }
+      const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
       const float m_new = fmaxf(m_run, mt);
       const bool need = m_new > m_run + 8.f;   // lazy rescale: only when P could exceed 2^8
       float alpha = 1.f;
@@ -319,19 +325,22 @@ __global__ void __launch_bounds__(384, 1) phase1_tc_kernel(const __grid_constant
         m_run = m_new;
       }
       const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-      float sum = 0.f;
+      float sm[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) sm[e] = 0.f;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float p0 = fast_exp2(__uint_as_float(sr[c][2 * i]) - m_use);
-          const float p1 = fast_exp2(__uint_as_float(sr[c][2 * i + 1]) - m_use);
-          sum += p0 + p1;
+          const float p0 = fast_exp2(__uint_as_float(sr[32 * c + 2 * i]) - m_use);
+          const float p1 = fast_exp2(__uint_as_float(sr[32 * c + 2 * i + 1]) - m_use);
+          sm[i & 7] += p0 + p1;
           pk[i] = pack_bf16x2(p0, p1);
         }
         tmem_st_x16(s_tmem + 16 * c, pk);
       }
+      const float sum = ((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7]));
       l_run = l_run * alpha + sum;
       if (j > 0 && __any_sync(0xffffffffu, need)) {
         // O was last written by PV_{j-1}, which completed before S_j (the
