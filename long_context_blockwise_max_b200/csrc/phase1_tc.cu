@@ -38,6 +38,7 @@ using namespace sm100;
 namespace {
 
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
+constexpr int kEmuSlot = -1;  // element pairs i with i % 4 == kEmuSlot use exp2_fma2 (-1: none)
 
 template <int D>
 struct TcCfg {
@@ -106,6 +107,30 @@ __device__ void decode_item(const HostTable& ht, int max_tiles, int item, int* h
   }
   *host = h;
   *tile = lo;
+}
+
+// 2^x for two values at once on the FMA pipe (packed f32x2), used for part
+// of the softmax so that the MUFU unit is not the only source of
+// exponentials.  x = j + f with j the nearest integer (adding 1.5 * 2^23
+// leaves j in the low mantissa bits) and f in [-0.5, 0.5]; 2^f = e^(f ln 2)
+// by its Taylor series to degree 4 (relative error below 5e-5 on that
+// interval); j is then added to the exponent field.  Inputs are clamped at
+// -125 so that the result stays a normal float.
+__device__ __forceinline__ void exp2_fma2(float x0, float x1, float& y0, float& y1) {
+  const uint64_t x = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t t = f2_add(x, f2_pack(12582912.f, 12582912.f));
+  const uint64_t r = f2_add(t, f2_pack(-12582912.f, -12582912.f));
+  const uint64_t f = f2_fma(r, f2_pack(-1.f, -1.f), x);
+  uint64_t p = f2_fma(f2_pack(9.6181291076284772e-3f, 9.6181291076284772e-3f), f,      // (ln 2)^4 / 4!
+                      f2_pack(5.5504108664821580e-2f, 5.5504108664821580e-2f));        // (ln 2)^3 / 3!
+  p = f2_fma(p, f, f2_pack(2.4022650695910071e-1f, 2.4022650695910071e-1f));          // (ln 2)^2 / 2!
+  p = f2_fma(p, f, f2_pack(6.9314718055994531e-1f, 6.9314718055994531e-1f));          // ln 2
+  p = f2_fma(p, f, f2_pack(1.f, 1.f));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -298,25 +323,23 @@ __global__ void __launch_bounds__(384, 1) phase1_tc_kernel(const __grid_constant
       tc_fence_after();
       uint32_t sr[128];
       tmem_ld_x128(s_tmem, sr);
-      // row max with 8 independent partial maxima (short dependency chains);
-      // only the diagonal tile needs the causal / ragged-end mask
+      // row max with 8 independent partial maxima (three-input max, short
+      // dependency chains); only the diagonal tile needs the causal /
+      // ragged-end mask
       float mx[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) mx[e] = -INFINITY;
-      if (j == nkv - 1) {
+      const bool diag = (j == nkv - 1);
+      if (diag) {
         const int lim = min(r, n - 1) - j * 128;   // columns <= lim are visible
 #pragma unroll
-        for (int i = 0; i < 128; ++i) {
-          const float x = (i > lim) ? -INFINITY : __uint_as_float(sr[i]);
-          sr[i] = __float_as_uint(x);
-          mx[i & 7] = fmaxf(mx[i & 7], x);
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 128; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(sr[i]));
+        for (int i = 0; i < 128; ++i)
+          if (i > lim) sr[i] = __float_as_uint(-INFINITY);
       }
-      const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+#pragma unroll
+      for (int i = 0; i < 64; ++i)
+        mx[i & 7] = fmax3(mx[i & 7], __uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]));
+      const float mt = fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(fmax3(mx[3], mx[4], mx[5]), mx[6], mx[7]));
       const float m_new = fmaxf(m_run, mt);
       const bool need = m_new > m_run + 8.f;   // lazy rescale: only when P could exceed 2^8
       float alpha = 1.f;
@@ -325,22 +348,36 @@ __global__ void __launch_bounds__(384, 1) phase1_tc_kernel(const __grid_constant
         m_run = m_new;
       }
       const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-      float sm[8];
+      const uint64_t nm2 = f2_pack(-m_use, -m_use);
+      uint64_t acc2[4];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) sm[e] = 0.f;
+      for (int e = 0; e < 4; ++e) acc2[e] = 0ull;   // two 0.0f
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float p0 = fast_exp2(__uint_as_float(sr[32 * c + 2 * i]) - m_use);
-          const float p1 = fast_exp2(__uint_as_float(sr[32 * c + 2 * i + 1]) - m_use);
-          sm[i & 7] += p0 + p1;
+          float x0, x1, p0, p1;
+          f2_unpack(f2_add(f2_pack(__uint_as_float(sr[32 * c + 2 * i]), __uint_as_float(sr[32 * c + 2 * i + 1])),
+                           nm2), x0, x1);
+          if (!diag && (i & 3) == kEmuSlot) {
+            exp2_fma2(x0, x1, p0, p1);          // FMA pipe
+          } else {
+            p0 = fast_exp2(x0);                 // MUFU
+            p1 = fast_exp2(x1);
+          }
+          acc2[i & 3] = f2_add(acc2[i & 3], f2_pack(p0, p1));
           pk[i] = pack_bf16x2(p0, p1);
         }
         tmem_st_x16(s_tmem + 16 * c, pk);
       }
-      const float sum = ((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7]));
+      float sum = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float a0, a1;
+        f2_unpack(acc2[e], a0, a1);
+        sum += a0 + a1;
+      }
       l_run = l_run * alpha + sum;
       if (j > 0 && __any_sync(0xffffffffu, need)) {
         // O was last written by PV_{j-1}, which completed before S_j (the
