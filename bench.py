@@ -170,19 +170,28 @@ def attn_flops(w, star=False):
     return float(sum(4.0 * w.d * w.hq * n * (n + 1) / 2.0 for n in host_lengths(w, star)))
 
 
-def sync_all(dist_on):
-    torch.cuda.synchronize()
+def sync_all(dist_on, device="cuda"):
+    """Barrier across ranks with the device drained on both sides."""
+    if str(device).startswith("cuda"):
+        torch.cuda.synchronize()
     if dist_on:
         torch.distributed.barrier()
-        torch.cuda.synchronize()
+        if str(device).startswith("cuda"):
+            torch.cuda.synchronize()
 
 
-def max_over_ranks(x: float, dist_on: bool) -> float:
+def max_over_ranks(x: float, dist_on: bool, device="cuda") -> float:
+    """The largest of the ranks' values (every rank gets it)."""
     if not dist_on:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, world: int, ms_per_step: float) -> float:
+    """Units processed by all ranks per second, timed by the slowest rank."""
+    return units_per_rank * world / (ms_per_step * 1e-3)
 
 
 def run_ours(args, rank, world, local_rank, dist_on):
@@ -222,7 +231,7 @@ def run_ours(args, rank, world, local_rank, dist_on):
     p2_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_p2)
 
     flops = attn_flops(w)
-    tokens_per_s = w.L * world / (ms * 1e-3)
+    tokens_per_s = whole_job_rate(w.L, world, ms)
     peak_tf = peaks["bf16_tflops_sustained"]
     attn_tf = flops / (attn_ms * 1e-3) / 1e12
 
@@ -337,7 +346,7 @@ def run_ours(args, rank, world, local_rank, dist_on):
                    "rope_theta": w.rope_theta, "per_rank": "one independent 128K sequence",
                    "l2": "inputs larger than L2 (Q alone is 1 GiB)"},
         "clocks": clocks,
-        "e2e": {"value": round(w.L * world / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
+        "e2e": {"value": round(whole_job_rate(w.L, world, e2e_ms), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3)},
         "gpu_launches": Step.LAUNCHES * K,
         "roofline": {"bound": "tensor", "kernel": "phase-1 attention", "achieved": round(attn_tf, 1),
@@ -428,9 +437,10 @@ def run_reference(args):
 
 def run_profile_case(name, steps, warmup):
     """A single kernel family on a small workload, for ncu captures:
-    phase1-32k (Pulsar Phase 1, 32K shape), decode-128k (Phase-2 decode),
-    query-128k (Phase-2 64-token query), rope-32k (the RoPE prepass alone is
-    part of phase1-32k).  Prints one JSON line with the mean call time."""
+    phase1-32k (Pulsar Phase 1 incl. its RoPE prepass, 32K shape),
+    decode-128k / decode-16k (Phase-2 decode, 16 queries over a 128K / 16K
+    cache in 8 shards), query-128k (Phase-2 64-token query).  Prints one JSON
+    line with the mean call time."""
     from long_context_blockwise_max_b200 import pulsar as P
     dev = torch.device("cuda", 0)
     if name == "phase1-32k":
@@ -444,13 +454,16 @@ def run_profile_case(name, steps, warmup):
         def call():
             P.pulsar_phase1_encode(q, k, v, w.rope_theta, w.block, w.sink, w.chunk, w.k_chunks, sel, o=o, lse=lse,
                                    k_ret=kr, v_ret=vr, ws=ws)
-    elif name == "decode-128k":
+    elif name in ("decode-128k", "decode-16k"):
         w = DECODE
-        q, kc, vc = w.decode_inputs(device=dev)
-        o, lse, _, _, ws = P.star_phase2_attend(q, kc, vc, w.decode_shards, w.decode_T, w.rope_theta)
+        T = w.decode_T if name == "decode-128k" else 16384
+        q = workloads.normal((w.decode_batch, 1, w.hq, w.d), workloads.SEED_QUERY, w.dtype, dev)
+        kc = workloads.normal((w.decode_batch, T, w.hkv, w.d), workloads.SEED_KC, w.dtype, dev)
+        vc = workloads.normal((w.decode_batch, T, w.hkv, w.d), workloads.SEED_VC, w.dtype, dev)
+        o, lse, _, _, ws = P.star_phase2_attend(q, kc, vc, w.decode_shards, T, w.rope_theta)
 
         def call():
-            P.star_phase2_attend(q, kc, vc, w.decode_shards, w.decode_T, w.rope_theta, o=o, lse=lse, ws=ws)
+            P.star_phase2_attend(q, kc, vc, w.decode_shards, T, w.rope_theta, o=o, lse=lse, ws=ws)
     elif name == "query-128k":
         w = WORKLOAD
         q = w.query(device=dev)

@@ -280,29 +280,201 @@ __global__ void __launch_bounds__(kWarps * 32) phase2_mma_kernel(Phase2Args a, i
   }
 }
 
+// Variant for many query rows per kv head (a multi-token query): the four
+// warps own four different groups of 8 rows and share every K / V tile,
+// which the whole CTA streams through one 3-stage cp.async ring, so a
+// unit's keys are read once per 32 rows instead of once per 8 rows.
+template <int D>
+__global__ void __launch_bounds__(kWarps * 32) phase2_mma_rows_kernel(Phase2Args a, int row_blocks) {
+  using C = P2Cfg<D>;
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int units = a.n_shards * a.n_split;
+  const int rb = blockIdx.x % row_blocks;
+  const int bu = blockIdx.x / row_blocks;
+  const int b = bu / units, u = bu % units;
+  const int kvh = blockIdx.y;
+  const int g = a.hq / a.hkv;
+  const int R = a.Tq * g;
+  const int rg = rb * kWarps + warp;   // this warp's group of 8 rows
+
+  int64_t k0, k1;
+  {
+    const int64_t step = (a.T + a.n_shards - 1) / a.n_shards;
+    const int sh = u / a.n_split, sp = u % a.n_split;
+    const int64_t lo = min((int64_t)sh * step, a.T), hi = min((int64_t)(sh + 1) * step, a.T);
+    const int64_t len = (hi - lo + a.n_split - 1) / a.n_split;
+    k0 = min(lo + (int64_t)sp * len, hi);
+    k1 = min(lo + (int64_t)(sp + 1) * len, hi);
+  }
+  const int qi = lane >> 2, qc = (lane & 3) * 2;
+  const int rr = rg * 8 + qi;
+  const bool row_ok = rr < R;
+  const int t_row = row_ok ? rr / g : 0;
+  const int head = kvh * g + (row_ok ? rr % g : 0);
+  uint32_t qa[D / 16][4];
+  {
+    const float* qp = a.qr + (((int64_t)b * a.Tq + t_row) * a.hq + head) * D;
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      float x[4];
+      x[0] = row_ok ? qp[16 * ks + qc] : 0.f;
+      x[1] = row_ok ? qp[16 * ks + qc + 1] : 0.f;
+      x[2] = row_ok ? qp[16 * ks + qc + 8] : 0.f;
+      x[3] = row_ok ? qp[16 * ks + qc + 9] : 0.f;
+      float h[4], l[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        h[e] = __bfloat162float(__float2bfloat16_rn(x[e]));
+        l[e] = x[e] - h[e];
+      }
+      qa[ks][0] = pack_bf16(h[0], h[1]);
+      qa[ks][1] = pack_bf16(l[0], l[1]);
+      qa[ks][2] = pack_bf16(h[2], h[3]);
+      qa[ks][3] = pack_bf16(l[2], l[3]);
+    }
+  }
+  const int n_tiles = static_cast<int>((k1 - k0 + kKT - 1) / kKT);
+  const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+  const __nv_bfloat16* Kg = static_cast<const __nv_bfloat16*>(a.k_ret);
+  const __nv_bfloat16* Vg = static_cast<const __nv_bfloat16*>(a.v_ret);
+  const int64_t key_stride = (int64_t)a.hkv * D;
+  const int64_t base_off = ((int64_t)b * a.T) * key_stride + (int64_t)kvh * D;
+  auto issue = [&](int it) {
+    if (it < n_tiles) {
+      const int64_t key0 = k0 + (int64_t)it * kKT;
+      const uint32_t sbase = base + (it % kStages) * C::STAGE;
+#pragma unroll
+      for (int e = 0; e < (kKT * C::CH) / (kWarps * 32); ++e) {
+        const int idx = e * kWarps * 32 + threadIdx.x;
+        const int key = idx / C::CH, ch = idx % C::CH;
+        const int64_t kg = key0 + key;
+        const bool valid = kg < k1;
+        const int64_t off = base_off + (valid ? kg : k0) * key_stride + ch * 8;
+        cp_async16(sbase + swz<D>(key, ch), Kg + off, valid);
+        cp_async16(sbase + C::TILE + swz<D>(key, ch), Vg + off, valid);
+      }
+    }
+    cp_async_commit();
+  };
+  float o[D / 8][4];
+#pragma unroll
+  for (int j = 0; j < D / 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+  float m_run = -INFINITY, l_run = 0.f;
+#pragma unroll
+  for (int s = 0; s < kStages - 1; ++s) issue(s);
+  for (int it = 0; it < n_tiles; ++it) {
+    issue(it + kStages - 1);
+    cp_async_wait<kStages - 1>();
+    __syncthreads();
+    const uint32_t sK = base + (it % kStages) * C::STAGE;
+    const uint32_t sV = sK + C::TILE;
+    const int64_t key0 = k0 + (int64_t)it * kKT;
+    float s[4][4];
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+#pragma unroll
+      for (int kk = 0; kk < D / 32; ++kk) {
+        uint32_t b0, b1, b2, b3;
+        const int key = nt * 8 + (lane & 7);
+        const int ch = kk * 4 + (lane >> 3);
+        ldsm_x4(sK + swz<D>(key, ch), b0, b1, b2, b3);
+        mma_bf16(s[nt], qa[2 * kk][0], qa[2 * kk][1], qa[2 * kk][2], qa[2 * kk][3], b0, b1);
+        mma_bf16(s[nt], qa[2 * kk + 1][0], qa[2 * kk + 1][1], qa[2 * kk + 1][2], qa[2 * kk + 1][3], b2, b3);
+      }
+    }
+    float sv[4][2];
+    float mt = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int64_t kg = key0 + nt * 8 + qc + e;
+        const float x = (kg < k1) ? s[nt][e] + s[nt][e + 2] : -INFINITY;
+        sv[nt][e] = x;
+        mt = fmaxf(mt, x);
+      }
+    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
+    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
+    const float m_new = fmaxf(m_run, mt);
+    const float alpha = fast_exp2(m_run - m_new);
+    m_run = m_new;
+    l_run *= alpha;
+#pragma unroll
+    for (int j = 0; j < D / 8; ++j) {
+      o[j][0] *= alpha;
+      o[j][1] *= alpha;
+    }
+    uint32_t pa_[4];
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+      const float p0 = fast_exp2(sv[nt][0] - m_new), p1 = fast_exp2(sv[nt][1] - m_new);
+      l_run += p0 + p1;
+      pa_[nt] = pack_bf16(p0, p1);
+    }
+#pragma unroll
+    for (int k2 = 0; k2 < 2; ++k2) {
+#pragma unroll
+      for (int cj = 0; cj < D / 16; ++cj) {
+        uint32_t b0, b1, b2, b3;
+        const int mtx = lane >> 3;
+        const int key = k2 * 16 + (mtx & 1) * 8 + (lane & 7);
+        const int ch = cj * 2 + (mtx >> 1);
+        ldsm_x4_t(sV + swz<D>(key, ch), b0, b1, b2, b3);
+        mma_bf16(o[2 * cj], pa_[2 * k2], 0u, pa_[2 * k2 + 1], 0u, b0, b1);
+        mma_bf16(o[2 * cj + 1], pa_[2 * k2], 0u, pa_[2 * k2 + 1], 0u, b2, b3);
+      }
+    }
+    __syncthreads();   // the stage is refilled by the next issue
+  }
+  cp_async_wait<0>();
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+  if (!row_ok) return;
+  const int64_t orow = (((int64_t)b * units + u) * a.Tq + t_row) * a.hq + head;
+  const bool empty = (m_run == -INFINITY);
+  const float inv = empty ? 0.f : 1.f / l_run;
+  float* dst = a.unit_o + orow * D;
+#pragma unroll
+  for (int j = 0; j < D / 8; ++j)
+    *reinterpret_cast<float2*>(dst + 8 * j + qc) = make_float2(o[j][0] * inv, o[j][1] * inv);
+  if ((lane & 3) == 0) a.unit_lse[orow] = empty ? -INFINITY : (m_run + __log2f(l_run)) * kLn2f;
+}
+
+template <int D>
+int launch_d(const Phase2Args& a, cudaStream_t s) {
+  const int g = a.hq / a.hkv;
+  const int R = a.Tq * g;
+  const int units = a.n_shards * a.n_split;
+  if (R <= 8) {
+    // a few rows per kv head (decode): the 4 warps split the keys
+    const int64_t gx = (int64_t)a.B * units;
+    if (gx <= 0) return PA_OK;
+    const int sm = P2Cfg<D>::SMEM;
+    if (cudaFuncSetAttribute(phase2_mma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm) !=
+        cudaSuccess)
+      return PA_ERR_CUDA;
+    phase2_mma_kernel<D><<<dim3(static_cast<unsigned>(gx), a.hkv), kWarps * 32, sm, s>>>(a, 1);
+  } else {
+    // many rows per kv head: the 4 warps split the rows and share K / V
+    const int row_blocks = (R + 8 * kWarps - 1) / (8 * kWarps);
+    const int64_t gx = (int64_t)a.B * units * row_blocks;
+    if (gx <= 0) return PA_OK;
+    const int sm = kStages * P2Cfg<D>::STAGE;
+    if (cudaFuncSetAttribute(phase2_mma_rows_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm) !=
+        cudaSuccess)
+      return PA_ERR_CUDA;
+    phase2_mma_rows_kernel<D><<<dim3(static_cast<unsigned>(gx), a.hkv), kWarps * 32, sm, s>>>(a, row_blocks);
+  }
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
 }  // namespace
 
 int launch_phase2_mma(const Phase2Args& a, cudaStream_t s) {
-  const int g = a.hq / a.hkv;
-  const int row_groups = (a.Tq * g + 7) / 8;
-  const int units = a.n_shards * a.n_split;
-  const int64_t gx = (int64_t)a.B * units * row_groups;
-  if (gx <= 0) return PA_OK;
-  const dim3 grid(static_cast<unsigned>(gx), a.hkv);
-  if (a.d == 128) {
-    const int sm = P2Cfg<128>::SMEM;
-    if (cudaFuncSetAttribute(phase2_mma_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm) !=
-        cudaSuccess)
-      return PA_ERR_CUDA;
-    phase2_mma_kernel<128><<<grid, kWarps * 32, sm, s>>>(a, row_groups);
-  } else {
-    const int sm = P2Cfg<64>::SMEM;
-    if (cudaFuncSetAttribute(phase2_mma_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm) !=
-        cudaSuccess)
-      return PA_ERR_CUDA;
-    phase2_mma_kernel<64><<<grid, kWarps * 32, sm, s>>>(a, row_groups);
-  }
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  return a.d == 128 ? launch_d<128>(a, s) : launch_d<64>(a, s);
 }
 
 }  // namespace pa
