@@ -6,6 +6,7 @@
 #include <cstring>
 
 #include "pa_internal.h"
+#include "../../include/pulsar_testing.h"
 
 using namespace pa;
 
@@ -60,7 +61,7 @@ int phase1_common(const void* q, const void* k, const void* v, int dtype, int64_
                   int32_t hkv, int32_t d, double rope_theta, int32_t block, int32_t sink,
                   int32_t chunk, int32_t k_chunks, const int32_t* sel, int star, void* o,
                   float* lse_opt, void* k_ret, void* v_ret, void* ws, size_t ws_bytes,
-                  cudaStream_t s) {
+                  cudaStream_t s, uint64_t wait_limit_ns = 1000000000ull, int stall = 0) {
   int rc = check_heads(hq, hkv, d, dtype);
   if (rc) return rc;
   if (!q || !k || !v || !o || !k_ret || !v_ret) return PA_ERR_INVALID;
@@ -117,6 +118,8 @@ int phase1_common(const void* q, const void* k, const void* v, int dtype, int64_
   off += align_up(qk_elem * (size_t)L * hq * d);
   a.kr = nullptr;
   if (dtype == PA_BF16) a.kr = w + off;
+  a.wait_limit_ns = wait_limit_ns;
+  a.stall = stall;
   return launch_phase1(a, s);
 }
 
@@ -277,6 +280,17 @@ int star_phase2_attend(const void* q, int dtype, int32_t B, int32_t Tq, int64_t 
   a.unit_lse = reinterpret_cast<float*>(w + off);
   if (B == 0 || Tq == 0) return PA_OK;
   return launch_phase2(a, s);
+}
+
+int pa_testing_phase1_stall(const void* q, const void* k, const void* v, int64_t L, int32_t hq,
+                            int32_t hkv, int32_t d, int32_t block, void* o, void* k_ret,
+                            void* v_ret, void* ws, size_t ws_bytes, int32_t wait_limit_us,
+                            void* stream) {
+  if (wait_limit_us <= 0 || wait_limit_us > 10000000) return PA_ERR_INVALID;
+  if (hkv <= 0 || hq % hkv != 0 || (hq / hkv) % 2 != 0) return PA_ERR_UNSUPPORTED;   // tensor-core path only
+  return phase1_common(q, k, v, PA_BF16, L, hq, hkv, d, 10000.0, block, 0, 16, 0, nullptr, 1, o,
+                       nullptr, k_ret, v_ret, ws, ws_bytes, static_cast<cudaStream_t>(stream),
+                       static_cast<uint64_t>(wait_limit_us) * 1000ull, 1);
 }
 
 }  // extern "C"

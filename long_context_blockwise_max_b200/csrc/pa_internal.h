@@ -62,6 +62,9 @@ struct Phase1Args {
   void* qr;                     // [L][hq][d] rotated, scaled Q (fp16 or fp32)
   void* kr;                     // [L][hkv][d] rotated K in QK type (fp16) or == k_ret (fp32)
   DeviceStatus* status;
+  // bounded-wait limit of the tensor-core kernel and a test-only stall
+  uint64_t wait_limit_ns = 1000000000ull;
+  int stall = 0;
 };
 bool phase1_tc_supported(const Phase1Args& a);
 int launch_phase1_tc(const Phase1Args& a, cudaStream_t s);

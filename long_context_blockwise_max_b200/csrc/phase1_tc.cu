@@ -23,8 +23,8 @@
 // PA_ERR_TIMEOUT in the status block, drains its copies and MMAs, frees
 // TMEM and returns.
 //
-// Scheduling: one CTA per (host, row tile, kv head, head pair), ordered so
-// that the tiles with the most key tiles (deepest in their host) start first.
+// Scheduling: one CTA per (host, kv head, row tile, head pair), host-major
+// so that concurrent CTAs share one host's K / V in L2 (see decode_item).
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -37,7 +37,6 @@ using namespace sm100;
 
 namespace {
 
-constexpr uint64_t kWaitLimitNs = 1000000000ull;
 constexpr int kEmuSlot = -1;  // element pairs i with i % 4 == kEmuSlot use exp2_fma2 (-1: none)
 
 template <int D>
@@ -62,7 +61,7 @@ struct TcBars {
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
-  int host, tile;
+  int host, tile, kvh, pair;
 };
 
 struct TcParams {
@@ -73,40 +72,33 @@ struct TcParams {
   int hq, hkv, pairs;   // pairs = (hq / hkv) / 2 head pairs per kv head
   int max_tiles;
   DeviceStatus* status;
+  uint64_t wait_ns;   // limit of every bounded wait
+  int stall;          // test only: the Q barrier expects 16 bytes more than are copied
 };
 
 __device__ __forceinline__ int host_tiles(const HostTable& ht, int i) {
   return ht.tile_off[i + 1] - ht.tile_off[i];
 }
 
-// Number of (host, tile) items whose tile index within its host is >= t.
-__device__ int items_from_depth(const HostTable& ht, int t) {
-  int s = 0;
-  for (int i = 0; i < ht.n_hosts; ++i) {
-    const int x = host_tiles(ht, i) - t;
-    s += x > 0 ? x : 0;
+// Work order: hosts from the longest to the shortest (host lengths never
+// decrease with the host index), then kv head, then row tile from the
+// deepest (most key tiles) to the shallowest, then head pair.  CTAs that run
+// at the same time therefore share one host's K / V for one kv head, which
+// stays in L2, and the shortest tiles come last.
+__device__ void decode_item(const HostTable& ht, int hkv, int pairs, int idx, int* host, int* kvh,
+                            int* tile, int* pair) {
+  int h = ht.n_hosts - 1;
+  for (; h > 0; --h) {
+    const int cnt = host_tiles(ht, h) * hkv * pairs;
+    if (idx < cnt) break;
+    idx -= cnt;
   }
-  return s;
-}
-
-// Work order: deepest tiles (most key tiles) first; within a depth, hosts in
-// ascending order.
-__device__ void decode_item(const HostTable& ht, int max_tiles, int item, int* host, int* tile) {
-  int lo = 0, hi = max_tiles - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (items_from_depth(ht, mid) > item) lo = mid; else hi = mid - 1;
-  }
-  int idx = item - items_from_depth(ht, lo + 1);
-  int h = 0;
-  for (int i = 0; i < ht.n_hosts; ++i) {
-    if (host_tiles(ht, i) > lo) {
-      if (idx == 0) { h = i; break; }
-      --idx;
-    }
-  }
+  const int nt = host_tiles(ht, h);
   *host = h;
-  *tile = lo;
+  *kvh = idx / (nt * pairs);
+  const int rem = idx % (nt * pairs);
+  *tile = nt - 1 - rem / pairs;
+  *pair = rem % pairs;
 }
 
 // 2^x for two values at once on the FMA pipe (packed f32x2), used for part
@@ -151,16 +143,14 @@ __global__ void __launch_bounds__(384, 1) phase1_tc_kernel(const __grid_constant
   uint8_t* sK = smem + C::OFF_K;
   uint8_t* sV = smem + C::OFF_V;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int hp_count = p.hkv * p.pairs;
-  const int item = blockIdx.x / hp_count, hp = blockIdx.x % hp_count;
-  const int kvh = hp / p.pairs, pair = hp % p.pairs;
-  const int h0 = kvh * (2 * p.pairs) + 2 * pair;
 
   if (threadIdx.x == 0) {
-    int host, tile;
-    decode_item(p.ht, p.max_tiles, item, &host, &tile);
+    int host, kvh_, tile, pair_;
+    decode_item(p.ht, p.hkv, p.pairs, blockIdx.x, &host, &kvh_, &tile, &pair_);
     bars->host = host;
     bars->tile = tile;
+    bars->kvh = kvh_;
+    bars->pair = pair_;
     mbar_init(&bars->q_full, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars->k_full[s], 1);
@@ -186,6 +176,8 @@ __global__ void __launch_bounds__(384, 1) phase1_tc_kernel(const __grid_constant
   volatile int* abort = &bars->abort;
   const volatile int* gabort = &p.status->code;   // set by any CTA that gave up
   const int host = bars->host, tile = bars->tile;
+  const int kvh = bars->kvh;
+  const int h0 = kvh * (2 * p.pairs) + 2 * bars->pair;
   const int64_t row0 = p.ht.row_off[host];
   const int n = static_cast<int>(p.ht.row_off[host + 1] - row0);
   const int r0 = tile * 128;
@@ -202,7 +194,7 @@ __global__ void __launch_bounds__(384, 1) phase1_tc_kernel(const __grid_constant
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       auto pos_of = [&](int r) -> int { return p.rowpos[row0 + (r < n ? r : 0)]; };
-      mbar_arrive_expect_tx(&bars->q_full, 2 * C::TILE_BYTES);
+      mbar_arrive_expect_tx(&bars->q_full, 2 * C::TILE_BYTES + (p.stall ? 16 : 0));
       for (int grp = 0; grp < 8; ++grp) {
         const int pq = pos_of(r0 + 16 * grp);
         for (int t = 0; t < 2; ++t)
@@ -216,14 +208,14 @@ __global__ void __launch_bounds__(384, 1) phase1_tc_kernel(const __grid_constant
         const uint32_t ph = (j >> 1) & 1;
         int pk[8];
         for (int grp = 0; grp < 8; ++grp) pk[grp] = pos_of(j * 128 + 16 * grp);
-        if (!mbar_wait(&bars->k_empty[st], ph ^ 1, abort, kWaitLimitNs, gabort)) { fail(1); break; }
+        if (!mbar_wait(&bars->k_empty[st], ph ^ 1, abort, p.wait_ns, gabort)) { fail(1); break; }
         mbar_arrive_expect_tx(&bars->k_full[st], C::TILE_BYTES);
         for (int grp = 0; grp < 8; ++grp)
           for (int kb = 0; kb < C::NKB; ++kb)
             tma_load_3d(sK + st * C::TILE_BYTES + kb * C::KB_BYTES + grp * 2048, &tmK, &bars->k_full[st],
                         kb * 64, kvh, pk[grp]);
         ++armed_k[st];
-        if (!mbar_wait(&bars->v_empty[st], ph ^ 1, abort, kWaitLimitNs, gabort)) { fail(2); break; }
+        if (!mbar_wait(&bars->v_empty[st], ph ^ 1, abort, p.wait_ns, gabort)) { fail(2); break; }
         mbar_arrive_expect_tx(&bars->v_full[st], C::TILE_BYTES);
         for (int grp = 0; grp < 8; ++grp)
           for (int kb = 0; kb < C::NKB; ++kb)
@@ -233,10 +225,10 @@ __global__ void __launch_bounds__(384, 1) phase1_tc_kernel(const __grid_constant
       }
       // Drain: every copy this thread started has landed before the CTA ends.
       int zero = 0;
-      mbar_wait(&bars->q_full, 0, &zero, kWaitLimitNs);
+      mbar_wait(&bars->q_full, 0, &zero, p.wait_ns);
       for (int s = 0; s < 2; ++s) {
-        if (armed_k[s]) mbar_wait(&bars->k_full[s], (armed_k[s] - 1) & 1, &zero, kWaitLimitNs);
-        if (armed_v[s]) mbar_wait(&bars->v_full[s], (armed_v[s] - 1) & 1, &zero, kWaitLimitNs);
+        if (armed_k[s]) mbar_wait(&bars->k_full[s], (armed_k[s] - 1) & 1, &zero, p.wait_ns);
+        if (armed_v[s]) mbar_wait(&bars->v_full[s], (armed_v[s] - 1) & 1, &zero, p.wait_ns);
       }
     }
   } else if (warp == 1) {
@@ -262,7 +254,7 @@ __global__ void __launch_bounds__(384, 1) phase1_tc_kernel(const __grid_constant
           mma_ts(d_tmem, tmem + t * 256 + ks * 8, b, C::IDESC_PV, (acc | ks) != 0);
         }
       };
-      bool ok = mbar_wait(&bars->q_full, 0, abort, kWaitLimitNs, gabort);
+      bool ok = mbar_wait(&bars->q_full, 0, abort, p.wait_ns, gabort);
       if (!ok) fail(3);
       for (int j = 0; ok && j < nkv; ++j) {
         const int st = j & 1;
@@ -270,7 +262,7 @@ __global__ void __launch_bounds__(384, 1) phase1_tc_kernel(const __grid_constant
         const int st1 = (j + 1) & 1;
         const uint32_t ph1 = ((j + 1) >> 1) & 1;
         if (j == 0) {
-          if (!mbar_wait(&bars->k_full[0], 0, abort, kWaitLimitNs, gabort)) { fail(4); break; }
+          if (!mbar_wait(&bars->k_full[0], 0, abort, p.wait_ns, gabort)) { fail(4); break; }
           tc_fence_after();
           qk(0, 0);
           mma_commit(&bars->s_full[0]);
@@ -279,19 +271,19 @@ __global__ void __launch_bounds__(384, 1) phase1_tc_kernel(const __grid_constant
           mma_commit(&bars->k_empty[0]);
         }
         // head 0: O0 += P0 V_j, then S0 = Q0 K_{j+1}
-        if (!mbar_wait(&bars->p_full[0], j & 1, abort, kWaitLimitNs, gabort)) { fail(5); break; }
-        if (!mbar_wait(&bars->v_full[st], ph, abort, kWaitLimitNs, gabort)) { fail(6); break; }
+        if (!mbar_wait(&bars->p_full[0], j & 1, abort, p.wait_ns, gabort)) { fail(5); break; }
+        if (!mbar_wait(&bars->v_full[st], ph, abort, p.wait_ns, gabort)) { fail(6); break; }
         tc_fence_after();
         pv(0, st, j > 0);
         if (j == nkv - 1) mma_commit(&bars->o_final[0]);
         if (j + 1 < nkv) {
-          if (!mbar_wait(&bars->k_full[st1], ph1, abort, kWaitLimitNs, gabort)) { fail(7); break; }
+          if (!mbar_wait(&bars->k_full[st1], ph1, abort, p.wait_ns, gabort)) { fail(7); break; }
           tc_fence_after();
           qk(0, st1);
           mma_commit(&bars->s_full[0]);
         }
         // head 1: O1 += P1 V_j, then S1 = Q1 K_{j+1}
-        if (!mbar_wait(&bars->p_full[1], j & 1, abort, kWaitLimitNs, gabort)) { fail(8); break; }
+        if (!mbar_wait(&bars->p_full[1], j & 1, abort, p.wait_ns, gabort)) { fail(8); break; }
         tc_fence_after();
         pv(1, st, j > 0);
         if (j == nkv - 1) mma_commit(&bars->o_final[1]);
@@ -305,7 +297,7 @@ __global__ void __launch_bounds__(384, 1) phase1_tc_kernel(const __grid_constant
       // Drain: all MMAs issued by this thread complete before TMEM is freed.
       int zero = 0;
       mma_commit(&bars->drain);
-      mbar_wait(&bars->drain, 0, &zero, kWaitLimitNs);
+      mbar_wait(&bars->drain, 0, &zero, p.wait_ns);
     }
   } else if (warp >= 4) {
     // -------------------------------------------------------------- softmax
@@ -319,7 +311,7 @@ __global__ void __launch_bounds__(384, 1) phase1_tc_kernel(const __grid_constant
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
-      if (!mbar_wait(&bars->s_full[t], j & 1, abort, kWaitLimitNs, gabort)) { fail(9); ok = false; break; }
+      if (!mbar_wait(&bars->s_full[t], j & 1, abort, p.wait_ns, gabort)) { fail(9); ok = false; break; }
       tc_fence_after();
       uint32_t sr[128];
       tmem_ld_x128(s_tmem, sr);
@@ -395,7 +387,7 @@ __global__ void __launch_bounds__(384, 1) phase1_tc_kernel(const __grid_constant
       tc_fence_before();
       mbar_arrive(&bars->p_full[t]);
     }
-    if (ok && mbar_wait(&bars->o_final[t], 0, abort, kWaitLimitNs, gabort)) {
+    if (ok && mbar_wait(&bars->o_final[t], 0, abort, p.wait_ns, gabort)) {
       tc_fence_after();
       const float inv = 1.f / l_run;
       __nv_bfloat16* dst = p.o + ((row0 + r) * p.hq + head) * static_cast<int64_t>(D);
@@ -474,6 +466,8 @@ int launch_tc(const Phase1Args& a, cudaStream_t s) {
   for (int i = 0; i < a.ht.n_hosts; ++i)
     p.max_tiles = std::max(p.max_tiles, a.ht.tile_off[i + 1] - a.ht.tile_off[i]);
   p.status = a.status;
+  p.wait_ns = a.wait_limit_ns;
+  p.stall = a.stall;
   const int64_t items = a.ht.tile_off[a.ht.n_hosts];
   const int64_t grid = items * a.hkv * p.pairs;
   if (grid <= 0) return PA_OK;

@@ -60,6 +60,8 @@ def _load() -> ctypes.CDLL:
         "star_phase2_attend": (ctypes.c_int, [P, ctypes.c_int, I32, I32, I64, D, P, P, I64, I32, I32, I32,
                                               I32, P, P, P, P, P, SZ, P]),
     }
+    # test hook (include/pulsar_testing.h)
+    sig["pa_testing_phase1_stall"] = (ctypes.c_int, [P, P, P, I64, I32, I32, I32, I32, P, P, P, P, SZ, I32, P])
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
         fn.restype, fn.argtypes = res, args
@@ -253,3 +255,19 @@ def star_phase2_attend(q, k_ret, v_ret, n_shards, q_pos0=0, rope_theta=0.0, o=No
                                  _ptr(ws), ws.numel() * ws.element_size(), _stream())
     _check(rc, "star_phase2_attend")
     return o, lse, part_o, part_lse, ws
+
+
+def pa_testing_phase1_stall(q, k, v, block, wait_limit_us):
+    """Test hook: Star Phase 1 through the tensor-core kernel with one
+    unsatisfiable barrier and waits limited to ``wait_limit_us``; the
+    workspace status then reads PA_ERR_TIMEOUT.  Returns the workspace."""
+    _dev(q, k, v)
+    L, hq, d = q.shape
+    hkv = k.shape[1]
+    row_off = pa_phase1_layout(L, block, 0, 0, True)
+    o, _, k_ret, v_ret = _phase1_outputs(q, k, row_off[-1], None, None, None, None, False)
+    ws = _workspace(pa_phase1_workspace_size(L, hq, hkv, d, PA_BF16, block, 0, 0, True), q.device)
+    rc = _lib.pa_testing_phase1_stall(_ptr(q), _ptr(k), _ptr(v), L, hq, hkv, d, block, _ptr(o), _ptr(k_ret),
+                                      _ptr(v_ret), _ptr(ws), ws.numel(), int(wait_limit_us), _stream())
+    _check(rc, "pa_testing_phase1_stall")
+    return ws

@@ -94,6 +94,22 @@ def test_bf16_small_all_rows(P, case, star):
     _parity(P, q, k, v, theta, block, sink, chunk, kc, sel, star)
 
 
+def test_bf16_sixty_four_hosts_and_full_sink(P):
+    # the largest host count (64 blocks of 128) with a 16-token sink, and a
+    # sink as long as a block
+    for L, block, sink, chunk, kc in ((64 * 128, 128, 16, 16, 1), (3 * 128, 128, 128, 16, 2)):
+        q, k, v = _inputs(L, 4, 2, 64, torch.bfloat16, seed=L + sink)
+        n = L // block
+        rng = np.random.default_rng(n)
+        sel = np.sort(np.stack([rng.choice(block // chunk, kc, replace=False) for _ in range(n)]), axis=1)
+        _parity(P, q, k, v, 10000.0, block, sink, chunk, kc, sel, False)
+
+
+def test_star_single_block(P):
+    q, k, v = _inputs(384, 8, 2, 128, torch.bfloat16, seed=31)
+    _parity(P, q, k, v, 500000.0, 384, 0, 16, 0, np.zeros((1, 0), dtype=np.int64), True)
+
+
 def test_bf16_zero_sink_zero_budget(P):
     L, block = 3 * 256, 256
     q, k, v = _inputs(L, 4, 2, 128, torch.bfloat16, seed=5)

@@ -51,6 +51,8 @@ def test_tiny_fp32_full(P):
     (3, 1, 999, 4, 32, 8, 128, 500000.0),      # decode rows, ragged cache
     (2, 7, 10, 16, 4, 4, 64, 0.0),             # more shards than keys: empty shards, no RoPE
     (1, 3, 0, 2, 4, 2, 64, 10000.0),           # empty cache: O = 0, lse = -inf
+    (2, 20, 700, 3, 8, 2, 64, 10000.0),        # d = 64, 80 rows per kv head (row-split kernel)
+    (1, 2, 5000, 4096, 4, 1, 128, 500000.0),   # the largest shard count: most shards of 1-2 keys
 ])
 def test_bf16_small_full(P, case):
     B, Tq, T, S, hq, hkv, d, theta = case
