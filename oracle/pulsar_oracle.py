@@ -133,6 +133,70 @@ def select_summaries(ids: np.ndarray, block: int, chunk: int, k: int, vocab: int
 
 
 # ----------------------------------------------------------------------------
+# Alternative summary scorers ([P] §3.1 and Table 1: the other statistical
+# scores and the non-statistical baselines; [P] §2.1 contrasts max with mean)
+# ----------------------------------------------------------------------------
+
+FIXED_BITS = 24
+
+
+def idf_fixed_table(n_blocks: int) -> list:
+    """q[df] = nearest integer to ln(N / df) * 2^24 for df = 1..N (q[0] = 0).
+    Mean-IDF ranks chunks by a sum of IDF values; the decision is taken on
+    this fixed-point scale (the precision the CUDA path uses), so that equal
+    multisets of df give equal sums whatever the summation order."""
+    return [0] + [int(round(math.log(float(n_blocks) / df) * (1 << FIXED_BITS)))
+                  for df in range(1, n_blocks + 1)]
+
+
+def chunk_mean_idf(ids: np.ndarray, block: int, chunk: int, idf: np.ndarray) -> np.ndarray:
+    """Mean IDF over each chunk's tokens (exactly rounded sum / chunk),
+    float64 [N][C]."""
+    blocks = _blocks(ids, block)
+    C = block // chunk
+    out = np.empty((len(blocks), C), dtype=np.float64)
+    for j, blk in enumerate(blocks):
+        for c in range(C):
+            out[j, c] = math.fsum(idf[t] for t in blk[c * chunk:(c + 1) * chunk].tolist()) / chunk
+    return out
+
+
+def chunk_mean_idf_fixed(ids: np.ndarray, block: int, chunk: int, df: np.ndarray) -> np.ndarray:
+    """Sum over each chunk's tokens of q[df(t)] (see idf_fixed_table),
+    int64 [N * C] in sequence order."""
+    blocks = _blocks(ids, block)
+    q = idf_fixed_table(len(blocks))
+    C = block // chunk
+    out = np.empty(len(blocks) * C, dtype=np.int64)
+    for j, blk in enumerate(blocks):
+        for c in range(C):
+            out[j * C + c] = sum(q[int(df[t])] for t in blk[c * chunk:(c + 1) * chunk].tolist())
+    return out
+
+
+def select_evenly_spaced(n_blocks: int, block: int, chunk: int, k: int) -> np.ndarray:
+    """Evenly spaced chunks, the same in every block: chunk floor(m * C / k)
+    for m = 0..k-1 (the non-statistical baseline of [P] §3.1)."""
+    C = block // chunk
+    row = [(m * C) // k for m in range(k)]
+    return np.tile(np.array(row, dtype=np.int64), (n_blocks, 1)).reshape(n_blocks, k)
+
+
+def select_summaries_mean_idf(ids: np.ndarray, block: int, chunk: int, k: int, vocab: int):
+    """Top-k chunks per block by mean IDF (on the fixed-point scale of
+    idf_fixed_table), kept in original order; ties go to the lower index."""
+    n_blocks = len(ids) // block
+    C = block // chunk
+    df = document_frequency(ids, block, vocab)
+    sc = chunk_mean_idf_fixed(ids, block, chunk, df).reshape(n_blocks, C)
+    sel = np.empty((n_blocks, k), dtype=np.int64)
+    for j in range(n_blocks):
+        order = sorted(range(C), key=lambda c: (-int(sc[j, c]), c))
+        sel[j] = sorted(order[:k])
+    return sel
+
+
+# ----------------------------------------------------------------------------
 # Phase 1: host inputs  ([PS] Fase 1; [P] §2, Figure 1; [S] key_machinery)
 # ----------------------------------------------------------------------------
 

@@ -144,3 +144,40 @@ def test_budget_and_prefix_arithmetic():
     pos = oracle.host_positions(L, b, 64, 32, sel)
     assert len(pos[3]) - b == 1600
     assert [len(p) for p in pos] == [4096, 4096 + 64 + 512, 4096 + 64 + 1024, 4096 + 1600]
+
+
+def test_mean_idf_figure2_and_fixed_scale():
+    g = json.load(open(os.path.join(GOLDEN, "figure2_toy.json")))
+    ids = np.array(g["ids"], dtype=np.int64)
+    df = oracle.document_frequency(ids, g["block"], g["vocab"])
+    idf = oracle.idf_table(df, 4)
+    vals = {"0": 0.0, "log2": math.log(2.0), "log4/4": math.log(4.0) / 4}
+    want = np.array([[vals[t] for t in row] for row in g["expected_mean_scores"]])
+    np.testing.assert_allclose(oracle.chunk_mean_idf(ids, g["block"], g["chunk"], idf), want, rtol=0, atol=1e-15)
+    assert oracle.select_summaries_mean_idf(ids, g["block"], g["chunk"], 1, g["vocab"]).tolist() == \
+        g["expected_mean_idf_selection"]
+    # the fixed-point table: q[df] ~ ln(N/df) * 2^24, q[N] = 0
+    q = oracle.idf_fixed_table(4)
+    assert q[4] == 0 and abs(q[1] - math.log(4.0) * 2 ** 24) <= 0.5 and abs(q[2] - math.log(2.0) * 2 ** 24) <= 0.5
+    fx = oracle.chunk_mean_idf_fixed(ids, g["block"], g["chunk"], df).reshape(4, 4)
+    assert (np.abs(fx / 2.0 ** 24 / g["chunk"] - want) <= 4 * 0.5 / 2 ** 24 / g["chunk"] + 1e-15).all()
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_mean_idf_brute_force(seed):
+    rng = np.random.default_rng(500 + seed)
+    block, chunk, n, vocab = 32, 4, 4, 14
+    ids = rng.integers(0, vocab, size=block * n)
+    df = oracle.document_frequency(ids, block, vocab)
+    sc = oracle.chunk_mean_idf_fixed(ids, block, chunk, df).reshape(n, block // chunk)
+    for k in (1, 3, 8):
+        sel = oracle.select_summaries_mean_idf(ids, block, chunk, k, vocab)
+        for j in range(n):
+            assert sel[j].tolist() == _brute_force_topk(sc[j].tolist(), k)
+
+
+def test_evenly_spaced_closed_form():
+    sel = oracle.select_evenly_spaced(3, 4096, 32, 16)      # 128 chunks, 16 kept: every 8th
+    assert sel.shape == (3, 16) and sel[1].tolist() == list(range(0, 128, 8))
+    assert oracle.select_evenly_spaced(1, 96, 32, 3).tolist() == [[0, 1, 2]]
+    assert oracle.select_evenly_spaced(2, 320, 32, 3).tolist() == [[0, 3, 6]] * 2
