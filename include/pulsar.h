@@ -122,6 +122,32 @@ int pulsar_select_summaries(const int32_t* ids, int64_t L, int32_t vocab, int32_
                             int32_t chunk, int32_t k_chunks, int32_t* sel, int32_t* df_opt,
                             int32_t* chunk_mindf_opt, void* ws, size_t ws_bytes, void* stream);
 
+/* Chunk scorers of pulsar_select_summaries_scored. */
+typedef enum {
+  PA_SCORE_MAX_IDF = 0,       /* the method: max IDF over the chunk (= pulsar_select_summaries) */
+  PA_SCORE_MEAN_IDF = 1,      /* mean IDF over the chunk's tokens */
+  PA_SCORE_EVENLY_SPACED = 2  /* no score: chunks floor(m * C / k), m = 0..k-1, in every block */
+} pa_score_method;
+
+/*
+ * Summary selection with another chunk scorer, for the scorer ablation of
+ * [P] §3.1 (Table 1 compares Max-IDF with other statistical scores and with
+ * non-statistical baselines; §2.1 contrasts the maximum with the mean).
+ * Same sizes, rules, outputs and tie-break as pulsar_select_summaries.
+ *  - PA_SCORE_MEAN_IDF ranks chunks by sum_t q[df(t)] with
+ *    q[df] = round(ln(N/df) * 2^24) (the mean times the chunk length, on a
+ *    fixed-point scale so that ranking is exact and order-independent);
+ *    block / chunk <= 8192 (PA_ERR_UNSUPPORTED otherwise).
+ *  - PA_SCORE_EVENLY_SPACED does not read ids (may be NULL).
+ *  chunk_score_opt  out [L / chunk] int64: the fixed-point sums (mean-IDF),
+ *                   the min df (max-IDF), not written (evenly spaced); or NULL.
+ * Workspace: pa_select_workspace_size.
+ */
+int pulsar_select_summaries_scored(const int32_t* ids, int64_t L, int32_t vocab, int32_t block,
+                                   int32_t chunk, int32_t k_chunks, int method, int32_t* sel,
+                                   int64_t* chunk_score_opt, void* ws, size_t ws_bytes,
+                                   void* stream);
+
 /*
  * Allocation-free variant of pulsar_select_summaries.  The paper has no
  * counterpart to this call: it exists for callers that cannot allocate

@@ -164,7 +164,57 @@ size_t pa_select_workspace_size(int64_t L, int32_t vocab, int32_t block, int32_t
   size_t b = kStatusBytes;
   b += align_up(sizeof(unsigned long long) * (size_t)vocab);
   b += align_up(sizeof(int32_t) * (size_t)(L / chunk));
+  b += align_up(sizeof(long long) * (size_t)(L / chunk));   // fixed-point scores (scorer variants)
   return b;
+}
+
+int pulsar_select_summaries_scored(const int32_t* ids, int64_t L, int32_t vocab, int32_t block,
+                                   int32_t chunk, int32_t k_chunks, int method, int32_t* sel,
+                                   int64_t* chunk_score_opt, void* ws, size_t ws_bytes,
+                                   void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (method != PA_SCORE_MAX_IDF && method != PA_SCORE_MEAN_IDF && method != PA_SCORE_EVENLY_SPACED)
+    return PA_ERR_INVALID;
+  if (L <= 0 || vocab <= 0 || block <= 0 || chunk <= 0) return PA_ERR_INVALID;
+  if (L % block != 0 || block % chunk != 0) return PA_ERR_INVALID;
+  if (k_chunks < 0 || k_chunks > block / chunk) return PA_ERR_INVALID;
+  if ((ids == nullptr && method != PA_SCORE_EVENLY_SPACED) || (sel == nullptr && k_chunks > 0))
+    return PA_ERR_INVALID;
+  if (L / block > kMaxBlocks) return PA_ERR_UNSUPPORTED;
+  if (method == PA_SCORE_MEAN_IDF && block / chunk > kMaxScoredChunks) return PA_ERR_UNSUPPORTED;
+  const size_t need = pa_select_workspace_size(L, vocab, block, chunk);
+  int rc = check_ws(ws, ws_bytes, need);
+  if (rc) return rc;
+  rc = clear_status(ws, s);
+  if (rc) return rc;
+  char* w = static_cast<char*>(ws);
+  SelectArgs a;
+  a.ids = ids; a.L = L; a.vocab = vocab; a.block = block; a.chunk = chunk; a.k = k_chunks;
+  a.sel = sel; a.df_out = nullptr;
+  a.status = reinterpret_cast<DeviceStatus*>(w);
+  size_t off = kStatusBytes;
+  a.mask = reinterpret_cast<unsigned long long*>(w + off);
+  off += align_up(sizeof(unsigned long long) * (size_t)vocab);
+  int32_t* mindf = reinterpret_cast<int32_t*>(w + off);
+  off += align_up(sizeof(int32_t) * (size_t)(L / chunk));
+  long long* score = chunk_score_opt ? reinterpret_cast<long long*>(chunk_score_opt)
+                                     : reinterpret_cast<long long*>(w + off);
+  if (method == PA_SCORE_MAX_IDF) {
+    a.mindf = mindf;
+    rc = launch_select(a, s);
+    if (rc == PA_OK && chunk_score_opt != nullptr) {
+      // widen the min df of every chunk into the caller's int64 array
+      rc = launch_widen_i32(mindf, score, L / chunk, s);
+    }
+    return rc;
+  }
+  FixedIdf tab;
+  const int n = (int)(L / block);
+  tab.q[0] = 0;
+  for (int df = 1; df <= kMaxBlocks; ++df)
+    tab.q[df] = df <= n ? llround(std::log((double)n / df) * (double)(1 << 24)) : 0;
+  a.mindf = mindf;
+  return launch_select_scored(a, method, tab, score, s);
 }
 
 int pulsar_select_summaries(const int32_t* ids, int64_t L, int32_t vocab, int32_t block,

@@ -32,6 +32,15 @@ struct SelectArgs {
 };
 int launch_select(const SelectArgs& a, cudaStream_t s);
 
+// q[df] = round(ln(N/df) * 2^24), df = 0..N (q[0] unused)
+struct FixedIdf {
+  long long q[kMaxBlocks + 1];
+};
+constexpr int kMaxScoredChunks = 8192;   // chunks per block for the rank-based top-k
+int launch_widen_i32(const int32_t* in, long long* out, int64_t n, cudaStream_t s);
+int launch_select_scored(const SelectArgs& a, int method, const FixedIdf& tab, long long* score,
+                         cudaStream_t s);
+
 // Host-computed RoPE frequencies omega_m = theta^(-2m/d), fp64.
 struct RopeFreqs {
   double omega[kMaxHalfDim];

@@ -141,6 +141,118 @@ __global__ void __launch_bounds__(THREADS) topk_kernel(const int32_t* __restrict
   }
 }
 
+// ---------------------------------------------------------------------------
+// Alternative scorers (Pulsar Attention page §3.1, Table 1).
+//  chunk_fixed_score_kernel: mean-IDF as the sum over the chunk's tokens of
+//    q[df] = round(ln(N/df) * 2^24) (int64, exact and order-independent).
+//  topk_rank_kernel: per block, a chunk is kept when fewer than k chunks
+//    beat it (higher score, or equal score and lower index); ordered
+//    compaction as in topk_kernel.
+//  evenly_spaced_kernel: chunk floor(m * C / k) in every block.
+// ---------------------------------------------------------------------------
+__global__ void chunk_fixed_score_kernel(const int32_t* __restrict__ ids, int64_t n_chunks,
+                                         int32_t chunk, int32_t vocab,
+                                         const unsigned long long* __restrict__ mask, FixedIdf tab,
+                                         long long* __restrict__ score) {
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t c = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; c < n_chunks;
+       c += nwarps) {
+    long long acc = 0;
+    const int32_t* tok = ids + c * chunk;
+    for (int u = lane; u < chunk; u += 32) {
+      const int t = tok[u];
+      if (t >= 0 && t < vocab) acc += tab.q[__popcll(mask[t])];
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) score[c] = acc;
+  }
+}
+
+template <int THREADS>
+__global__ void __launch_bounds__(THREADS) topk_rank_kernel(const long long* __restrict__ score,
+                                                            int32_t C, int32_t k,
+                                                            int32_t* __restrict__ sel) {
+  extern __shared__ long long sc[];
+  __shared__ int warp_tot[THREADS / 32];
+  const int j = blockIdx.x;
+  for (int c = threadIdx.x; c < C; c += THREADS) sc[c] = score[(int64_t)j * C + c];
+  __syncthreads();
+  int base_sel = 0;
+  for (int base = 0; base < C; base += THREADS) {
+    const int c = base + threadIdx.x;
+    bool take = false;
+    if (c < C) {
+      const long long v = sc[c];
+      int better = 0;
+      for (int o = 0; o < C && better < k; ++o) {
+        const long long w = sc[o];
+        better += (w > v) || (w == v && o < c);
+      }
+      take = better < k;
+    }
+    int tot;
+    const int pos = base_sel + block_exclusive_count<THREADS>(take, warp_tot, &tot);
+    if (take) sel[(int64_t)j * k + pos] = c;
+    base_sel += tot;
+  }
+}
+
+__global__ void evenly_spaced_kernel(int32_t n_blocks, int32_t C, int32_t k, int32_t* __restrict__ sel) {
+  const int64_t n = (int64_t)n_blocks * k;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int m = (int)(i % k);
+    sel[i] = (int32_t)(((int64_t)m * C) / k);
+  }
+}
+
+int launch_select_scored(const SelectArgs& a, int method, const FixedIdf& tab, long long* score,
+                         cudaStream_t s) {
+  const int64_t n_chunks = a.L / a.chunk;
+  const int C = a.block / a.chunk;
+  const int n_blocks = (int)(a.L / a.block);
+  if (method == PA_SCORE_EVENLY_SPACED) {
+    if (a.k > 0) {
+      const int64_t n = (int64_t)n_blocks * a.k;
+      evenly_spaced_kernel<<<(int)((n + 255) / 256), 256, 0, s>>>(n_blocks, C, a.k, a.sel);
+    }
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  }
+  if (cudaMemsetAsync(a.mask, 0, sizeof(unsigned long long) * (size_t)a.vocab, s) != cudaSuccess)
+    return PA_ERR_CUDA;
+  const int threads = 256;
+  const int64_t want = (a.L + threads - 1) / threads;
+  presence_mask_kernel<<<(int)(want < 148 * 16 ? want : 148 * 16), threads, 0, s>>>(
+      a.ids, a.L, a.vocab, a.block, a.mask, a.status);
+  const int64_t wgrid = (n_chunks * 32 + threads - 1) / threads;
+  chunk_fixed_score_kernel<<<(int)(wgrid < 148 * 32 ? wgrid : 148 * 32), threads, 0, s>>>(
+      a.ids, n_chunks, a.chunk, a.vocab, a.mask, tab, score);
+  if (a.k > 0) {
+    const size_t sm = sizeof(long long) * (size_t)C;
+    if (cudaFuncSetAttribute(topk_rank_kernel<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sm) != cudaSuccess)
+      return PA_ERR_CUDA;
+    topk_rank_kernel<1024><<<n_blocks, 1024, sm, s>>>(score, C, a.k, a.sel);
+  }
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+__global__ void widen_i32_kernel(const int32_t* __restrict__ in, long long* __restrict__ out, int64_t n) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x)
+    out[i] = in[i];
+}
+
+int launch_widen_i32(const int32_t* in, long long* out, int64_t n, cudaStream_t s) {
+  if (n > 0) {
+    const int64_t want = (n + 255) / 256;
+    widen_i32_kernel<<<(int)(want < 148 * 8 ? want : 148 * 8), 256, 0, s>>>(in, out, n);
+  }
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
 int launch_select(const SelectArgs& a, cudaStream_t s) {
   const int64_t n_chunks = a.L / a.chunk;
   const int C = a.block / a.chunk;

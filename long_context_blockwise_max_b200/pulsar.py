@@ -17,6 +17,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libpulsar_b200.so")
 
 PA_F32, PA_BF16 = 0, 1
+PA_SCORE_MAX_IDF, PA_SCORE_MEAN_IDF, PA_SCORE_EVENLY_SPACED = 0, 1, 2
 _STATUS = {0: "PA_OK", -1: "PA_ERR_INVALID", -2: "PA_ERR_UNSUPPORTED", -3: "PA_ERR_WORKSPACE",
            -4: "PA_ERR_CUDA", -5: "PA_ERR_TIMEOUT", -6: "PA_ERR_RANGE"}
 
@@ -24,6 +25,7 @@ _STATUS = {0: "PA_OK", -1: "PA_ERR_INVALID", -2: "PA_ERR_UNSUPPORTED", -3: "PA_E
 ABI_SYMBOLS = (
     "pa_abi_version", "pa_status_string", "pa_workspace_status", "pa_set_profile_events",
     "pa_select_workspace_size", "pulsar_select_summaries", "pulsar_select_summaries_noalloc",
+    "pulsar_select_summaries_scored",
     "pa_phase1_layout", "pa_phase1_workspace_size", "pulsar_phase1_encode", "star_phase1_encode",
     "pa_phase2_workspace_size", "star_phase2_attend",
 )
@@ -50,6 +52,8 @@ def _load() -> ctypes.CDLL:
         "pa_select_workspace_size": (SZ, [I64, I32, I32, I32]),
         "pulsar_select_summaries": (ctypes.c_int, [P, I64, I32, I32, I32, I32, P, P, P, P, SZ, P]),
         "pulsar_select_summaries_noalloc": (ctypes.c_int, [P, I64, I32, I32, I32, I32, P, P, P, P]),
+        "pulsar_select_summaries_scored": (ctypes.c_int, [P, I64, I32, I32, I32, I32, ctypes.c_int, P, P, P, SZ,
+                                                          P]),
         "pa_phase1_layout": (ctypes.c_int, [I64, I32, I32, I32, ctypes.c_int, P]),
         "pa_phase1_workspace_size": (SZ, [I64, I32, I32, I32, ctypes.c_int, I32, I32, I32, ctypes.c_int]),
         "pulsar_phase1_encode": (ctypes.c_int, [P, P, P, ctypes.c_int, I64, I32, I32, I32, D, I32, I32, I32,
@@ -163,6 +167,24 @@ def pulsar_select_summaries_noalloc(ids: torch.Tensor, vocab: int, block: int, c
                                               _ptr(df), _ptr(chunk_mindf), _stream())
     _check(rc, "pulsar_select_summaries_noalloc")
     return sel
+
+
+def pulsar_select_summaries_scored(ids, vocab: int, block: int, chunk: int, k_chunks: int, method: int,
+                                   L: int | None = None, sel=None, want_scores=False, ws=None):
+    """Selection with another chunk scorer (PA_SCORE_*).  ``ids`` may be None
+    for PA_SCORE_EVENLY_SPACED (then pass ``L``).  Returns (sel, scores or None, ws)."""
+    _dev(ids, sel)
+    L = ids.numel() if ids is not None else int(L)
+    dev = ids.device if ids is not None else torch.device("cuda", torch.cuda.current_device())
+    n = L // block if block > 0 else 0
+    if sel is None:
+        sel = torch.empty((n, k_chunks), dtype=torch.int32, device=dev)
+    scores = torch.empty(L // chunk, dtype=torch.int64, device=dev) if want_scores else None
+    ws = _workspace(pa_select_workspace_size(L, vocab, block, chunk), dev, ws)
+    rc = _lib.pulsar_select_summaries_scored(_ptr(ids), L, vocab, block, chunk, k_chunks, int(method), _ptr(sel),
+                                             _ptr(scores), _ptr(ws), ws.numel() * ws.element_size(), _stream())
+    _check(rc, "pulsar_select_summaries_scored")
+    return sel, scores, ws
 
 
 def pa_phase1_layout(L, block, sink, summary_tokens, star) -> list[int]:
