@@ -30,4 +30,5 @@ from .pulsar_oracle import (  # noqa: F401
     chunk_mean_idf_fixed,
     select_evenly_spaced,
     select_summaries_mean_idf,
+    phase2_attend_with_self,
 )

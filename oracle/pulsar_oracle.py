@@ -394,3 +394,40 @@ def phase2_attend(q, k_cache, v_cache, n_shards: int, q_pos0: int, theta: float)
                            n_shards)
     o, lse = lse_merge(A, s)
     return o, lse, A, s
+
+
+def phase2_attend_with_self(q, k_cache, v_cache, n_shards: int, k_self, v_self, self_off: int,
+                            q_pos0: int, theta: float):
+    """Query-host step: the query and generated tokens attend globally ([S]
+    summary: "only the query and generated tokens attend globally"; [P] §5
+    --tokens_to_generate).  Row j of q (rotated at q_pos0 + j) attends to
+    every retained key of the shards and, causally, to the query host's own
+    keys 0 .. self_off + j; the own keys form one more partial, merged with
+    the shards' by the same exact LSE merge.
+
+    q: [B][Tq][Hq][d] pre-RoPE; caches [B][T][Hkv][d]; k_self/v_self
+    [B][S][Hkv][d] with K already rotated, S >= self_off + Tq.
+    Returns (O [B][Tq][Hq][d], lse [B][Tq][Hq])."""
+    q = np.asarray(q, dtype=np.float64)
+    B, Tq, hq, d = q.shape
+    if theta > 0:
+        pos = q_pos0 + np.arange(Tq)
+        q = np.stack([rope(q[b], pos, theta) for b in range(B)])
+    A, s = phase2_partials(q, np.asarray(k_cache, np.float64), np.asarray(v_cache, np.float64), n_shards)
+    hkv = k_self.shape[2]
+    g = hq // hkv
+    scale = 1.0 / math.sqrt(d)
+    A_self = np.zeros((B, 1, Tq, hq, d), dtype=np.float64)
+    s_self = np.full((B, 1, Tq, hq), -np.inf, dtype=np.float64)
+    ks = np.asarray(k_self, np.float64)
+    vs = np.asarray(v_self, np.float64)
+    for b in range(B):
+        for j in range(Tq):
+            n = self_off + j + 1                       # own keys 0 .. self_off + j
+            for head in range(hq):
+                sc = (ks[b, :n, head // g, :] @ q[b, j, head, :]) * scale
+                mx = sc.max()
+                e = np.exp(sc - mx)
+                A_self[b, 0, j, head] = (e @ vs[b, :n, head // g, :]) / e.sum()
+                s_self[b, 0, j, head] = mx + np.log(e.sum())
+    return lse_merge(np.concatenate([A, A_self], axis=1), np.concatenate([s, s_self], axis=1))

@@ -179,3 +179,33 @@ def test_phase2_query_rotation_position():
     o, _, _, _ = oracle.phase2_attend(q, kr[None], vr[None], 4, p0, theta)
     want = _sdpa(_rope_complex(q[0], p0 + np.arange(3), theta), kr, v, False)
     np.testing.assert_allclose(o[0], want, rtol=0, atol=1e-12)
+
+
+def test_query_step_equals_dense_masked_attention():
+    # row j sees the whole context plus own keys 0..self_off+j: compare with
+    # library attention over the concatenated keys under an explicit mask
+    B, Tq, hq, hkv, d, T, S, off = 2, 5, 4, 2, 16, 37, 3, 4
+    q = _rand((B, Tq, hq, d), 60)
+    kc, vc = _rand((B, T, hkv, d), 61), _rand((B, T, hkv, d), 62)
+    ks, vs = _rand((B, off + Tq + 2, hkv, d), 63), _rand((B, off + Tq + 2, hkv, d), 64)
+    o, lse = oracle.phase2_attend_with_self(q, kc, vc, S, ks, vs, off, 0, 0.0)
+    for b in range(B):
+        keys = np.concatenate([kc[b], ks[b, :off + Tq]])
+        vals = np.concatenate([vc[b], vs[b, :off + Tq]])
+        mask = np.ones((Tq, T + off + Tq), dtype=bool)
+        for j in range(Tq):
+            mask[j, T + off + j + 1:] = False
+        tq = torch.from_numpy(q[b]).permute(1, 0, 2)[None]
+        tk = torch.from_numpy(keys).repeat_interleave(2, dim=1).permute(1, 0, 2)[None]
+        tv = torch.from_numpy(vals).repeat_interleave(2, dim=1).permute(1, 0, 2)[None]
+        want = F.scaled_dot_product_attention(tq, tk, tv, attn_mask=torch.from_numpy(mask))[0].permute(1, 0, 2)
+        np.testing.assert_allclose(o[b], want.numpy(), rtol=0, atol=1e-12)
+
+
+def test_query_step_without_context_is_causal_attention():
+    B, Tq, hq, hkv, d = 1, 9, 2, 1, 8
+    q = _rand((B, Tq, hq, d), 70)
+    ks, vs = _rand((B, Tq, hkv, d), 71), _rand((B, Tq, hkv, d), 72)
+    o, _ = oracle.phase2_attend_with_self(q, np.zeros((B, 0, hkv, d)), np.zeros((B, 0, hkv, d)), 2, ks, vs, 0,
+                                          0, 0.0)
+    np.testing.assert_allclose(o[0], _sdpa(q[0], ks[0], vs[0], True), rtol=0, atol=1e-12)
