@@ -388,6 +388,64 @@ def run_ours(args, rank, world, local_rank, dist_on):
         del dq, dk, dv
         torch.cuda.empty_cache()
 
+        # generation loop on the query host: the 64-token query, then 128
+        # tokens generated one at a time over the retained 128K cache
+        gen = 128
+        ng = w.q_tokens + gen
+        gq = workloads.normal((1, ng, w.hq, w.d), workloads.SEED_QUERY + 10, w.dtype, dev)
+        gk = workloads.normal((1, ng, w.hkv, w.d), workloads.SEED_QUERY + 11, w.dtype, dev)
+        gv = workloads.normal((1, ng, w.hkv, w.d), workloads.SEED_QUERY + 12, w.dtype, dev)
+        ks = torch.zeros((1, ng, w.hkv, w.d), dtype=w.dtype, device=dev)
+        vs = torch.zeros_like(ks)
+        kr1, vr1 = step.k_ret[None], step.v_ret[None]
+        go = torch.empty((1, 1, w.hq, w.d), dtype=w.dtype, device=dev)
+        gl = torch.empty((1, 1, w.hq), dtype=torch.float32, device=dev)
+        gws = torch.empty(P.pa_phase2_workspace_size(1, w.q_tokens, w.L, w.n_blocks, w.hq, w.hkv, w.d),
+                          dtype=torch.uint8, device=dev)
+        P.star_phase2_query_step(gq[:, :w.q_tokens].contiguous(), gk[:, :w.q_tokens].contiguous(),
+                                 gv[:, :w.q_tokens].contiguous(), kr1, vr1, w.n_blocks, ks, vs, 0, w.L,
+                                 w.rope_theta, ws=gws)
+        toks = [(gq[:, t:t + 1].contiguous(), gk[:, t:t + 1].contiguous(), gv[:, t:t + 1].contiguous())
+                for t in range(w.q_tokens, ng)]
+        torch.cuda.synchronize()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record()
+        for i, (a_q, a_k, a_v) in enumerate(toks):
+            t = w.q_tokens + i
+            P.star_phase2_query_step(a_q, a_k, a_v, kr1, vr1, w.n_blocks, ks, vs, t, w.L + t, w.rope_theta,
+                                     o=go, lse=gl, ws=gws)
+        g1.record()
+        torch.cuda.synchronize()
+        gen_ms = g0.elapsed_time(g1) / gen
+        cache_bytes = 2.0 * w.L * w.hkv * w.d * 2
+        extra["generation"] = {"context": w.L, "query_tokens": w.q_tokens, "generated": gen,
+                               "ms_per_token": round(gen_ms, 4), "tokens_per_s": round(1e3 / gen_ms, 1),
+                               "cache_gb_s": round(cache_bytes / (gen_ms * 1e-3) / 1e9, 1)}
+        del gq, gk, gv, ks, vs, toks
+
+        # summary scorers on the 128K and 1M token ids (selection alone)
+        sc = {}
+        for wl in (WORKLOAD, workloads.SCALE_1M):
+            idd = torch.from_numpy(wl.token_ids()).to(dev)
+            sws = torch.empty(P.pa_select_workspace_size(wl.L, wl.vocab, wl.block, wl.chunk), dtype=torch.uint8,
+                              device=dev)
+            for name, method in (("max_idf", P.PA_SCORE_MAX_IDF), ("mean_idf", P.PA_SCORE_MEAN_IDF),
+                                 ("evenly_spaced", P.PA_SCORE_EVENLY_SPACED)):
+                def sel_call():
+                    P.pulsar_select_summaries_scored(idd, wl.vocab, wl.block, wl.chunk, wl.k_chunks, method,
+                                                     ws=sws)
+                for _ in range(3):
+                    sel_call()
+                torch.cuda.synchronize()
+                a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a0.record()
+                for _ in range(10):
+                    sel_call()
+                a1.record()
+                torch.cuda.synchronize()
+                sc[f"{wl.name}:{name}_us"] = round(a0.elapsed_time(a1) / 10 * 1e3, 1)
+        extra["selection_us"] = sc
+
     q2_bytes = 2.0 * w.L * w.hkv * w.d * 2
     clocks = clk.summary()
     line = {
@@ -491,7 +549,7 @@ def run_reference(args):
 
 
 def run_profile_case(name, steps, warmup):
-    """A single kernel family on a small workload, for ncu captures:
+    """One kernel family on a small workload, for ncu captures:
     phase1-32k (Pulsar Phase 1 incl. its RoPE prepass, 32K shape),
     decode-128k / decode-16k (Phase-2 decode, 16 queries over a 128K / 16K
     cache in 8 shards), query-128k (Phase-2 64-token query).  Prints one JSON

@@ -276,6 +276,43 @@ int star_phase2_attend(const void* q, int dtype, int32_t B, int32_t Tq, int64_t 
                        float* part_o_opt, float* part_lse_opt, void* ws, size_t ws_bytes,
                        void* stream);
 
+/*
+ * Exact merge of Phase-2 partials ([S] Algorithm 2 as corrected in the
+ * referee's comment; [P] §2.2 "an all_gather followed by an online-softmax
+ * merge"), for partials gathered from several GPUs:
+ * lse = ln sum_h exp(s_h), O = sum_h exp(s_h - lse) A_h.
+ *  part_o    [B][S][Tq][hq][d] float (A_h, as star_phase2_attend writes it)
+ *  part_lse  [B][S][Tq][hq] float (s_h; -inf marks an empty shard)
+ *  o         out [B][Tq][hq][d] dtype;  lse out [B][Tq][hq] float.
+ * All shards empty: O = 0, lse = -inf.  No workspace.
+ */
+int pa_lse_merge(const float* part_o, const float* part_lse, int32_t B, int32_t S, int32_t Tq,
+                 int32_t hq, int32_t d, int dtype, void* o, float* lse, void* stream);
+
+/*
+ * One step of the query host (NEXT row: query and generation loop).  The
+ * query and the generated tokens attend globally ([S] summary: "only the
+ * query and generated tokens attend globally"; [P] §5 --tokens_to_generate):
+ * the Tq new tokens' K (rotated at q_pos0 + j) and V are appended to the
+ * query host's own cache at rows self_len + j, then row j of q (rotated at
+ * q_pos0 + j) attends to every key of the retained shards and, causally, to
+ * own-cache rows 0 .. self_len + j; the result is merged exactly with the
+ * shards'.  Calling it once with the query (self_len = 0) and then once per
+ * generated token (Tq = 1, self_len growing) is the generation loop.
+ *
+ *  q, k_new, v_new  [B][Tq][hq | hkv | hkv][d] dtype, unrotated.
+ *  k_self, v_self   in/out [B][self_cap][hkv][d] dtype, the own cache (K
+ *                   rotated); self_len + Tq <= self_cap.
+ *  o, lse           out as star_phase2_attend.
+ * Other arguments, errors and workspace (pa_phase2_workspace_size) as
+ * star_phase2_attend.
+ */
+int star_phase2_query_step(const void* q, const void* k_new, const void* v_new, int dtype, int32_t B,
+                           int32_t Tq, int64_t q_pos0, double rope_theta, const void* k_ret,
+                           const void* v_ret, int64_t T, int32_t n_shards, void* k_self, void* v_self,
+                           int64_t self_cap, int64_t self_len, int32_t hq, int32_t hkv, int32_t d,
+                           void* o, float* lse, void* ws, size_t ws_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -123,6 +123,19 @@ int phase1_common(const void* q, const void* k, const void* v, int dtype, int64_
   return launch_phase1(a, s);
 }
 
+void carve_phase2(Phase2Args& a, void* ws) {
+  char* w = static_cast<char*>(ws);
+  a.status = reinterpret_cast<DeviceStatus*>(w);
+  const size_t rows = (size_t)a.B * a.Tq * a.hq;
+  const size_t units = (size_t)a.n_shards * a.n_split + 1;   // + the own-cache unit
+  size_t off = kStatusBytes;
+  a.qr = reinterpret_cast<float*>(w + off);
+  off += align_up(sizeof(float) * rows * a.d);
+  a.unit_o = reinterpret_cast<float*>(w + off);
+  off += align_up(sizeof(float) * rows * units * a.d);
+  a.unit_lse = reinterpret_cast<float*>(w + off);
+}
+
 }  // namespace
 
 extern "C" {
@@ -318,17 +331,66 @@ int star_phase2_attend(const void* q, int dtype, int32_t B, int32_t Tq, int64_t 
   a.n_split = phase2_split(B, Tq, T, n_shards, hq, hkv);
   a.hq = hq; a.hkv = hkv; a.d = d;
   a.o = o; a.lse = lse; a.part_o_opt = part_o_opt; a.part_lse_opt = part_lse_opt;
-  char* w = static_cast<char*>(ws);
-  a.status = reinterpret_cast<DeviceStatus*>(w);
-  const size_t rows = (size_t)B * Tq * hq;
-  const size_t units = (size_t)n_shards * a.n_split;
-  size_t off = kStatusBytes;
-  a.qr = reinterpret_cast<float*>(w + off);
-  off += align_up(sizeof(float) * rows * d);
-  a.unit_o = reinterpret_cast<float*>(w + off);
-  off += align_up(sizeof(float) * rows * units * d);
-  a.unit_lse = reinterpret_cast<float*>(w + off);
+  carve_phase2(a, ws);
   if (B == 0 || Tq == 0) return PA_OK;
+  return launch_phase2(a, s);
+}
+
+int pa_lse_merge(const float* part_o, const float* part_lse, int32_t B, int32_t S, int32_t Tq,
+                 int32_t hq, int32_t d, int dtype, void* o, float* lse, void* stream) {
+  if (B < 0 || S < 1 || Tq < 0 || hq < 1) return PA_ERR_INVALID;
+  if (d != 64 && d != 128) return PA_ERR_UNSUPPORTED;
+  if (dtype != PA_F32 && dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+  if (B > 0 && Tq > 0 && (!part_o || !part_lse || !o || !lse)) return PA_ERR_INVALID;
+  Phase2Args a;
+  a.dtype = dtype;
+  a.B = B; a.Tq = Tq; a.hq = hq; a.hkv = hq; a.d = d;
+  a.n_shards = S; a.n_split = 1; a.has_self = 0;
+  a.unit_o = const_cast<float*>(part_o);
+  a.unit_lse = const_cast<float*>(part_lse);
+  a.part_o_opt = nullptr; a.part_lse_opt = nullptr;
+  a.o = o; a.lse = lse;
+  a.status = nullptr;
+  return launch_merge_only(a, static_cast<cudaStream_t>(stream));
+}
+
+int star_phase2_query_step(const void* q, const void* k_new, const void* v_new, int dtype, int32_t B,
+                           int32_t Tq, int64_t q_pos0, double rope_theta, const void* k_ret,
+                           const void* v_ret, int64_t T, int32_t n_shards, void* k_self, void* v_self,
+                           int64_t self_cap, int64_t self_len, int32_t hq, int32_t hkv, int32_t d,
+                           void* o, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int rc = check_heads(hq, hkv, d, dtype);
+  if (rc) return rc;
+  if (B < 0 || Tq < 0 || T < 0 || n_shards < 1 || n_shards > 4096) return PA_ERR_INVALID;
+  if (!std::isfinite(rope_theta)) return PA_ERR_INVALID;
+  if (self_len < 0 || self_cap < 0 || self_len + Tq > self_cap) return PA_ERR_INVALID;
+  if (B > 0 && Tq > 0) {
+    if (!q || !k_new || !v_new || !k_self || !v_self || !o || !lse) return PA_ERR_INVALID;
+    if (T > 0 && (!k_ret || !v_ret)) return PA_ERR_INVALID;
+  }
+  const void* ptrs[] = {q, k_new, v_new, k_ret, v_ret, k_self, v_self, o};
+  for (const void* p : ptrs)
+    if (p && !aligned(p, 16)) return PA_ERR_UNSUPPORTED;
+  const size_t need = phase2_workspace_bytes(B, Tq, T, n_shards, hq, hkv, d);
+  rc = check_ws(ws, ws_bytes, need);
+  if (rc) return rc;
+  rc = clear_status(ws, s);
+  if (rc) return rc;
+  Phase2Args a;
+  a.dtype = dtype;
+  a.q = q; a.B = B; a.Tq = Tq; a.q_pos0 = q_pos0; a.rope_theta = rope_theta;
+  a.k_ret = k_ret; a.v_ret = v_ret; a.T = T;
+  a.n_shards = n_shards;
+  a.n_split = phase2_split(B, Tq, T, n_shards, hq, hkv);
+  a.hq = hq; a.hkv = hkv; a.d = d;
+  a.o = o; a.lse = lse; a.part_o_opt = nullptr; a.part_lse_opt = nullptr;
+  a.k_self = k_self; a.v_self = v_self; a.self_cap = self_cap; a.self_len = self_len;
+  a.has_self = 1;
+  carve_phase2(a, ws);
+  if (B == 0 || Tq == 0) return PA_OK;
+  rc = launch_self_append(a, k_new, v_new, s);
+  if (rc) return rc;
   return launch_phase2(a, s);
 }
 

@@ -99,12 +99,60 @@ struct Phase2Args {
   float* unit_o;                // workspace [B][units][Tq][hq][d]
   float* unit_lse;              // workspace [B][units][Tq][hq]
   DeviceStatus* status;
+  // optional own cache of the query host ([B][self_cap][hkv][d], K rotated):
+  // query row t also sees its rows 0 .. self_len + t (one extra unit)
+  const void* k_self = nullptr;
+  const void* v_self = nullptr;
+  int64_t self_cap = 0, self_len = 0;
+  int has_self = 0;
 };
+
+// One Phase-2 work unit: a split of a context shard, or (the last unit, when
+// the own cache is attached) the own cache with its causal limit.
+struct UnitView {
+  const void* K;
+  const void* V;
+  int64_t stride_rows;    // rows per batch element of K / V
+  int64_t k0, k1;         // key range
+  int64_t causal_base;    // row t sees keys <= causal_base + t; -1: every key
+};
+
+__host__ __device__ inline int phase2_units(const Phase2Args& a) {
+  return a.n_shards * a.n_split + (a.has_self ? 1 : 0);
+}
+
+__device__ inline UnitView phase2_unit(const Phase2Args& a, int u) {
+  UnitView v;
+  const int ctx = a.n_shards * a.n_split;
+  if (u >= ctx) {
+    v.K = a.k_self;
+    v.V = a.v_self;
+    v.stride_rows = a.self_cap;
+    v.k0 = 0;
+    v.k1 = a.self_len + a.Tq;
+    v.causal_base = a.self_len;
+    return v;
+  }
+  v.K = a.k_ret;
+  v.V = a.v_ret;
+  v.stride_rows = a.T;
+  const int64_t step = (a.T + a.n_shards - 1) / a.n_shards;
+  const int sh = u / a.n_split, sp = u % a.n_split;
+  const int64_t lo = min((int64_t)sh * step, a.T), hi = min((int64_t)(sh + 1) * step, a.T);
+  const int64_t len = (hi - lo + a.n_split - 1) / a.n_split;
+  v.k0 = min(lo + (int64_t)sp * len, hi);
+  v.k1 = min(lo + (int64_t)(sp + 1) * len, hi);
+  v.causal_base = -1;
+  return v;
+}
 int launch_phase2_mma(const Phase2Args& a, cudaStream_t s);
 int32_t phase2_split(int32_t B, int32_t Tq, int64_t T, int32_t n_shards, int32_t hq,
                      int32_t hkv);
 size_t phase2_workspace_bytes(int32_t B, int32_t Tq, int64_t T, int32_t n_shards, int32_t hq,
                               int32_t hkv, int32_t d);
 int launch_phase2(const Phase2Args& a, cudaStream_t s);
+int launch_merge_only(const Phase2Args& a, cudaStream_t s);
+// rotate the new tokens' K at q_pos0 + j and append K, V to the own cache
+int launch_self_append(const Phase2Args& a, const void* k_new, const void* v_new, cudaStream_t s);
 
 }  // namespace pa

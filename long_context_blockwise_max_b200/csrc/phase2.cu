@@ -39,32 +39,23 @@ __global__ void rope_query_kernel(const IT* __restrict__ q, int B, int Tq, int h
   }
 }
 
-__host__ __device__ inline void unit_range(int64_t T, int n_shards, int n_split, int u,
-                                           int64_t* k0, int64_t* k1) {
-  const int64_t step = (T + n_shards - 1) / n_shards;
-  const int sh = u / n_split, sp = u % n_split;
-  const int64_t lo = min((int64_t)sh * step, T), hi = min((int64_t)(sh + 1) * step, T);
-  const int64_t len = (hi - lo + n_split - 1) / n_split;
-  *k0 = min(lo + (int64_t)sp * len, hi);
-  *k1 = min(lo + (int64_t)(sp + 1) * len, hi);
-}
-
 template <int D, typename VT>
 __global__ void __launch_bounds__(256) phase2_simt_kernel(Phase2Args a) {
   constexpr int BK = 32, HALF = D / 2, G4 = HALF / 4;
   __shared__ __align__(16) float ks[BK][D];
   __shared__ __align__(16) float vs[BK][D];
-  const int units = a.n_shards * a.n_split;
+  const int units = phase2_units(a);
   const int b = blockIdx.x / units, u = blockIdx.x % units;
   const int kvh = blockIdx.y, g = a.hq / a.hkv;
   const int idx = blockIdx.z * 128 + (threadIdx.x >> 1);
   const int hf = threadIdx.x & 1;
   const bool active = idx < a.Tq * g;
   const int t = active ? idx / g : 0, head = kvh * g + (active ? idx % g : 0);
-  int64_t k0, k1;
-  unit_range(a.T, a.n_shards, a.n_split, u, &k0, &k1);
-  const VT* K = static_cast<const VT*>(a.k_ret) + (int64_t)b * a.T * a.hkv * D;
-  const VT* V = static_cast<const VT*>(a.v_ret) + (int64_t)b * a.T * a.hkv * D;
+  const UnitView uv = phase2_unit(a, u);
+  const int64_t k0 = uv.k0, k1 = uv.k1;
+  const int64_t lim = uv.causal_base < 0 ? INT64_MAX : uv.causal_base + t;   // last visible key
+  const VT* K = static_cast<const VT*>(uv.K) + (int64_t)b * uv.stride_rows * a.hkv * D;
+  const VT* V = static_cast<const VT*>(uv.V) + (int64_t)b * uv.stride_rows * a.hkv * D;
   float qv[HALF], acc[HALF];
   {
     const float* src = a.qr + (((int64_t)b * a.Tq + t) * a.hq + head) * D;
@@ -105,9 +96,10 @@ __global__ void __launch_bounds__(256) phase2_simt_kernel(Phase2Args a) {
         acc_s = fmaf(qv[4 * gg + 3], kk4.w, acc_s);
       }
       acc_s += __shfl_xor_sync(0xffffffffu, acc_s, 1);
-      s[j] = (c0 + j < k1) ? acc_s : -INFINITY;
+      s[j] = (c0 + j < k1 && c0 + j <= lim) ? acc_s : -INFINITY;
       mt = fmaxf(mt, s[j]);
     }
+    if (mt == -INFINITY) continue;   // every key of this tile is masked for this row
     const float alpha = fast_exp2(m_run - mt);
     l_run *= alpha;
 #pragma unroll
@@ -130,7 +122,7 @@ __global__ void __launch_bounds__(256) phase2_simt_kernel(Phase2Args a) {
   if (!active) return;
   const int64_t orow = (((int64_t)b * units + u) * a.Tq + t) * a.hq + head;
   float* dst = a.unit_o + orow * D;
-  const bool empty = k1 <= k0;
+  const bool empty = (m_run == -INFINITY);
   const float inv = empty ? 0.f : 1.f / l_run;
 #pragma unroll
   for (int gg = 0; gg < G4; ++gg)
@@ -145,7 +137,7 @@ template <typename OT>
 __global__ void merge_kernel(Phase2Args a) {
   const int lane = threadIdx.x & 31;
   const int64_t nrows = (int64_t)a.B * a.Tq * a.hq;
-  const int units = a.n_shards * a.n_split;
+  const int units = phase2_units(a);
   const int per_lane = a.d / 32;   // 2 or 4
   for (int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < nrows;
        row += ((int64_t)gridDim.x * blockDim.x) >> 5) {
@@ -182,6 +174,18 @@ __global__ void merge_kernel(Phase2Args a) {
       for (int e = 0; e < per_lane; ++e) gacc[e] = gacc[e] * c_old + sacc[e] * c_new;
       gm = mn;
     }
+    if (a.has_self) {   // the own cache's unit (after the shards)
+      const int64_t urow = (b * units + (units - 1)) * (int64_t)a.Tq * a.hq + th;
+      const float s = a.unit_lse[urow];
+      if (s != -INFINITY) {
+        const float mn = fmaxf(gm, s);
+        const float c_old = expf(gm - mn), c_new = expf(s - mn);
+        gz = gz * c_old + c_new;
+        const float* A = a.unit_o + urow * a.d;
+        for (int e = 0; e < per_lane; ++e) gacc[e] = gacc[e] * c_old + c_new * A[lane + 32 * e];
+        gm = mn;
+      }
+    }
     OT* O = static_cast<OT*>(a.o) + row * a.d;
     const float inv = (gm == -INFINITY) ? 0.f : 1.f / gz;
     for (int e = 0; e < per_lane; ++e) O[lane + 32 * e] = from_f32<OT>(gacc[e] * inv);
@@ -210,7 +214,7 @@ int32_t phase2_split(int32_t B, int32_t Tq, int64_t T, int32_t n_shards, int32_t
 size_t phase2_workspace_bytes(int32_t B, int32_t Tq, int64_t T, int32_t n_shards, int32_t hq,
                               int32_t hkv, int32_t d) {
   const int32_t ns = phase2_split(B, Tq, T, n_shards, hq, hkv);
-  const size_t units = (size_t)n_shards * ns;
+  const size_t units = (size_t)n_shards * ns + 1;   // + the query host's own cache
   const size_t rows = (size_t)B * Tq * hq;
   size_t b = kStatusBytes;
   b += align_up(sizeof(float) * rows * d);          // rotated query
@@ -232,7 +236,7 @@ static int launch_phase2_t(const Phase2Args& a, cudaStream_t s) {
         static_cast<const IT*>(a.q), a.B, a.Tq, a.hq, a.d, a.q_pos0, a.rope_theta > 0, f, qscale,
         a.qr);
   }
-  const int units = a.n_shards * a.n_split;
+  const int units = phase2_units(a);
   const int g = a.hq / a.hkv;
   const dim3 grid((unsigned)(a.B * units), a.hkv, (unsigned)((a.Tq * g + 127) / 128));
   int rc = PA_OK;
@@ -249,6 +253,73 @@ static int launch_phase2_t(const Phase2Args& a, cudaStream_t s) {
   if (nrows > 0) {
     const int64_t want = (nrows * 32 + 255) / 256;
     merge_kernel<IT><<<(int)(want < 148 * 16 ? want : 148 * 16), 256, 0, s>>>(a);
+  }
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+// Own-cache append: K of the new token j is rotated at q_pos0 + j and written
+// with its V at row self_len + j of the query host's cache.
+template <typename IT>
+__global__ void self_append_kernel(const IT* __restrict__ k_new, const IT* __restrict__ v_new, int B,
+                                   int Tq, int hkv, int d, int64_t q_pos0, int use_rope, RopeFreqs f,
+                                   IT* __restrict__ k_self, IT* __restrict__ v_self, int64_t self_cap,
+                                   int64_t self_len) {
+  const int half = d / 2;
+  const int64_t n = (int64_t)B * Tq * hkv * half;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int m = (int)(e % half);
+    const int64_t row = e / half;               // (b, t, h)
+    const int h = (int)(row % hkv);
+    const int t = (int)((row / hkv) % Tq);
+    const int64_t b = row / ((int64_t)hkv * Tq);
+    const int64_t src = row * d;
+    const int64_t dst = ((b * self_cap + self_len + t) * hkv + h) * (int64_t)d;
+    const float x1 = to_f32(k_new[src + m]), x2 = to_f32(k_new[src + m + half]);
+    float y1 = x1, y2 = x2;
+    if (use_rope) {
+      double sn, cn;
+      sincos((double)(q_pos0 + t) * f.omega[m], &sn, &cn);
+      const float c = (float)cn, sv = (float)sn;
+      y1 = x1 * c - x2 * sv;
+      y2 = x2 * c + x1 * sv;
+    }
+    k_self[dst + m] = from_f32<IT>(y1);
+    k_self[dst + m + half] = from_f32<IT>(y2);
+    v_self[dst + m] = v_new[src + m];
+    v_self[dst + m + half] = v_new[src + m + half];
+  }
+}
+
+template <typename IT>
+static int launch_self_append_t(const Phase2Args& a, const void* k_new, const void* v_new, cudaStream_t s) {
+  RopeFreqs f;
+  for (int m = 0; m < kMaxHalfDim; ++m)
+    f.omega[m] = (m < a.d / 2 && a.rope_theta > 0) ? pow(a.rope_theta, -2.0 * m / a.d) : 0.0;
+  const int64_t n = (int64_t)a.B * a.Tq * a.hkv * (a.d / 2);
+  if (n > 0) {
+    const int64_t want = (n + 255) / 256;
+    self_append_kernel<IT><<<(int)(want < 148 * 8 ? want : 148 * 8), 256, 0, s>>>(
+        static_cast<const IT*>(k_new), static_cast<const IT*>(v_new), a.B, a.Tq, a.hkv, a.d, a.q_pos0,
+        a.rope_theta > 0, f, static_cast<IT*>(const_cast<void*>(a.k_self)),
+        static_cast<IT*>(const_cast<void*>(a.v_self)), a.self_cap, a.self_len);
+  }
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+int launch_self_append(const Phase2Args& a, const void* k_new, const void* v_new, cudaStream_t s) {
+  if (a.dtype == PA_F32) return launch_self_append_t<float>(a, k_new, v_new, s);
+  return launch_self_append_t<__nv_bfloat16>(a, k_new, v_new, s);
+}
+
+int launch_merge_only(const Phase2Args& a, cudaStream_t s) {
+  const int64_t nrows = (int64_t)a.B * a.Tq * a.hq;
+  if (nrows > 0) {
+    const int64_t want = (nrows * 32 + 255) / 256;
+    if (a.dtype == PA_F32)
+      merge_kernel<float><<<(int)(want < 148 * 16 ? want : 148 * 16), 256, 0, s>>>(a);
+    else
+      merge_kernel<__nv_bfloat16><<<(int)(want < 148 * 16 ? want : 148 * 16), 256, 0, s>>>(a);
   }
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }

@@ -79,7 +79,7 @@ __global__ void __launch_bounds__(kWarps * 32) phase2_mma_kernel(Phase2Args a, i
   using C = P2Cfg<D>;
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int units = a.n_shards * a.n_split;
+  const int units = phase2_units(a);
   const int rg = blockIdx.x % row_groups;
   const int bu = blockIdx.x / row_groups;
   const int b = bu / units, u = bu % units;
@@ -87,15 +87,8 @@ __global__ void __launch_bounds__(kWarps * 32) phase2_mma_kernel(Phase2Args a, i
   const int g = a.hq / a.hkv;
   const int R = a.Tq * g;
 
-  int64_t k0, k1;
-  {
-    const int64_t step = (a.T + a.n_shards - 1) / a.n_shards;
-    const int sh = u / a.n_split, sp = u % a.n_split;
-    const int64_t lo = min((int64_t)sh * step, a.T), hi = min((int64_t)(sh + 1) * step, a.T);
-    const int64_t len = (hi - lo + a.n_split - 1) / a.n_split;
-    k0 = min(lo + (int64_t)sp * len, hi);
-    k1 = min(lo + (int64_t)(sp + 1) * len, hi);
-  }
+  const UnitView uv = phase2_unit(a, u);
+  const int64_t k0 = uv.k0, k1 = uv.k1;
 
   // ---- query fragments: rows 0-7 high part, rows 8-15 residual ----------
   const int qi = lane >> 2;            // real row of this thread (0..7)
@@ -131,10 +124,11 @@ __global__ void __launch_bounds__(kWarps * 32) phase2_mma_kernel(Phase2Args a, i
   const int64_t n_tiles = (k1 - k0 + kKT - 1) / kKT;
   const int my_tiles = n_tiles > warp ? (int)((n_tiles - 1 - warp) / kWarps + 1) : 0;
   const uint32_t wbase = static_cast<uint32_t>(__cvta_generic_to_shared(smem)) + warp * C::WARP_BYTES;
-  const __nv_bfloat16* Kg = static_cast<const __nv_bfloat16*>(a.k_ret);
-  const __nv_bfloat16* Vg = static_cast<const __nv_bfloat16*>(a.v_ret);
+  const __nv_bfloat16* Kg = static_cast<const __nv_bfloat16*>(uv.K);
+  const __nv_bfloat16* Vg = static_cast<const __nv_bfloat16*>(uv.V);
   const int64_t key_stride = (int64_t)a.hkv * D;   // elements between consecutive keys
-  const int64_t base_off = ((int64_t)b * a.T) * key_stride + (int64_t)kvh * D;
+  const int64_t base_off = ((int64_t)b * uv.stride_rows) * key_stride + (int64_t)kvh * D;
+  const int64_t lim = uv.causal_base < 0 ? INT64_MAX : uv.causal_base + t_row;   // last visible key
 
   auto issue = [&](int it) {
     if (it < my_tiles) {
@@ -192,14 +186,15 @@ __global__ void __launch_bounds__(kWarps * 32) phase2_mma_kernel(Phase2Args a, i
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int64_t kg = key0 + nt * 8 + qc + e;
-        const float x = (kg < k1) ? s[nt][e] + s[nt][e + 2] : -INFINITY;
+        const float x = (kg < k1 && kg <= lim) ? s[nt][e] + s[nt][e + 2] : -INFINITY;
         sv[nt][e] = x;
         mt = fmaxf(mt, x);
       }
     mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
     mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
     const float m_new = fmaxf(m_run, mt);
-    const float alpha = fast_exp2(m_run - m_new);
+    const float alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(m_run - m_new);
+    const float m_sub = (m_new == -INFINITY) ? 0.f : m_new;   // rows that see no key yet
     m_run = m_new;
     l_run *= alpha;
 #pragma unroll
@@ -210,7 +205,7 @@ __global__ void __launch_bounds__(kWarps * 32) phase2_mma_kernel(Phase2Args a, i
     uint32_t pa_[4];
 #pragma unroll
     for (int nt = 0; nt < 4; ++nt) {
-      const float p0 = fast_exp2(sv[nt][0] - m_new), p1 = fast_exp2(sv[nt][1] - m_new);
+      const float p0 = fast_exp2(sv[nt][0] - m_sub), p1 = fast_exp2(sv[nt][1] - m_sub);
       l_run += p0 + p1;
       pa_[nt] = pack_bf16(p0, p1);
     }
@@ -289,7 +284,7 @@ __global__ void __launch_bounds__(kWarps * 32) phase2_mma_rows_kernel(Phase2Args
   using C = P2Cfg<D>;
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int units = a.n_shards * a.n_split;
+  const int units = phase2_units(a);
   const int rb = blockIdx.x % row_blocks;
   const int bu = blockIdx.x / row_blocks;
   const int b = bu / units, u = bu % units;
@@ -298,15 +293,8 @@ __global__ void __launch_bounds__(kWarps * 32) phase2_mma_rows_kernel(Phase2Args
   const int R = a.Tq * g;
   const int rg = rb * kWarps + warp;   // this warp's group of 8 rows
 
-  int64_t k0, k1;
-  {
-    const int64_t step = (a.T + a.n_shards - 1) / a.n_shards;
-    const int sh = u / a.n_split, sp = u % a.n_split;
-    const int64_t lo = min((int64_t)sh * step, a.T), hi = min((int64_t)(sh + 1) * step, a.T);
-    const int64_t len = (hi - lo + a.n_split - 1) / a.n_split;
-    k0 = min(lo + (int64_t)sp * len, hi);
-    k1 = min(lo + (int64_t)(sp + 1) * len, hi);
-  }
+  const UnitView uv = phase2_unit(a, u);
+  const int64_t k0 = uv.k0, k1 = uv.k1;
   const int qi = lane >> 2, qc = (lane & 3) * 2;
   const int rr = rg * 8 + qi;
   const bool row_ok = rr < R;
@@ -336,10 +324,11 @@ __global__ void __launch_bounds__(kWarps * 32) phase2_mma_rows_kernel(Phase2Args
   }
   const int n_tiles = static_cast<int>((k1 - k0 + kKT - 1) / kKT);
   const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
-  const __nv_bfloat16* Kg = static_cast<const __nv_bfloat16*>(a.k_ret);
-  const __nv_bfloat16* Vg = static_cast<const __nv_bfloat16*>(a.v_ret);
+  const __nv_bfloat16* Kg = static_cast<const __nv_bfloat16*>(uv.K);
+  const __nv_bfloat16* Vg = static_cast<const __nv_bfloat16*>(uv.V);
   const int64_t key_stride = (int64_t)a.hkv * D;
-  const int64_t base_off = ((int64_t)b * a.T) * key_stride + (int64_t)kvh * D;
+  const int64_t base_off = ((int64_t)b * uv.stride_rows) * key_stride + (int64_t)kvh * D;
+  const int64_t lim = uv.causal_base < 0 ? INT64_MAX : uv.causal_base + t_row;   // last visible key
   auto issue = [&](int it) {
     if (it < n_tiles) {
       const int64_t key0 = k0 + (int64_t)it * kKT;
@@ -392,14 +381,15 @@ __global__ void __launch_bounds__(kWarps * 32) phase2_mma_rows_kernel(Phase2Args
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int64_t kg = key0 + nt * 8 + qc + e;
-        const float x = (kg < k1) ? s[nt][e] + s[nt][e + 2] : -INFINITY;
+        const float x = (kg < k1 && kg <= lim) ? s[nt][e] + s[nt][e + 2] : -INFINITY;
         sv[nt][e] = x;
         mt = fmaxf(mt, x);
       }
     mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
     mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
     const float m_new = fmaxf(m_run, mt);
-    const float alpha = fast_exp2(m_run - m_new);
+    const float alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(m_run - m_new);
+    const float m_sub = (m_new == -INFINITY) ? 0.f : m_new;   // rows that see no key yet
     m_run = m_new;
     l_run *= alpha;
 #pragma unroll
@@ -410,7 +400,7 @@ __global__ void __launch_bounds__(kWarps * 32) phase2_mma_rows_kernel(Phase2Args
     uint32_t pa_[4];
 #pragma unroll
     for (int nt = 0; nt < 4; ++nt) {
-      const float p0 = fast_exp2(sv[nt][0] - m_new), p1 = fast_exp2(sv[nt][1] - m_new);
+      const float p0 = fast_exp2(sv[nt][0] - m_sub), p1 = fast_exp2(sv[nt][1] - m_sub);
       l_run += p0 + p1;
       pa_[nt] = pack_bf16(p0, p1);
     }
@@ -447,7 +437,7 @@ template <int D>
 int launch_d(const Phase2Args& a, cudaStream_t s) {
   const int g = a.hq / a.hkv;
   const int R = a.Tq * g;
-  const int units = a.n_shards * a.n_split;
+  const int units = phase2_units(a);
   if (R <= 8) {
     // a few rows per kv head (decode): the 4 warps split the keys
     const int64_t gx = (int64_t)a.B * units;

@@ -1,0 +1,74 @@
+"""Phase 2 across GPUs: the exchange step of the query phase.
+
+The Pulsar Attention page (§2.2) and the Star Attention review
+(key_machinery) describe the only communication of the method.
+
+1. The query is broadcast.
+2. Each host attends over the retained cache it holds.
+3. The partial results (one vector and one scalar per query token and head)
+   are all-gathered.
+4. An exact online-softmax merge follows.
+
+Here every rank holds a contiguous range of shards. It computes their
+partials with ``star_phase2_attend`` and all-gathers the packed partials
+with ``torch.distributed`` (NCCL on GPUs). Every rank then merges all of them
+with ``pa_lse_merge``. The partial and merge steps can be replaced by other
+functions of the same contract, which the CPU tests use with the gloo
+backend.
+"""
+from __future__ import annotations
+
+import torch
+import torch.distributed as dist
+
+
+def shard_ranges(n_shards: int, world: int) -> list[tuple[int, int]]:
+    """Contiguous shard ranges of the ranks: ceil(n_shards / world) each, the
+    last ranks possibly shorter or empty."""
+    per = -(-n_shards // world)
+    return [(min(r * per, n_shards), min((r + 1) * per, n_shards)) for r in range(world)]
+
+
+def _gpu_partials(q, k_local, v_local, n_local, q_pos0, rope_theta):
+    from . import pulsar
+    _, _, part_o, part_lse, _ = pulsar.star_phase2_attend(q, k_local, v_local, n_local, q_pos0=q_pos0,
+                                                          rope_theta=rope_theta, want_partials=True)
+    return part_o, part_lse
+
+
+def _gpu_merge(part_o, part_lse, dtype):
+    from . import pulsar
+    return pulsar.pa_lse_merge(part_o, part_lse, dtype=dtype)
+
+
+def phase2_attend_distributed(q, k_local, v_local, n_local: int, n_shards_total: int, q_pos0: int,
+                              rope_theta: float, group=None, partials_fn=None, merge_fn=None):
+    """Exact global query attention over shards spread across ranks.
+
+    q: [B][Tq][hq][d], the same on every rank.
+    k_local, v_local: [B][T_local][hkv][d], this rank's n_local shards in
+    order (K rotated). The ranks' shards, concatenated in rank order, are
+    the n_shards_total shards of the whole cache.
+    Returns (O [B][Tq][hq][d], lse [B][Tq][hq]) on every rank.
+    """
+    partials_fn = partials_fn or _gpu_partials
+    merge_fn = merge_fn or _gpu_merge
+    world = dist.get_world_size(group)
+    per = -(-n_shards_total // world)
+    B, Tq, hq, d = q.shape
+    if n_local > 0:
+        part_o, part_lse = partials_fn(q, k_local, v_local, n_local, q_pos0, rope_theta)
+    else:
+        part_o = q.new_zeros((B, 0, Tq, hq, d), dtype=torch.float32)
+        part_lse = q.new_zeros((B, 0, Tq, hq), dtype=torch.float32)
+    # pack [per][B][Tq][hq][d + 1]; ranks with fewer shards pad with empty ones (lse -inf)
+    packed = torch.zeros((per, B, Tq, hq, d + 1), dtype=torch.float32, device=q.device)
+    packed[..., d] = float("-inf")
+    if n_local:
+        packed[:n_local, ..., :d] = part_o.permute(1, 0, 2, 3, 4)
+        packed[:n_local, ..., d] = part_lse.permute(1, 0, 2, 3)
+    gathered = torch.empty((world * per,) + tuple(packed.shape[1:]), dtype=torch.float32, device=q.device)
+    dist.all_gather_into_tensor(gathered, packed, group=group)
+    all_o = gathered[..., :d].permute(1, 0, 2, 3, 4).contiguous()      # [B][world*per][Tq][hq][d]
+    all_lse = gathered[..., d].permute(1, 0, 2, 3).contiguous()        # [B][world*per][Tq][hq]
+    return merge_fn(all_o, all_lse, q.dtype)

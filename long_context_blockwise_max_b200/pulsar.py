@@ -27,7 +27,7 @@ ABI_SYMBOLS = (
     "pa_select_workspace_size", "pulsar_select_summaries", "pulsar_select_summaries_noalloc",
     "pulsar_select_summaries_scored",
     "pa_phase1_layout", "pa_phase1_workspace_size", "pulsar_phase1_encode", "star_phase1_encode",
-    "pa_phase2_workspace_size", "star_phase2_attend",
+    "pa_phase2_workspace_size", "star_phase2_attend", "star_phase2_query_step", "pa_lse_merge",
 )
 
 
@@ -63,6 +63,9 @@ def _load() -> ctypes.CDLL:
         "pa_phase2_workspace_size": (SZ, [I32, I32, I64, I32, I32, I32, I32]),
         "star_phase2_attend": (ctypes.c_int, [P, ctypes.c_int, I32, I32, I64, D, P, P, I64, I32, I32, I32,
                                               I32, P, P, P, P, P, SZ, P]),
+        "pa_lse_merge": (ctypes.c_int, [P, P, I32, I32, I32, I32, I32, ctypes.c_int, P, P, P]),
+        "star_phase2_query_step": (ctypes.c_int, [P, P, P, ctypes.c_int, I32, I32, I64, D, P, P, I64, I32, P, P,
+                                                  I64, I64, I32, I32, I32, P, P, P, SZ, P]),
     }
     # test hook (include/pulsar_testing.h)
     sig["pa_testing_phase1_stall"] = (ctypes.c_int, [P, P, P, I64, I32, I32, I32, I32, P, P, P, P, SZ, I32, P])
@@ -277,6 +280,43 @@ def star_phase2_attend(q, k_ret, v_ret, n_shards, q_pos0=0, rope_theta=0.0, o=No
                                  _ptr(ws), ws.numel() * ws.element_size(), _stream())
     _check(rc, "star_phase2_attend")
     return o, lse, part_o, part_lse, ws
+
+
+def pa_lse_merge(part_o, part_lse, dtype=torch.bfloat16, o=None, lse=None):
+    """Exact merge of partials part_o [B][S][Tq][hq][d], part_lse [B][S][Tq][hq]
+    (float32, on the GPU).  Returns (o in ``dtype``, lse)."""
+    _dev(part_o, part_lse, o, lse)
+    B, S, Tq, hq, d = part_o.shape
+    if o is None:
+        o = torch.empty((B, Tq, hq, d), dtype=dtype, device=part_o.device)
+    if lse is None:
+        lse = torch.empty((B, Tq, hq), dtype=torch.float32, device=part_o.device)
+    rc = _lib.pa_lse_merge(_ptr(part_o), _ptr(part_lse), B, S, Tq, hq, d, _dtype_code(o), _ptr(o), _ptr(lse),
+                           _stream())
+    _check(rc, "pa_lse_merge")
+    return o, lse
+
+
+def star_phase2_query_step(q, k_new, v_new, k_ret, v_ret, n_shards, k_self, v_self, self_len, q_pos0,
+                           rope_theta, o=None, lse=None, ws=None):
+    """Query-host step: append the new tokens' K/V (K rotated at q_pos0 + j)
+    to the own cache at rows self_len + j, then attend (shards + own keys
+    0..self_len + j, causal).  q/k_new/v_new [B][Tq][h][d]; caches
+    [B][T][hkv][d]; k_self/v_self [B][cap][hkv][d].  Returns (o, lse, ws)."""
+    _dev(q, k_new, v_new, k_ret, v_ret, k_self, v_self, o, lse)
+    B, Tq, hq, d = q.shape
+    T, hkv = k_ret.shape[1], k_ret.shape[2]
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Tq, hq), dtype=torch.float32, device=q.device)
+    ws = _workspace(pa_phase2_workspace_size(B, Tq, T, n_shards, hq, hkv, d), q.device, ws)
+    rc = _lib.star_phase2_query_step(_ptr(q), _ptr(k_new), _ptr(v_new), _dtype_code(q), B, Tq, int(q_pos0),
+                                     float(rope_theta), _ptr(k_ret), _ptr(v_ret), T, n_shards, _ptr(k_self),
+                                     _ptr(v_self), k_self.shape[1], int(self_len), hq, hkv, d, _ptr(o), _ptr(lse),
+                                     _ptr(ws), ws.numel() * ws.element_size(), _stream())
+    _check(rc, "star_phase2_query_step")
+    return o, lse, ws
 
 
 def pa_testing_phase1_stall(q, k, v, block, wait_limit_us):

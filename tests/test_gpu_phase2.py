@@ -101,3 +101,19 @@ def test_query_128k_sampled_groups(P):
         hs = slice(kvh * g, (kvh + 1) * g)
         assert_close(f64(o[:, :, hs].cpu()), ro, O_TOL[torch.bfloat16], "O")
         assert_close(lse[:, :, hs].cpu().double().numpy(), rl, LSE_TOL, "lse")
+
+
+def test_lse_merge_entry_point(P):
+    # partials from star_phase2_attend, merged again by pa_lse_merge, give the
+    # same O / lse; an all-empty row merges to O = 0, lse = -inf
+    B, Tq, hq, hkv, d, T, S = 2, 3, 8, 2, 128, 1000, 5
+    q = workloads.normal((B, Tq, hq, d), 70, torch.bfloat16).to(DEV)
+    kc = workloads.normal((B, T, hkv, d), 71, torch.bfloat16).to(DEV)
+    vc = workloads.normal((B, T, hkv, d), 72, torch.bfloat16).to(DEV)
+    o, lse, po, pl, _ = P.star_phase2_attend(q, kc, vc, S, q_pos0=T, rope_theta=1e4, want_partials=True)
+    o2, lse2 = P.pa_lse_merge(po, pl, dtype=torch.bfloat16)
+    assert (o2.float() - o.float()).abs().max().item() <= 1e-2
+    assert (lse2 - lse).abs().max().item() <= 1e-5
+    pl_empty = torch.full_like(pl, float("-inf"))
+    o3, lse3 = P.pa_lse_merge(torch.zeros_like(po), pl_empty, dtype=torch.float32)
+    assert (o3 == 0).all() and torch.isneginf(lse3).all()
