@@ -37,7 +37,6 @@ using namespace sm100;
 
 namespace {
 
-constexpr int kEmuSlot = -1;  // element pairs i with i % 4 == kEmuSlot use exp2_fma2 (-1: none)
 
 template <int D>
 struct TcCfg {
@@ -99,30 +98,6 @@ __device__ void decode_item(const HostTable& ht, int hkv, int pairs, int idx, in
   const int rem = idx % (nt * pairs);
   *tile = nt - 1 - rem / pairs;
   *pair = rem % pairs;
-}
-
-// 2^x for two values at once on the FMA pipe (packed f32x2), used for part
-// of the softmax so that the MUFU unit is not the only source of
-// exponentials.  x = j + f with j the nearest integer (adding 1.5 * 2^23
-// leaves j in the low mantissa bits) and f in [-0.5, 0.5]; 2^f = e^(f ln 2)
-// by its Taylor series to degree 4 (relative error below 5e-5 on that
-// interval); j is then added to the exponent field.  Inputs are clamped at
-// -125 so that the result stays a normal float.
-__device__ __forceinline__ void exp2_fma2(float x0, float x1, float& y0, float& y1) {
-  const uint64_t x = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
-  const uint64_t t = f2_add(x, f2_pack(12582912.f, 12582912.f));
-  const uint64_t r = f2_add(t, f2_pack(-12582912.f, -12582912.f));
-  const uint64_t f = f2_fma(r, f2_pack(-1.f, -1.f), x);
-  uint64_t p = f2_fma(f2_pack(9.6181291076284772e-3f, 9.6181291076284772e-3f), f,      // (ln 2)^4 / 4!
-                      f2_pack(5.5504108664821580e-2f, 5.5504108664821580e-2f));        // (ln 2)^3 / 3!
-  p = f2_fma(p, f, f2_pack(2.4022650695910071e-1f, 2.4022650695910071e-1f));          // (ln 2)^2 / 2!
-  p = f2_fma(p, f, f2_pack(6.9314718055994531e-1f, 6.9314718055994531e-1f));          // ln 2
-  p = f2_fma(p, f, f2_pack(1.f, 1.f));
-  float p0, p1, t0, t1;
-  f2_unpack(p, p0, p1);
-  f2_unpack(t, t0, t1);
-  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -352,12 +327,8 @@ __global__ void __launch_bounds__(384, 1) phase1_tc_kernel(const __grid_constant
           float x0, x1, p0, p1;
           f2_unpack(f2_add(f2_pack(__uint_as_float(sr[32 * c + 2 * i]), __uint_as_float(sr[32 * c + 2 * i + 1])),
                            nm2), x0, x1);
-          if (!diag && (i & 3) == kEmuSlot) {
-            exp2_fma2(x0, x1, p0, p1);          // FMA pipe
-          } else {
-            p0 = fast_exp2(x0);                 // MUFU
-            p1 = fast_exp2(x1);
-          }
+          p0 = fast_exp2(x0);
+          p1 = fast_exp2(x1);
           acc2[i & 3] = f2_add(acc2[i & 3], f2_pack(p0, p1));
           pk[i] = pack_bf16x2(p0, p1);
         }
