@@ -31,4 +31,5 @@ from .pulsar_oracle import (  # noqa: F401
     select_evenly_spaced,
     select_summaries_mean_idf,
     phase2_attend_with_self,
+    phase2_attend_art,
 )

@@ -431,3 +431,74 @@ def phase2_attend_with_self(q, k_cache, v_cache, n_shards: int, k_self, v_self, 
                 A_self[b, 0, j, head] = (e @ vs[b, :n, head // g, :]) / e.sum()
                 s_self[b, 0, j, head] = mx + np.log(e.sum())
     return lse_merge(np.concatenate([A, A_self], axis=1), np.concatenate([s, s_self], axis=1))
+
+
+def phase2_attend_art(q, k_cache, v_cache, q_pos0: int, theta: float, block_keys: int = 128,
+                      tau: float = 1e-5, phi: float = 1e-3, patience: int = 5):
+    """Run-time early termination of the key traversal (ART review page:
+    "Attention Run-time Termination" -- stop walking the KV cache once a
+    probe of the running attention output has been stable in magnitude and
+    direction for `patience` consecutive blocks; defaults tau = 1e-5,
+    phi = 1e-3, p = 5; reverse-temporal traversal).
+
+    Readings: blocks of `block_keys` keys from the newest backwards
+    (block 1 = keys [T - block_keys, T)); the probe x_t is the full
+    normalised running output after block t; step t >= 2 is stable when
+    | |x_t| - |x_{t-1}| | <= tau |x_{t-1}| and 1 - cos(x_t, x_{t-1}) <= phi;
+    a (batch, kv head) group stops after block t when its last `patience`
+    steps were stable for every query row of the group (Tq tokens x the
+    group's query heads); otherwise every block is visited.
+
+    q: [B][Tq][Hq][d] pre-RoPE (rotated at q_pos0 + j when theta > 0);
+    caches [B][T][Hkv][d] with K rotated.  Returns (O, lse over the visited
+    keys, visited block counts [B][Hkv])."""
+    q = np.asarray(q, dtype=np.float64)
+    B, Tq, hq, d = q.shape
+    if theta > 0:
+        pos = q_pos0 + np.arange(Tq)
+        q = np.stack([rope(q[b], pos, theta) for b in range(B)])
+    kc = np.asarray(k_cache, np.float64)
+    vc = np.asarray(v_cache, np.float64)
+    T, hkv = kc.shape[1], kc.shape[2]
+    g = hq // hkv
+    scale = 1.0 / math.sqrt(d)
+    n_blocks = -(-T // block_keys) if T else 0
+    O = np.zeros((B, Tq, hq, d))
+    lse = np.full((B, Tq, hq), -np.inf)
+    visited = np.zeros((B, hkv), dtype=np.int64)
+    for b in range(B):
+        for kvh in range(hkv):
+            heads = list(range(kvh * g, (kvh + 1) * g))
+            m = np.full((Tq, g), -np.inf)
+            l = np.zeros((Tq, g))
+            acc = np.zeros((Tq, g, d))
+            prev = None
+            run = 0
+            t = 0
+            while t < n_blocks:
+                t += 1
+                lo, hi = max(T - t * block_keys, 0), T - (t - 1) * block_keys
+                for jj in range(Tq):
+                    for hh, head in enumerate(heads):
+                        sc = (kc[b, lo:hi, kvh, :] @ q[b, jj, head, :]) * scale
+                        mn = max(m[jj, hh], sc.max())
+                        c_old = math.exp(m[jj, hh] - mn) if m[jj, hh] > -np.inf else 0.0
+                        e = np.exp(sc - mn)
+                        l[jj, hh] = l[jj, hh] * c_old + e.sum()
+                        acc[jj, hh] = acc[jj, hh] * c_old + e @ vc[b, lo:hi, kvh, :]
+                        m[jj, hh] = mn
+                x = acc / l[..., None]
+                if prev is not None:
+                    nx = np.linalg.norm(x, axis=-1)
+                    npv = np.linalg.norm(prev, axis=-1)
+                    cos = (x * prev).sum(-1) / (nx * npv)
+                    stable = (np.abs(nx - npv) <= tau * npv) & (1.0 - cos <= phi)
+                    run = run + 1 if stable.all() else 0
+                prev = x
+                if run >= patience:
+                    break
+            visited[b, kvh] = t
+            for hh, head in enumerate(heads):
+                O[b, :, head, :] = acc[:, hh, :] / l[:, hh, None] if t else 0.0
+                lse[b, :, head] = (m[:, hh] + np.log(l[:, hh])) if t else -np.inf
+    return O, lse, visited

@@ -209,3 +209,31 @@ def test_query_step_without_context_is_causal_attention():
     o, _ = oracle.phase2_attend_with_self(q, np.zeros((B, 0, hkv, d)), np.zeros((B, 0, hkv, d)), 2, ks, vs, 0,
                                           0, 0.0)
     np.testing.assert_allclose(o[0], _sdpa(q[0], ks[0], vs[0], True), rtol=0, atol=1e-12)
+
+
+def test_art_never_stable_equals_exact_attention():
+    # thresholds of zero: no step is stable, every block is visited, and the
+    # result is exact attention over the whole cache
+    B, Tq, hq, hkv, d, T = 2, 1, 4, 2, 16, 300
+    q = _rand((B, Tq, hq, d), 90)
+    kc, vc = _rand((B, T, hkv, d), 91), _rand((B, T, hkv, d), 92)
+    o, lse, visited = oracle.phase2_attend_art(q, kc, vc, 0, 0.0, block_keys=64, tau=0.0, phi=0.0, patience=3)
+    assert (visited == 5).all()
+    for b in range(B):
+        np.testing.assert_allclose(o[b], _sdpa(q[b], kc[b], vc[b], False), rtol=0, atol=1e-12)
+
+
+def test_art_stops_after_patience_when_old_keys_carry_no_weight():
+    # keys older than the newest block score -1000 below it: their weights
+    # underflow to exactly 0, every later step is exactly stable, so the walk
+    # stops after 1 + patience blocks and equals attention over the newest block
+    B, Tq, hq, hkv, d, T, bk, pat = 1, 2, 2, 1, 8, 64 * 10, 64, 3
+    q = np.zeros((B, Tq, hq, d))
+    q[..., 0] = 1.0
+    kc = _rand((B, T, hkv, d), 93) * 0.1
+    kc[0, :T - bk, 0, 0] = -1000.0 * np.sqrt(d)      # q.k / sqrt(d) = -1000 for old keys
+    vc = _rand((B, T, hkv, d), 94)
+    o, lse, visited = oracle.phase2_attend_art(q, kc, vc, 0, 0.0, block_keys=bk, tau=1e-5, phi=1e-3, patience=pat)
+    assert visited[0, 0] == 1 + pat
+    want = _sdpa(q[0], kc[0, T - bk:], vc[0, T - bk:], False)
+    np.testing.assert_allclose(o[0], want, rtol=0, atol=1e-12)
