@@ -385,6 +385,28 @@ def run_ours(args, rank, world, local_rank, dist_on):
             "kernel_gb_s": round(kv_bytes / (dec_kernel_ms * 1e-3) / 1e9, 1),
             "frac_hbm": round(kv_bytes / (dec_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
             "bytes_per_call": kv_bytes}
+        # ART early termination on the same decode (the page's defaults)
+        ao = torch.empty_like(dq)
+        al = torch.empty((B, 1, DECODE.hq), dtype=torch.float32, device=dev)
+        aws = torch.empty(P.pa_phase2_workspace_size(B, 1, T, 1, DECODE.hq, DECODE.hkv, DECODE.d),
+                          dtype=torch.uint8, device=dev)
+
+        def art():
+            return P.star_phase2_attend_art(dq, dk, dv, T, DECODE.rope_theta, o=ao, lse=al, ws=aws)
+        for _ in range(3):
+            art()
+        torch.cuda.synchronize()
+        r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        r0.record()
+        for _ in range(K):
+            _, _, vis, _ = art()
+        r1.record()
+        torch.cuda.synchronize()
+        art_ms = r0.elapsed_time(r1) / K
+        frac = float(vis.float().mean().item()) * 128 / T
+        extra["phase2_decode_art"] = {"ms": round(art_ms, 4), "visited_fraction": round(frac, 4),
+                                      "gb_s_of_visited": round(kv_bytes * frac / (art_ms * 1e-3) / 1e9, 1),
+                                      "tau": 1e-5, "phi": 1e-3, "patience": 5, "block_keys": 128}
         del dq, dk, dv
         torch.cuda.empty_cache()
 

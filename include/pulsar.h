@@ -277,6 +277,31 @@ int star_phase2_attend(const void* q, int dtype, int32_t B, int32_t Tq, int64_t 
                        void* stream);
 
 /*
+ * Phase-2 attention with run-time early termination of the key walk (NEXT
+ * row; "ART: Attention Run-time Termination" review page: stop fetching
+ * further KV blocks once a probe of the running output has been stable in
+ * magnitude and direction for a patience window; defaults tau = 1e-5,
+ * phi = 1e-3, patience = 5).  An approximation: its result is attention
+ * over the keys visited.  For every (batch, kv head) group the cache is
+ * walked from the newest key backwards in blocks of block_keys keys; after
+ * block t >= 2 the step is stable when, for every query row of the group
+ * (Tq tokens x the group's query heads), the normalised running output x_t
+ * satisfies | |x_t| - |x_{t-1}| | <= tau |x_{t-1}| and 1 - cos(x_t, x_{t-1})
+ * <= phi; the walk stops after `patience` consecutive stable steps.
+ *  q              [B][Tq][hq][d] bf16 (rotated at q_pos0 + j when rope_theta > 0).
+ *  k_ret, v_ret   [B][T][hkv][d] bf16, K rotated.
+ *  o, lse         out: attention over the visited keys.
+ *  visited_blocks_opt  out [B][hkv] int32: blocks walked, or NULL.
+ * bf16 only; Tq * hq / hkv <= 8 (decode rows); block_keys a multiple of 32;
+ * workspace pa_phase2_workspace_size(B, Tq, T, 1, hq, hkv, d).
+ */
+int star_phase2_attend_art(const void* q, int dtype, int32_t B, int32_t Tq, int64_t q_pos0,
+                           double rope_theta, const void* k_ret, const void* v_ret, int64_t T,
+                           int32_t hq, int32_t hkv, int32_t d, int32_t block_keys, double tau,
+                           double phi, int32_t patience, void* o, float* lse,
+                           int32_t* visited_blocks_opt, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Exact merge of Phase-2 partials ([S] Algorithm 2 as corrected in the
  * referee's comment; [P] §2.2 "an all_gather followed by an online-softmax
  * merge"), for partials gathered from several GPUs:

@@ -336,6 +336,48 @@ int star_phase2_attend(const void* q, int dtype, int32_t B, int32_t Tq, int64_t 
   return launch_phase2(a, s);
 }
 
+int star_phase2_attend_art(const void* q, int dtype, int32_t B, int32_t Tq, int64_t q_pos0,
+                           double rope_theta, const void* k_ret, const void* v_ret, int64_t T,
+                           int32_t hq, int32_t hkv, int32_t d, int32_t block_keys, double tau,
+                           double phi, int32_t patience, void* o, float* lse,
+                           int32_t* visited_blocks_opt, void* ws, size_t ws_bytes, void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int rc = check_heads(hq, hkv, d, dtype);
+  if (rc) return rc;
+  if (dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+  if (B < 0 || Tq < 0 || T < 0 || !std::isfinite(rope_theta)) return PA_ERR_INVALID;
+  if (block_keys < 32 || block_keys % 32 != 0 || patience < 1 || !(tau >= 0) || !(phi >= 0))
+    return PA_ERR_INVALID;
+  if ((int64_t)Tq * (hq / hkv) > 8) return PA_ERR_UNSUPPORTED;
+  if (B > 0 && Tq > 0 && (!q || !o || !lse || (T > 0 && (!k_ret || !v_ret)))) return PA_ERR_INVALID;
+  const void* ptrs[] = {q, k_ret, v_ret, o};
+  for (const void* p : ptrs)
+    if (p && !aligned(p, 16)) return PA_ERR_UNSUPPORTED;
+  const size_t need = phase2_workspace_bytes(B, Tq, T, 1, hq, hkv, d);
+  rc = check_ws(ws, ws_bytes, need);
+  if (rc) return rc;
+  rc = clear_status(ws, s);
+  if (rc) return rc;
+  Phase2Args a;
+  a.dtype = dtype;
+  a.q = q; a.B = B; a.Tq = Tq; a.q_pos0 = q_pos0; a.rope_theta = rope_theta;
+  a.k_ret = k_ret; a.v_ret = v_ret; a.T = T;
+  a.n_shards = 1; a.n_split = 1;
+  a.hq = hq; a.hkv = hkv; a.d = d;
+  a.o = o; a.lse = lse; a.part_o_opt = nullptr; a.part_lse_opt = nullptr;
+  carve_phase2(a, ws);
+  if (B == 0 || Tq == 0) return PA_OK;
+  ArtArgs art;
+  art.block_keys = block_keys;
+  art.tau = static_cast<float>(tau);
+  art.phi = static_cast<float>(phi);
+  art.patience = patience;
+  art.visited = visited_blocks_opt;
+  rc = launch_rope_query(a, s);
+  if (rc) return rc;
+  return launch_phase2_art(a, art, s);
+}
+
 int pa_lse_merge(const float* part_o, const float* part_lse, int32_t B, int32_t S, int32_t Tq,
                  int32_t hq, int32_t d, int dtype, void* o, float* lse, void* stream) {
   if (B < 0 || S < 1 || Tq < 0 || hq < 1) return PA_ERR_INVALID;

@@ -146,6 +146,16 @@ __device__ inline UnitView phase2_unit(const Phase2Args& a, int u) {
   return v;
 }
 int launch_phase2_mma(const Phase2Args& a, cudaStream_t s);
+
+// ART early termination of the Phase-2 key walk (one warp per (b, kv head)).
+struct ArtArgs {
+  int block_keys;        // keys per stability check (multiple of 32)
+  float tau, phi;        // magnitude / direction thresholds
+  int patience;          // consecutive stable blocks before stopping
+  int32_t* visited;      // [B][hkv] blocks visited, or null
+};
+int launch_phase2_art(const Phase2Args& a, const ArtArgs& art, cudaStream_t s);
+int launch_rope_query(const Phase2Args& a, cudaStream_t s);
 int32_t phase2_split(int32_t B, int32_t Tq, int64_t T, int32_t n_shards, int32_t hq,
                      int32_t hkv);
 size_t phase2_workspace_bytes(int32_t B, int32_t Tq, int64_t T, int32_t n_shards, int32_t hq,

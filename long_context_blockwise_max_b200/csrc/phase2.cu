@@ -312,6 +312,25 @@ int launch_self_append(const Phase2Args& a, const void* k_new, const void* v_new
   return launch_self_append_t<__nv_bfloat16>(a, k_new, v_new, s);
 }
 
+int launch_rope_query(const Phase2Args& a, cudaStream_t s) {
+  RopeFreqs f;
+  for (int m = 0; m < kMaxHalfDim; ++m)
+    f.omega[m] = (m < a.d / 2 && a.rope_theta > 0) ? pow(a.rope_theta, -2.0 * m / a.d) : 0.0;
+  const float qscale = (float)(kLog2e / sqrt((double)a.d));
+  const int64_t nq = (int64_t)a.B * a.Tq * a.hq * (a.d / 2);
+  if (nq > 0) {
+    const int64_t want = (nq + 255) / 256;
+    if (a.dtype == PA_F32)
+      rope_query_kernel<float><<<(int)(want < 148 * 8 ? want : 148 * 8), 256, 0, s>>>(
+          static_cast<const float*>(a.q), a.B, a.Tq, a.hq, a.d, a.q_pos0, a.rope_theta > 0, f, qscale, a.qr);
+    else
+      rope_query_kernel<__nv_bfloat16><<<(int)(want < 148 * 8 ? want : 148 * 8), 256, 0, s>>>(
+          static_cast<const __nv_bfloat16*>(a.q), a.B, a.Tq, a.hq, a.d, a.q_pos0, a.rope_theta > 0, f, qscale,
+          a.qr);
+  }
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
 int launch_merge_only(const Phase2Args& a, cudaStream_t s) {
   const int64_t nrows = (int64_t)a.B * a.Tq * a.hq;
   if (nrows > 0) {

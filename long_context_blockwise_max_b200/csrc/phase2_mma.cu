@@ -433,6 +433,203 @@ __global__ void __launch_bounds__(kWarps * 32) phase2_mma_rows_kernel(Phase2Args
   if ((lane & 3) == 0) a.unit_lse[orow] = empty ? -INFINITY : (m_run + __log2f(l_run)) * kLn2f;
 }
 
+// ---------------------------------------------------------------------------
+// ART (run-time early termination, ART review page): one warp per (batch,
+// kv head) walks the cache from the newest key backwards in 32-key tiles
+// through an 8-stage cp.async ring; after every block of `block_keys` keys
+// it compares the normalised running output of each query row with the
+// previous block's (magnitude change <= tau * |x_prev|, 1 - cos <= phi) and
+// stops once `patience` consecutive blocks were stable for every row.
+// ---------------------------------------------------------------------------
+constexpr int kArtStages = 8;
+
+template <int D>
+__global__ void __launch_bounds__(32) phase2_art_kernel(Phase2Args a, ArtArgs art) {
+  using C = P2Cfg<D>;
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int lane = threadIdx.x;
+  const int b = blockIdx.x, kvh = blockIdx.y;
+  const int g = a.hq / a.hkv;
+  const int R = a.Tq * g;
+  const int qi = lane >> 2, qc = (lane & 3) * 2;
+  const bool row_ok = qi < R;
+  const int t_row = row_ok ? qi / g : 0;
+  const int head = kvh * g + (row_ok ? qi % g : 0);
+  uint32_t qa[D / 16][4];
+  {
+    const float* qp = a.qr + (((int64_t)b * a.Tq + t_row) * a.hq + head) * D;
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      float x[4];
+      x[0] = row_ok ? qp[16 * ks + qc] : 0.f;
+      x[1] = row_ok ? qp[16 * ks + qc + 1] : 0.f;
+      x[2] = row_ok ? qp[16 * ks + qc + 8] : 0.f;
+      x[3] = row_ok ? qp[16 * ks + qc + 9] : 0.f;
+      float h[4], l[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        h[e] = __bfloat162float(__float2bfloat16_rn(x[e]));
+        l[e] = x[e] - h[e];
+      }
+      qa[ks][0] = pack_bf16(h[0], h[1]);
+      qa[ks][1] = pack_bf16(l[0], l[1]);
+      qa[ks][2] = pack_bf16(h[2], h[3]);
+      qa[ks][3] = pack_bf16(l[2], l[3]);
+    }
+  }
+  const int64_t T = a.T;
+  const int n_tiles = static_cast<int>((T + kKT - 1) / kKT);
+  const int tiles_per_block = art.block_keys / kKT;
+  const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+  const __nv_bfloat16* Kg = static_cast<const __nv_bfloat16*>(a.k_ret);
+  const __nv_bfloat16* Vg = static_cast<const __nv_bfloat16*>(a.v_ret);
+  const int64_t key_stride = (int64_t)a.hkv * D;
+  const int64_t base_off = ((int64_t)b * T) * key_stride + (int64_t)kvh * D;
+  // tile s covers keys [T - 32 (s + 1), T - 32 s), clipped at 0
+  auto issue = [&](int it) {
+    if (it < n_tiles) {
+      const int64_t key0 = T - (int64_t)kKT * (it + 1);
+      const uint32_t sbase = base + (it % kArtStages) * C::STAGE;
+#pragma unroll
+      for (int e = 0; e < (kKT * C::CH) / 32; ++e) {
+        const int idx = e * 32 + lane;
+        const int key = idx / C::CH, ch = idx % C::CH;
+        const int64_t kg = key0 + key;
+        const bool valid = kg >= 0;
+        const int64_t off = base_off + (valid ? kg : 0) * key_stride + ch * 8;
+        cp_async16(sbase + swz<D>(key, ch), Kg + off, valid);
+        cp_async16(sbase + C::TILE + swz<D>(key, ch), Vg + off, valid);
+      }
+    }
+    cp_async_commit();
+  };
+  float o[D / 8][4];
+#pragma unroll
+  for (int j = 0; j < D / 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+  float prev[D / 8][2];
+#pragma unroll
+  for (int j = 0; j < D / 8; ++j) prev[j][0] = prev[j][1] = 0.f;
+  float prev_sq = 0.f;
+  float m_run = -INFINITY, l_run = 0.f;
+  int run = 0, blocks = 0;
+#pragma unroll
+  for (int s2 = 0; s2 < kArtStages - 1; ++s2) issue(s2);
+  int it = 0;
+  for (; it < n_tiles; ++it) {
+    issue(it + kArtStages - 1);
+    cp_async_wait<kArtStages - 1>();
+    __syncwarp();
+    const uint32_t sK = base + (it % kArtStages) * C::STAGE;
+    const uint32_t sV = sK + C::TILE;
+    const int64_t key0 = T - (int64_t)kKT * (it + 1);
+    float sc[4][4];
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+#pragma unroll
+      for (int kk = 0; kk < D / 32; ++kk) {
+        uint32_t b0, b1, b2, b3;
+        const int key = nt * 8 + (lane & 7);
+        const int ch = kk * 4 + (lane >> 3);
+        ldsm_x4(sK + swz<D>(key, ch), b0, b1, b2, b3);
+        mma_bf16(sc[nt], qa[2 * kk][0], qa[2 * kk][1], qa[2 * kk][2], qa[2 * kk][3], b0, b1);
+        mma_bf16(sc[nt], qa[2 * kk + 1][0], qa[2 * kk + 1][1], qa[2 * kk + 1][2], qa[2 * kk + 1][3], b2, b3);
+      }
+    }
+    float sv[4][2];
+    float mt = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int64_t kg = key0 + nt * 8 + qc + e;
+        const float x = (kg >= 0) ? sc[nt][e] + sc[nt][e + 2] : -INFINITY;
+        sv[nt][e] = x;
+        mt = fmaxf(mt, x);
+      }
+    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
+    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
+    const float m_new = fmaxf(m_run, mt);
+    const float alpha = fast_exp2(m_run - m_new);
+    m_run = m_new;
+    l_run *= alpha;
+#pragma unroll
+    for (int j = 0; j < D / 8; ++j) {
+      o[j][0] *= alpha;
+      o[j][1] *= alpha;
+    }
+    uint32_t pa_[4];
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+      const float p0 = fast_exp2(sv[nt][0] - m_new), p1 = fast_exp2(sv[nt][1] - m_new);
+      l_run += p0 + p1;
+      pa_[nt] = pack_bf16(p0, p1);
+    }
+#pragma unroll
+    for (int k2 = 0; k2 < 2; ++k2) {
+#pragma unroll
+      for (int cj = 0; cj < D / 16; ++cj) {
+        uint32_t b0, b1, b2, b3;
+        const int mtx = lane >> 3;
+        const int key = k2 * 16 + (mtx & 1) * 8 + (lane & 7);
+        const int ch = cj * 2 + (mtx >> 1);
+        ldsm_x4_t(sV + swz<D>(key, ch), b0, b1, b2, b3);
+        mma_bf16(o[2 * cj], pa_[2 * k2], 0u, pa_[2 * k2 + 1], 0u, b0, b1);
+        mma_bf16(o[2 * cj + 1], pa_[2 * k2], 0u, pa_[2 * k2 + 1], 0u, b2, b3);
+      }
+    }
+    __syncwarp();
+    // end of a block (or of the cache): stability of the normalised output
+    if ((it + 1) % tiles_per_block == 0 || it + 1 == n_tiles) {
+      ++blocks;
+      float l_tot = l_run;
+      l_tot += __shfl_xor_sync(0xffffffffu, l_tot, 1);
+      l_tot += __shfl_xor_sync(0xffffffffu, l_tot, 2);
+      const float inv = 1.f / l_tot;
+      float sq = 0.f, dot = 0.f;
+#pragma unroll
+      for (int j = 0; j < D / 8; ++j) {
+        const float x0 = o[j][0] * inv, x1 = o[j][1] * inv;
+        sq = fmaf(x0, x0, fmaf(x1, x1, sq));
+        dot = fmaf(x0, prev[j][0], fmaf(x1, prev[j][1], dot));
+        prev[j][0] = x0;
+        prev[j][1] = x1;
+      }
+      sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+      sq += __shfl_xor_sync(0xffffffffu, sq, 2);
+      dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+      dot += __shfl_xor_sync(0xffffffffu, dot, 2);
+      bool stable = true;
+      if (blocks >= 2 && row_ok) {
+        const float nx = sqrtf(sq), np = sqrtf(prev_sq);
+        stable = fabsf(nx - np) <= art.tau * np && 1.f - dot / (nx * np) <= art.phi;
+      } else if (row_ok) {
+        stable = false;
+      }
+      prev_sq = sq;
+      run = __all_sync(0xffffffffu, stable) ? run + 1 : 0;
+      if (run >= art.patience) {
+        ++it;
+        break;
+      }
+    }
+  }
+  cp_async_wait<0>();
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+  if (lane == 0 && art.visited) art.visited[(int64_t)b * a.hkv + kvh] = blocks;
+  if (!row_ok) return;
+  const bool empty = (m_run == -INFINITY);
+  const float inv = empty ? 0.f : 1.f / l_run;
+  const int64_t orow = ((int64_t)b * a.Tq + t_row) * a.hq + head;
+  __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.o) + orow * D;
+#pragma unroll
+  for (int j = 0; j < D / 8; ++j)
+    *reinterpret_cast<__nv_bfloat162*>(dst + 8 * j + qc) = __floats2bfloat162_rn(o[j][0] * inv, o[j][1] * inv);
+  if ((lane & 3) == 0) a.lse[orow] = empty ? -INFINITY : (m_run + __log2f(l_run)) * kLn2f;
+}
+
 template <int D>
 int launch_d(const Phase2Args& a, cudaStream_t s) {
   const int g = a.hq / a.hkv;
@@ -465,6 +662,25 @@ int launch_d(const Phase2Args& a, cudaStream_t s) {
 
 int launch_phase2_mma(const Phase2Args& a, cudaStream_t s) {
   return a.d == 128 ? launch_d<128>(a, s) : launch_d<64>(a, s);
+}
+
+int launch_phase2_art(const Phase2Args& a, const ArtArgs& art, cudaStream_t s) {
+  const dim3 grid(a.B, a.hkv);
+  if (a.B <= 0) return PA_OK;
+  if (a.d == 128) {
+    const int sm = kArtStages * P2Cfg<128>::STAGE;
+    if (cudaFuncSetAttribute(phase2_art_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm) !=
+        cudaSuccess)
+      return PA_ERR_CUDA;
+    phase2_art_kernel<128><<<grid, 32, sm, s>>>(a, art);
+  } else {
+    const int sm = kArtStages * P2Cfg<64>::STAGE;
+    if (cudaFuncSetAttribute(phase2_art_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm) !=
+        cudaSuccess)
+      return PA_ERR_CUDA;
+    phase2_art_kernel<64><<<grid, 32, sm, s>>>(a, art);
+  }
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 }  // namespace pa

@@ -28,6 +28,7 @@ ABI_SYMBOLS = (
     "pulsar_select_summaries_scored",
     "pa_phase1_layout", "pa_phase1_workspace_size", "pulsar_phase1_encode", "star_phase1_encode",
     "pa_phase2_workspace_size", "star_phase2_attend", "star_phase2_query_step", "pa_lse_merge",
+    "star_phase2_attend_art",
 )
 
 
@@ -63,6 +64,8 @@ def _load() -> ctypes.CDLL:
         "pa_phase2_workspace_size": (SZ, [I32, I32, I64, I32, I32, I32, I32]),
         "star_phase2_attend": (ctypes.c_int, [P, ctypes.c_int, I32, I32, I64, D, P, P, I64, I32, I32, I32,
                                               I32, P, P, P, P, P, SZ, P]),
+        "star_phase2_attend_art": (ctypes.c_int, [P, ctypes.c_int, I32, I32, I64, D, P, P, I64, I32, I32, I32, I32,
+                                                  D, D, I32, P, P, P, P, SZ, P]),
         "pa_lse_merge": (ctypes.c_int, [P, P, I32, I32, I32, I32, I32, ctypes.c_int, P, P, P]),
         "star_phase2_query_step": (ctypes.c_int, [P, P, P, ctypes.c_int, I32, I32, I64, D, P, P, I64, I32, P, P,
                                                   I64, I64, I32, I32, I32, P, P, P, SZ, P]),
@@ -280,6 +283,27 @@ def star_phase2_attend(q, k_ret, v_ret, n_shards, q_pos0=0, rope_theta=0.0, o=No
                                  _ptr(ws), ws.numel() * ws.element_size(), _stream())
     _check(rc, "star_phase2_attend")
     return o, lse, part_o, part_lse, ws
+
+
+def star_phase2_attend_art(q, k_ret, v_ret, q_pos0=0, rope_theta=0.0, block_keys=128, tau=1e-5, phi=1e-3,
+                           patience=5, o=None, lse=None, ws=None):
+    """Phase 2 with run-time early termination of the key walk (newest keys
+    first).  bf16; Tq * hq / hkv <= 8.  Returns (o, lse, visited_blocks [B][hkv], ws)."""
+    _dev(q, k_ret, v_ret, o, lse)
+    B, Tq, hq, d = q.shape
+    T, hkv = k_ret.shape[1], k_ret.shape[2]
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Tq, hq), dtype=torch.float32, device=q.device)
+    visited = torch.empty((B, hkv), dtype=torch.int32, device=q.device)
+    ws = _workspace(pa_phase2_workspace_size(B, Tq, T, 1, hq, hkv, d), q.device, ws)
+    rc = _lib.star_phase2_attend_art(_ptr(q), _dtype_code(q), B, Tq, int(q_pos0), float(rope_theta), _ptr(k_ret),
+                                     _ptr(v_ret), T, hq, hkv, d, int(block_keys), float(tau), float(phi),
+                                     int(patience), _ptr(o), _ptr(lse), _ptr(visited), _ptr(ws),
+                                     ws.numel() * ws.element_size(), _stream())
+    _check(rc, "star_phase2_attend_art")
+    return o, lse, visited, ws
 
 
 def pa_lse_merge(part_o, part_lse, dtype=torch.bfloat16, o=None, lse=None):
