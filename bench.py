@@ -66,24 +66,31 @@ def source_digest(paths):
 
 def recorded_traffic(kernel: str, workload: str):
     """DRAM bytes per launch of `kernel` on `workload` recorded from an ncu
-    capture in profiles/roofline_traffic.txt, or None when there is none or
-    the kernel's sources changed since it was taken."""
+    capture in profiles/roofline_traffic.txt (one record per kernel, each
+    starting at its `kernel` line), or None when there is none or the
+    kernel's sources changed since it was taken."""
     if not os.path.exists(TRAFFIC_FILE):
         return None
-    rec = {}
+    records, rec = [], None
     for line in open(TRAFFIC_FILE):
         line = line.strip()
         if line and not line.startswith("#"):
             key, _, val = line.partition(" ")
-            rec[key] = val.strip()
-    if rec.get("kernel") != kernel or rec.get("workload") != workload:
-        return None
-    try:
-        if source_digest(rec["sources"].split()) != rec["sources_sha256"]:
+            if key == "kernel":
+                rec = {}
+                records.append(rec)
+            if rec is not None:
+                rec[key] = val.strip()
+    for rec in records:
+        if rec.get("kernel") != kernel or rec.get("workload") != workload:
+            continue
+        try:
+            if source_digest(rec["sources"].split()) != rec["sources_sha256"]:
+                return None
+            return int(rec["dram_bytes_read"]) + int(rec["dram_bytes_write"])
+        except (KeyError, OSError, ValueError):
             return None
-        return int(rec["dram_bytes_read"]) + int(rec["dram_bytes_write"])
-    except (KeyError, OSError, ValueError):
-        return None
+    return None
 
 
 # --------------------------------------------------------------------------
@@ -490,7 +497,8 @@ def run_ours(args, rank, world, local_rank, dist_on):
                      "kernel_ms": round(attn_ms, 3), "flop_per_launch": flops},
         "phase1": {"attn_ms": round(attn_ms, 3), "tflop": round(flops / 1e12, 3),
                    "tflop_s": round(attn_tf, 1)},
-        "phase2_query": {"kernel_ms": round(p2_ms, 4), "kv_bytes": q2_bytes,
+        "phase2_query": {"kernel": "phase2_tc_kernel", "kernel_ms": round(p2_ms, 4), "kv_bytes": q2_bytes,
+                         "traffic": recorded_traffic("phase2_tc_kernel", w.name + ":query64"),
                          "gb_s": round(q2_bytes / (p2_ms * 1e-3) / 1e9, 1),
                          "frac_hbm": round(q2_bytes / (p2_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
                          "tflop_s": round(4.0 * w.d * w.hq * w.q_tokens * w.L / (p2_ms * 1e-3) / 1e12, 1)},

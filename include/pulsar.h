@@ -269,6 +269,13 @@ size_t pa_phase2_workspace_size(int32_t B, int32_t Tq, int64_t T, int32_t n_shar
  *
  * An empty shard has s_h = -inf and A_h = 0; with T == 0, O = 0 and
  * lse = -inf.  d must be 64 or 128, hq % hkv == 0, 1 <= n_shards <= 4096.
+ * Precision (bf16): on the tensor-core path (at least 64 query rows per kv
+ * head, Tq * hq / hkv; hq / hkv dividing 128; 16-byte aligned caches) the
+ * scores are computed from the rotated query rounded to fp16 against the
+ * keys converted exactly to fp16 (device status PA_ERR_RANGE if a rotated,
+ * scaled query value or a key is outside fp16 range); otherwise from a bf16
+ * high part plus a bf16 residual of the query, exact against the stored
+ * keys to fp32 rounding.  P is rounded to bf16 for P V.
  */
 int star_phase2_attend(const void* q, int dtype, int32_t B, int32_t Tq, int64_t q_pos0,
                        double rope_theta, const void* k_ret, const void* v_ret, int64_t T,
@@ -303,11 +310,14 @@ int star_phase2_attend_art(const void* q, int dtype, int32_t B, int32_t Tq, int6
 
 /*
  * Exact merge of Phase-2 partials ([S] Algorithm 2 as corrected in the
- * referee's comment; [P] §2.2 "an all_gather followed by an online-softmax
- * merge"), for partials gathered from several GPUs:
+ * referee's comment; [P] §2.2, where the hosts' partial results are
+ * all-gathered and combined by an online softmax), for partials gathered
+ * from several GPUs:
  * lse = ln sum_h exp(s_h), O = sum_h exp(s_h - lse) A_h.
- *  part_o    [B][S][Tq][hq][d] float (A_h, as star_phase2_attend writes it)
- *  part_lse  [B][S][Tq][hq] float (s_h; -inf marks an empty shard)
+ *  part_o    [B][S][Tq][hq][d] float (A_h, as star_phase2_attend writes it),
+ *            16-byte aligned (PA_ERR_INVALID otherwise)
+ *  part_lse  [B][S][Tq][hq] float (s_h; -inf marks an empty shard, whose
+ *            A_h is then ignored)
  *  o         out [B][Tq][hq][d] dtype;  lse out [B][Tq][hq] float.
  * All shards empty: O = 0, lse = -inf.  No workspace.
  */

@@ -384,6 +384,7 @@ int pa_lse_merge(const float* part_o, const float* part_lse, int32_t B, int32_t 
   if (d != 64 && d != 128) return PA_ERR_UNSUPPORTED;
   if (dtype != PA_F32 && dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
   if (B > 0 && Tq > 0 && (!part_o || !part_lse || !o || !lse)) return PA_ERR_INVALID;
+  if ((reinterpret_cast<uintptr_t>(part_o) & 15u) != 0) return PA_ERR_INVALID;   // vector loads
   Phase2Args a;
   a.dtype = dtype;
   a.B = B; a.Tq = Tq; a.hq = hq; a.hkv = hq; a.d = d;

@@ -146,6 +146,11 @@ __device__ inline UnitView phase2_unit(const Phase2Args& a, int u) {
   return v;
 }
 int launch_phase2_mma(const Phase2Args& a, cudaStream_t s);
+// Tensor-core (tcgen05) kernel for queries with at least kPhase2TcMinRows rows
+// per kv head; q16 is the rotated query scaled to log2 units, in fp16.
+constexpr int kPhase2TcMinRows = 64;
+bool phase2_tc_supported(const Phase2Args& a);
+int launch_phase2_tc(const Phase2Args& a, const __half* q16, cudaStream_t s);
 
 // ART early termination of the Phase-2 key walk (one warp per (b, kv head)).
 struct ArtArgs {

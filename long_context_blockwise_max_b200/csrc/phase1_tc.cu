@@ -390,31 +390,9 @@ __global__ void __launch_bounds__(384, 1) phase1_tc_kernel(const __grid_constant
   }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (fn == nullptr) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
-  return fn;
-}
-
-// [rows][heads][d] 16-bit tensor, boxes of 16 rows x 1 head x 64 elements,
-// 128-byte swizzle.
+// [rows][heads][d] 16-bit tensor, boxes of 16 rows x 1 head x 64 elements.
 bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int64_t rows, int heads, int d) {
-  auto enc = encode_fn();
-  if (enc == nullptr) return false;
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(heads),
-                        static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(heads) * d * 2};
-  cuuint32_t box[3] = {64, 1, 16};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return tma_map_3d(m, base, dt, d, heads, rows, 64, 1, 16);
 }
 
 template <int D>
@@ -450,6 +428,37 @@ int launch_tc(const Phase1Args& a, cudaStream_t s) {
 }
 
 }  // namespace
+
+namespace sm100 {
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+bool tma_map_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int64_t dim0, int64_t dim1,
+                int64_t dim2, int box0, int box1, int box2) {
+  auto enc = encode_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(dim0), static_cast<cuuint64_t>(dim1),
+                        static_cast<cuuint64_t>(dim2)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(dim0) * 2, static_cast<cuuint64_t>(dim1) * dim0 * 2};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(box0), static_cast<cuuint32_t>(box1),
+                       static_cast<cuuint32_t>(box2)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace sm100
 
 bool phase1_tc_supported(const Phase1Args& a) {
   const int g = a.hq / a.hkv;

@@ -12,11 +12,15 @@
 namespace pa {
 
 // q [B][Tq][hq][d] -> qr fp32, rotated at q_pos0 + t (theta > 0) and scaled
-// by log2(e)/sqrt(d) so that scores come out in log2 units.
+// by log2(e)/sqrt(d) so that scores come out in log2 units.  With `q16` set,
+// writes that value in fp16 instead (same layout; the operand of the
+// tensor-core query kernel) and sets PA_ERR_RANGE when it is not finite in
+// fp16.
 template <typename IT>
 __global__ void rope_query_kernel(const IT* __restrict__ q, int B, int Tq, int hq, int d,
                                   int64_t q_pos0, int use_rope, RopeFreqs f, float qscale,
-                                  float* __restrict__ qr) {
+                                  float* __restrict__ qr, __half* __restrict__ q16, DeviceStatus* st) {
+  bool bad = false;
   const int half = d / 2;
   const int64_t n = (int64_t)B * Tq * hq * half;
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n;
@@ -34,9 +38,17 @@ __global__ void rope_query_kernel(const IT* __restrict__ q, int B, int Tq, int h
       y1 = x1 * c - x2 * s;
       y2 = x2 * c + x1 * s;
     }
-    qr[base + m] = y1 * qscale;
-    qr[base + m + half] = y2 * qscale;
+    const float z1 = y1 * qscale, z2 = y2 * qscale;
+    if (q16 != nullptr) {
+      q16[base + m] = __float2half_rn(z1);
+      q16[base + m + half] = __float2half_rn(z2);
+      bad |= !(fabsf(z1) <= 65504.f) || !(fabsf(z2) <= 65504.f);
+    } else {
+      qr[base + m] = z1;
+      qr[base + m + half] = z2;
+    }
   }
+  if (bad) set_status(st, PA_ERR_RANGE, 0, 2);
 }
 
 template <int D, typename VT>
@@ -131,84 +143,154 @@ __global__ void __launch_bounds__(256) phase2_simt_kernel(Phase2Args a) {
   if (hf == 0) a.unit_lse[orow] = empty ? -INFINITY : (m_run + __log2f(l_run)) * kLn2f;
 }
 
-// One warp per (b, t, head): merge splits into shard partials, shards into
-// the global result.  s = ln sum exp(s_h) ; O = sum_h exp(s_h - s) A_h.
-template <typename OT>
+// One warp per (b, t, head) row: merge the unit partials (splits of shards,
+// then the own cache) into the global result, and, when asked for, into the
+// shard partials.  s = ln sum_h exp(s_h) ; O = sum_h exp(s_h - s) A_h.
+// Pass 1: the row's log-sum-exp over every unit, lanes over units.  Pass 2:
+// the weighted sum of the units' A, each lane holding D/32 consecutive
+// elements, units unrolled so that their loads are in flight together.
+template <typename OT, int D>
 __global__ void merge_kernel(Phase2Args a) {
+  constexpr int VPL = D / 32;   // 4 or 2 consecutive floats per lane
   const int lane = threadIdx.x & 31;
   const int64_t nrows = (int64_t)a.B * a.Tq * a.hq;
   const int units = phase2_units(a);
-  const int per_lane = a.d / 32;   // 2 or 4
+  const int64_t rs = (int64_t)a.Tq * a.hq;   // unit stride in rows
   for (int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < nrows;
        row += ((int64_t)gridDim.x * blockDim.x) >> 5) {
-    const int64_t b = row / ((int64_t)a.Tq * a.hq), th = row % ((int64_t)a.Tq * a.hq);
-    float gm = -INFINITY, gz = 0.f, gacc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int sh = 0; sh < a.n_shards; ++sh) {
-      float sm = -INFINITY, sz = 0.f, sacc[4] = {0.f, 0.f, 0.f, 0.f};
-      for (int sp = 0; sp < a.n_split; ++sp) {
-        const int u = sh * a.n_split + sp;
-        const int64_t urow = (b * units + u) * (int64_t)a.Tq * a.hq + th;
-        const float s = a.unit_lse[urow];
-        if (s == -INFINITY) continue;
-        const float mn = fmaxf(sm, s);
-        const float c_old = expf(sm - mn), c_new = expf(s - mn);
-        sz = sz * c_old + c_new;
-        const float* A = a.unit_o + urow * a.d;
-        for (int e = 0; e < per_lane; ++e) sacc[e] = sacc[e] * c_old + c_new * A[lane + 32 * e];
-        sm = mn;
+    const int64_t b = row / rs, th = row % rs;
+    const float* lse_u = a.unit_lse + b * units * rs + th;    // unit u at lse_u[u * rs]
+    const float* A_u = a.unit_o + (b * units * rs + th) * D + lane * VPL;
+    // pass 1: row log-sum-exp
+    float m = -INFINITY;
+    for (int u = lane; u < units; u += 32) m = fmaxf(m, lse_u[(int64_t)u * rs]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float z = 0.f;
+    if (m != -INFINITY)
+      for (int u = lane; u < units; u += 32) z += expf(lse_u[(int64_t)u * rs] - m);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    const float s_all = (m == -INFINITY) ? -INFINITY : m + logf(z);
+    float acc[VPL];
+#pragma unroll
+    for (int e = 0; e < VPL; ++e) acc[e] = 0.f;
+    // adds w * A_u; a unit of weight 0 (lse -inf) adds nothing, whatever its A
+    auto add_unit = [&](float* dst, int u, float w) {
+      const float* src = A_u + (int64_t)u * rs * D;
+      const bool on = w > 0.f;
+      if constexpr (VPL == 4) {
+        const float4 v = *reinterpret_cast<const float4*>(src);
+        dst[0] += on ? w * v.x : 0.f;
+        dst[1] += on ? w * v.y : 0.f;
+        dst[2] += on ? w * v.z : 0.f;
+        dst[3] += on ? w * v.w : 0.f;
+      } else {
+        const float2 v = *reinterpret_cast<const float2*>(src);
+        dst[0] += on ? w * v.x : 0.f;
+        dst[1] += on ? w * v.y : 0.f;
       }
-      const float s_h = (sm == -INFINITY) ? -INFINITY : sm + logf(sz);
-      if (a.part_o_opt != nullptr) {
-        const int64_t prow = (b * a.n_shards + sh) * (int64_t)a.Tq * a.hq + th;
-        const float inv = (sm == -INFINITY) ? 0.f : 1.f / sz;
-        for (int e = 0; e < per_lane; ++e) a.part_o_opt[prow * a.d + lane + 32 * e] = sacc[e] * inv;
-        if (lane == 0 && a.part_lse_opt != nullptr) a.part_lse_opt[prow] = s_h;
-      } else if (a.part_lse_opt != nullptr && lane == 0) {
-        a.part_lse_opt[(b * a.n_shards + sh) * (int64_t)a.Tq * a.hq + th] = s_h;
+    };
+    if (s_all != -INFINITY) {
+      if (a.part_o_opt == nullptr && a.part_lse_opt == nullptr) {
+        // pass 2, no shard partials: one flat sum over every unit (an empty
+        // unit has lse -inf, weight 0 and A = 0)
+        int u = 0;
+        for (; u + 4 <= units; u += 4) {
+          float w[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) w[i] = expf(lse_u[(int64_t)(u + i) * rs] - s_all);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) add_unit(acc, u + i, w[i]);
+        }
+        for (; u < units; ++u) add_unit(acc, u, expf(lse_u[(int64_t)u * rs] - s_all));
       }
-      if (s_h == -INFINITY) continue;
-      // fold the shard's (unnormalised) sums into the global accumulator
-      const float mn = fmaxf(gm, sm);
-      const float c_old = expf(gm - mn), c_new = expf(sm - mn);
-      gz = gz * c_old + sz * c_new;
-      for (int e = 0; e < per_lane; ++e) gacc[e] = gacc[e] * c_old + sacc[e] * c_new;
-      gm = mn;
     }
-    if (a.has_self) {   // the own cache's unit (after the shards)
-      const int64_t urow = (b * units + (units - 1)) * (int64_t)a.Tq * a.hq + th;
-      const float s = a.unit_lse[urow];
-      if (s != -INFINITY) {
-        const float mn = fmaxf(gm, s);
-        const float c_old = expf(gm - mn), c_new = expf(s - mn);
-        gz = gz * c_old + c_new;
-        const float* A = a.unit_o + urow * a.d;
-        for (int e = 0; e < per_lane; ++e) gacc[e] = gacc[e] * c_old + c_new * A[lane + 32 * e];
-        gm = mn;
+    if (a.part_o_opt != nullptr || a.part_lse_opt != nullptr) {
+      // pass 2 with shard partials: shard by shard, then the own cache
+      for (int sh = 0; sh < a.n_shards; ++sh) {
+        const int u0 = sh * a.n_split;
+        float sm = -INFINITY;
+        for (int sp = 0; sp < a.n_split; ++sp) sm = fmaxf(sm, lse_u[(int64_t)(u0 + sp) * rs]);
+        float sz = 0.f;
+        if (sm != -INFINITY)
+          for (int sp = 0; sp < a.n_split; ++sp) sz += expf(lse_u[(int64_t)(u0 + sp) * rs] - sm);
+        const float s_h = (sm == -INFINITY) ? -INFINITY : sm + logf(sz);
+        float hacc[VPL];
+#pragma unroll
+        for (int e = 0; e < VPL; ++e) hacc[e] = 0.f;
+        if (s_h != -INFINITY)
+          for (int sp = 0; sp < a.n_split; ++sp)
+            add_unit(hacc, u0 + sp, expf(lse_u[(int64_t)(u0 + sp) * rs] - s_h));
+        const int64_t prow = (b * a.n_shards + sh) * rs + th;
+        if (a.part_o_opt != nullptr) {
+#pragma unroll
+          for (int e = 0; e < VPL; ++e) a.part_o_opt[prow * D + lane * VPL + e] = hacc[e];
+        }
+        if (a.part_lse_opt != nullptr && lane == 0) a.part_lse_opt[prow] = s_h;
+        if (s_h != -INFINITY && s_all != -INFINITY) {
+          const float w = expf(s_h - s_all);
+#pragma unroll
+          for (int e = 0; e < VPL; ++e) acc[e] += w * hacc[e];
+        }
       }
+      if (a.has_self && s_all != -INFINITY)
+        add_unit(acc, units - 1, expf(lse_u[(int64_t)(units - 1) * rs] - s_all));
     }
-    OT* O = static_cast<OT*>(a.o) + row * a.d;
-    const float inv = (gm == -INFINITY) ? 0.f : 1.f / gz;
-    for (int e = 0; e < per_lane; ++e) O[lane + 32 * e] = from_f32<OT>(gacc[e] * inv);
-    if (lane == 0) a.lse[row] = (gm == -INFINITY) ? -INFINITY : gm + logf(gz);
+    OT* O = static_cast<OT*>(a.o) + row * D + lane * VPL;
+#pragma unroll
+    for (int e = 0; e < VPL; ++e) O[e] = from_f32<OT>(acc[e]);
+    if (lane == 0) a.lse[row] = s_all;
   }
 }
 
-// Splits per shard so that small batches still fill the GPU: work units are
-// (batch, shard split, kv head, group of 8 query rows); aim for 4 units per
-// SM, with at least 512 keys per split.  Independent of the dtype, so that
-// the workspace size does not depend on it.
+template <typename OT>
+static void launch_merge_kernel(const Phase2Args& a, cudaStream_t s) {
+  const int64_t nrows = (int64_t)a.B * a.Tq * a.hq;
+  if (nrows <= 0) return;
+  const int64_t want = (nrows * 32 + 255) / 256;
+  const int grid = (int)(want < 148 * 16 ? want : 148 * 16);
+  if (a.d == 128) merge_kernel<OT, 128><<<grid, 256, 0, s>>>(a);
+  else merge_kernel<OT, 64><<<grid, 256, 0, s>>>(a);
+}
+
+// Splits per shard so that small batches still fill the GPU.  Independent of
+// the dtype, so that the workspace size does not depend on it.
+//  - Few rows per kv head (decode, <= 8): work units are (batch, shard split,
+//    kv head); aim for 4 units per SM, with at least 512 keys per split.
+//  - Many rows: units are (batch, shard split, kv head, 256 query rows), one
+//    CTA per SM, keys in tiles of 128; pick the split count w that minimises
+//    waves x (fixed cost + tiles per split), waves = ceil(units x w / 148),
+//    the fixed cost of a unit (prologue, first tiles in flight, epilogue)
+//    taken as 7 tiles' work, with at least 512 keys per split.
 int32_t phase2_split(int32_t B, int32_t Tq, int64_t T, int32_t n_shards, int32_t hq,
                      int32_t hkv) {
   const int g = hq / hkv;
-  const int64_t row_groups = ((int64_t)Tq * g + 7) / 8;
-  const int64_t base = (int64_t)B * n_shards * hkv * row_groups;
+  const int64_t R = (int64_t)Tq * g;
   const int64_t shard_len = (T + n_shards - 1) / n_shards;
-  int64_t want = base > 0 ? (4 * 148 + base - 1) / base : 1;
-  const int64_t cap = shard_len / 512;
-  if (want > cap) want = cap;
-  if (want > 64) want = 64;
-  if (want < 1) want = 1;
-  return (int32_t)want;
+  int64_t cap = shard_len / 512;
+  if (cap > 64) cap = 64;
+  if (cap < 1) cap = 1;
+  if (R <= 8) {
+    const int64_t base = (int64_t)B * n_shards * hkv;
+    int64_t want = base > 0 ? (4 * 148 + base - 1) / base : 1;
+    if (want > cap) want = cap;
+    if (want < 1) want = 1;
+    return (int32_t)want;
+  }
+  const int64_t base = (int64_t)B * n_shards * hkv * ((R + 255) / 256);
+  if (base <= 0) return 1;
+  int64_t best = 1, best_cost = 0;
+  for (int64_t w = 1; w <= cap; ++w) {
+    const int64_t waves = (base * w + 147) / 148;
+    const int64_t tiles = (shard_len + w * 128 - 1) / (w * 128);
+    const int64_t cost = waves * (7 + tiles);
+    if (w == 1 || cost < best_cost) {
+      best = w;
+      best_cost = cost;
+    }
+  }
+  return (int32_t)best;
 }
 
 size_t phase2_workspace_bytes(int32_t B, int32_t Tq, int64_t T, int32_t n_shards, int32_t hq,
@@ -230,18 +312,24 @@ static int launch_phase2_t(const Phase2Args& a, cudaStream_t s) {
     f.omega[m] = (m < a.d / 2 && a.rope_theta > 0) ? pow(a.rope_theta, -2.0 * m / a.d) : 0.0;
   const float qscale = (float)(kLog2e / sqrt((double)a.d));
   const int64_t nq = (int64_t)a.B * a.Tq * a.hq * (a.d / 2);
+  // the tensor-core query kernel reads the query in fp16, which takes the
+  // place of the fp32 rotated query in the workspace
+  const bool tc = phase2_tc_supported(a);
+  __half* q16 = tc ? reinterpret_cast<__half*>(a.qr) : nullptr;
   if (nq > 0) {
     const int64_t want = (nq + 255) / 256;
     rope_query_kernel<IT><<<(int)(want < 148 * 8 ? want : 148 * 8), 256, 0, s>>>(
         static_cast<const IT*>(a.q), a.B, a.Tq, a.hq, a.d, a.q_pos0, a.rope_theta > 0, f, qscale,
-        a.qr);
+        a.qr, q16, a.status);
   }
   const int units = phase2_units(a);
   const int g = a.hq / a.hkv;
   const dim3 grid((unsigned)(a.B * units), a.hkv, (unsigned)((a.Tq * g + 127) / 128));
   int rc = PA_OK;
   profile_begin(s);
-  if (a.dtype == PA_BF16) {
+  if (tc) {
+    rc = launch_phase2_tc(a, q16, s);
+  } else if (a.dtype == PA_BF16) {
     rc = launch_phase2_mma(a, s);
   } else if (grid.x > 0 && grid.z > 0) {
     if (a.d == 128) phase2_simt_kernel<128, IT><<<grid, 256, 0, s>>>(a);
@@ -249,11 +337,7 @@ static int launch_phase2_t(const Phase2Args& a, cudaStream_t s) {
   }
   profile_end(s);
   if (rc != PA_OK) return rc;
-  const int64_t nrows = (int64_t)a.B * a.Tq * a.hq;
-  if (nrows > 0) {
-    const int64_t want = (nrows * 32 + 255) / 256;
-    merge_kernel<IT><<<(int)(want < 148 * 16 ? want : 148 * 16), 256, 0, s>>>(a);
-  }
+  launch_merge_kernel<IT>(a, s);
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
@@ -322,24 +406,19 @@ int launch_rope_query(const Phase2Args& a, cudaStream_t s) {
     const int64_t want = (nq + 255) / 256;
     if (a.dtype == PA_F32)
       rope_query_kernel<float><<<(int)(want < 148 * 8 ? want : 148 * 8), 256, 0, s>>>(
-          static_cast<const float*>(a.q), a.B, a.Tq, a.hq, a.d, a.q_pos0, a.rope_theta > 0, f, qscale, a.qr);
+          static_cast<const float*>(a.q), a.B, a.Tq, a.hq, a.d, a.q_pos0, a.rope_theta > 0, f, qscale, a.qr,
+          nullptr, a.status);
     else
       rope_query_kernel<__nv_bfloat16><<<(int)(want < 148 * 8 ? want : 148 * 8), 256, 0, s>>>(
           static_cast<const __nv_bfloat16*>(a.q), a.B, a.Tq, a.hq, a.d, a.q_pos0, a.rope_theta > 0, f, qscale,
-          a.qr);
+          a.qr, nullptr, a.status);
   }
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 int launch_merge_only(const Phase2Args& a, cudaStream_t s) {
-  const int64_t nrows = (int64_t)a.B * a.Tq * a.hq;
-  if (nrows > 0) {
-    const int64_t want = (nrows * 32 + 255) / 256;
-    if (a.dtype == PA_F32)
-      merge_kernel<float><<<(int)(want < 148 * 16 ? want : 148 * 16), 256, 0, s>>>(a);
-    else
-      merge_kernel<__nv_bfloat16><<<(int)(want < 148 * 16 ? want : 148 * 16), 256, 0, s>>>(a);
-  }
+  if (a.dtype == PA_F32) launch_merge_kernel<float>(a, s);
+  else launch_merge_kernel<__nv_bfloat16>(a, s);
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 

@@ -84,7 +84,7 @@ def idf_table(df: np.ndarray, n_blocks: int) -> np.ndarray:
 
 def chunk_scores(ids: np.ndarray, block: int, chunk: int, idf: np.ndarray) -> np.ndarray:
     """Score of every non-overlapping ``chunk``-token chunk of every block: the
-    maximum IDF over its tokens ("scored by its rarest token", [P] §2.1).
+    maximum IDF over its tokens, i.e. the IDF of its rarest token ([P] §2.1).
     Returns float64 [N][block // chunk]."""
     if block % chunk:
         raise ValueError("block must be a multiple of the chunk size")
@@ -113,8 +113,8 @@ def chunk_min_df(ids: np.ndarray, block: int, chunk: int, df: np.ndarray) -> np.
 def select_summaries(ids: np.ndarray, block: int, chunk: int, k: int, vocab: int,
                      return_scores: bool = False):
     """Top-k chunks per block by Max-IDF score, kept in original order
-    ([P] §2.1: "the top-k chunks, kept in their original order, form the
-    summary").  Equal scores: the lower chunk index wins.
+    ([P] §2.1: the summary is the k best chunks in their original order).
+    Equal scores: the lower chunk index wins.
 
     Returns int64 [N][k] local chunk indices, ascending within each block
     (and the [N][C] score table when ``return_scores``)."""
@@ -235,7 +235,7 @@ def host_row_offsets(positions) -> np.ndarray:
 
 def rope(x: np.ndarray, pos: np.ndarray, theta: float) -> np.ndarray:
     """Rotary embedding, rotate-half convention, at position ids ``pos``
-    ([P] §2.1: hosts encode "with original position IDs").
+    ([P] §2.1: every host encodes its tokens at their original position ids).
 
     x: [n][H][d] float64.  For m < d/2, with omega_m = theta^(-2m/d) and
     a = p * omega_m:  x'[m] = x[m] cos a - x[m + d/2] sin a,
@@ -308,8 +308,9 @@ def phase1_encode(q, k, v, positions, theta: float, rows_per_host=None):
 def retained_kv(k, v, theta: float):
     """KV kept after Phase 1: only each host's own block B_i survives, so the
     retained cache over all hosts is the whole sequence's K (rotated at its
-    original positions) and V ([P] §2.1 "discards the sink and summary KV";
-    §2.2 "holds the KV cache of its own block only").  Layout [L][Hkv][d] ==
+    original positions) and V ([P] §2.1: the KV of the sink and of the
+    summaries is dropped; §2.2: a host keeps the KV cache of its own block
+    alone).  Layout [L][Hkv][d] ==
     [N][block][Hkv][d]."""
     L = k.shape[0]
     return rope(k, np.arange(L), theta), np.asarray(v, dtype=np.float64)
@@ -399,7 +400,8 @@ def phase2_attend(q, k_cache, v_cache, n_shards: int, q_pos0: int, theta: float)
 def phase2_attend_with_self(q, k_cache, v_cache, n_shards: int, k_self, v_self, self_off: int,
                             q_pos0: int, theta: float):
     """Query-host step: the query and generated tokens attend globally ([S]
-    summary: "only the query and generated tokens attend globally"; [P] §5
+    summary: global attention is reserved for the query and the generated
+    tokens; [P] §5
     --tokens_to_generate).  Row j of q (rotated at q_pos0 + j) attends to
     every retained key of the shards and, causally, to the query host's own
     keys 0 .. self_off + j; the own keys form one more partial, merged with

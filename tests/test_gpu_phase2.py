@@ -51,8 +51,17 @@ def test_tiny_fp32_full(P):
     (3, 1, 999, 4, 32, 8, 128, 500000.0),      # decode rows, ragged cache
     (2, 7, 10, 16, 4, 4, 64, 0.0),             # more shards than keys: empty shards, no RoPE
     (1, 3, 0, 2, 4, 2, 64, 10000.0),           # empty cache: O = 0, lse = -inf
-    (2, 20, 700, 3, 8, 2, 64, 10000.0),        # d = 64, 80 rows per kv head (row-split kernel)
+    (2, 20, 700, 3, 8, 2, 64, 10000.0),        # d = 64, 80 rows per kv head (tensor-core kernel)
     (1, 2, 5000, 4096, 4, 1, 128, 500000.0),   # the largest shard count: most shards of 1-2 keys
+    # tensor-core query kernel (>= 64 rows per kv head, 128 % g == 0)
+    (1, 48, 2000, 3, 16, 2, 128, 500000.0),    # g = 8, 384 rows: 3 row tiles, a half-empty tile pair
+    (2, 100, 1500, 2, 4, 4, 64, 10000.0),      # g = 1, 100 rows, two batch elements
+    (1, 80, 777, 4, 32, 2, 128, 500000.0),     # g = 16, 1280 rows: 5 tile pairs share each unit
+    (1, 64, 20, 8, 8, 2, 128, 10000.0),        # 256 rows over 20 keys: 3-key shards, one empty
+    (1, 64, 0, 2, 8, 2, 64, 10000.0),          # 256 rows, empty cache: O = 0, lse = -inf
+    # row-split mma.sync kernel
+    (1, 30, 500, 2, 6, 2, 64, 10000.0),        # g = 3 does not divide 128
+    (1, 12, 900, 3, 8, 2, 128, 500000.0),      # 48 rows per kv head
 ])
 def test_bf16_small_full(P, case):
     B, Tq, T, S, hq, hkv, d, theta = case
@@ -117,3 +126,26 @@ def test_lse_merge_entry_point(P):
     pl_empty = torch.full_like(pl, float("-inf"))
     o3, lse3 = P.pa_lse_merge(torch.zeros_like(po), pl_empty, dtype=torch.float32)
     assert (o3 == 0).all() and torch.isneginf(lse3).all()
+
+
+@pytest.mark.parametrize("where", ["key", "query"])
+def test_query_kernel_range_status(P, where):
+    # the tensor-core query kernel carries the query and the keys in fp16: a
+    # value beyond fp16 range is reported as PA_ERR_RANGE (device status)
+    B, Tq, hq, hkv, d, T, S = 1, 64, 8, 2, 128, 700, 3   # 256 rows per kv head
+    q = workloads.normal((B, Tq, hq, d), 90, torch.bfloat16)
+    kc = workloads.normal((B, T, hkv, d), 91, torch.bfloat16)
+    vc = workloads.normal((B, T, hkv, d), 92, torch.bfloat16)
+    if where == "key":
+        kc[0, 321, 1, 7] = 1.0e5
+    else:
+        q[0, 5, 3, 9] = 1.0e7
+    *_, ws = P.star_phase2_attend(q.to(DEV), kc.to(DEV), vc.to(DEV), S, q_pos0=T, rope_theta=0.0)
+    assert P.pa_workspace_status(ws) == -6   # PA_ERR_RANGE
+    # the same inputs within range give PA_OK on the next call
+    if where == "key":
+        kc[0, 321, 1, 7] = 1.0
+    else:
+        q[0, 5, 3, 9] = 1.0
+    *_, ws = P.star_phase2_attend(q.to(DEV), kc.to(DEV), vc.to(DEV), S, q_pos0=T, rope_theta=0.0)
+    assert P.pa_workspace_status(ws) == 0
