@@ -241,6 +241,31 @@ int star_phase1_encode(const void* q, const void* k, const void* v, int dtype, i
                        void* o, float* lse_opt, void* k_ret, void* v_ret, void* ws,
                        size_t ws_bytes, void* stream);
 
+/*
+ * Phase 1 of a contiguous range of hosts, [host_begin, host_end) of the
+ * sequence's N = L / block hosts: the unit of work of one GPU when the hosts
+ * of one sequence are spread over GPUs ([P] §2.1, §2.2: each host encodes
+ * its own input and keeps its own block's KV; no communication in Phase 1).
+ * Inputs, arguments and workspace size as pulsar_phase1_encode /
+ * star_phase1_encode (q, k, v hold the whole sequence; only positions below
+ * host_end * block are read).  Outputs cover the range only:
+ *  o, lse_opt     rows row_off[host_begin] .. row_off[host_end] of the full
+ *                 layout (pa_phase1_layout), packed from row 0.
+ *  k_ret, v_ret   [host_end - host_begin][block][hkv][d]: the range's blocks.
+ * Results are bit-identical to the same rows of a call over every host.
+ * 0 <= host_begin <= host_end <= N (PA_ERR_INVALID otherwise); an empty range
+ * does nothing.
+ */
+int pulsar_phase1_encode_hosts(const void* q, const void* k, const void* v, int dtype, int64_t L,
+                               int32_t hq, int32_t hkv, int32_t d, double rope_theta, int32_t block,
+                               int32_t sink, int32_t chunk, int32_t k_chunks, const int32_t* sel,
+                               int32_t host_begin, int32_t host_end, void* o, float* lse_opt,
+                               void* k_ret, void* v_ret, void* ws, size_t ws_bytes, void* stream);
+int star_phase1_encode_hosts(const void* q, const void* k, const void* v, int dtype, int64_t L,
+                             int32_t hq, int32_t hkv, int32_t d, double rope_theta, int32_t block,
+                             int32_t host_begin, int32_t host_end, void* o, float* lse_opt,
+                             void* k_ret, void* v_ret, void* ws, size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------------------------------ */
 /* (a6-a7) Phase-2 split-KV attention + exact LSE merge                     */
 /*         [P] §2.2; [PS] Fase 2; [S] key_machinery, Algorithm 2 comment     */

@@ -61,10 +61,11 @@ int phase1_common(const void* q, const void* k, const void* v, int dtype, int64_
                   int32_t hkv, int32_t d, double rope_theta, int32_t block, int32_t sink,
                   int32_t chunk, int32_t k_chunks, const int32_t* sel, int star, void* o,
                   float* lse_opt, void* k_ret, void* v_ret, void* ws, size_t ws_bytes,
-                  cudaStream_t s, uint64_t wait_limit_ns = 1000000000ull, int stall = 0) {
+                  cudaStream_t s, uint64_t wait_limit_ns = 1000000000ull, int stall = 0,
+                  int32_t host_begin = 0, int32_t host_end = -1) {
   int rc = check_heads(hq, hkv, d, dtype);
   if (rc) return rc;
-  if (!q || !k || !v || !o || !k_ret || !v_ret) return PA_ERR_INVALID;
+  if (!q || !k || !v) return PA_ERR_INVALID;
   if (!(rope_theta > 0.0) || !std::isfinite(rope_theta)) return PA_ERR_INVALID;
   if (!star) {
     if (chunk <= 0 || block % chunk != 0 || k_chunks < 0 || k_chunks > block / chunk)
@@ -80,10 +81,18 @@ int phase1_common(const void* q, const void* k, const void* v, int dtype, int64_
     if (!aligned(p, 16)) return PA_ERR_UNSUPPORTED;
   HostTable ht;
   std::memset(&ht, 0, sizeof(ht));
-  int n = 0;
-  rc = layout(L, block, star ? 0 : sink, star ? 0 : k_chunks * chunk, star, ht.row_off, &n);
+  int n_all = 0;
+  int64_t off_all[kMaxBlocks + 1];
+  rc = layout(L, block, star ? 0 : sink, star ? 0 : k_chunks * chunk, star, off_all, &n_all);
   if (rc) return rc;
+  // the encoded hosts: [host_begin, host_end) of the sequence's n_all hosts
+  if (host_end < 0) host_end = n_all;
+  if (host_begin < 0 || host_begin > host_end || host_end > n_all) return PA_ERR_INVALID;
+  const int n = host_end - host_begin;
+  if (n > 0 && (!o || !k_ret || !v_ret)) return PA_ERR_INVALID;   // outputs may be null for no host
+  for (int i = 0; i <= n; ++i) ht.row_off[i] = off_all[host_begin + i] - off_all[host_begin];
   ht.n_hosts = n;
+  ht.host0 = host_begin;
   ht.star = star;
   ht.block = block;
   ht.sink = star ? 0 : sink;
@@ -95,7 +104,7 @@ int phase1_common(const void* q, const void* k, const void* v, int dtype, int64_
     ht.tile_off[i + 1] = ht.tile_off[i] + (int32_t)((ni + 127) / 128);
   }
   const int64_t R = ht.row_off[n];
-  const size_t need = phase1_workspace_bytes(L, hq, hkv, d, dtype, R);
+  const size_t need = phase1_workspace_bytes(L, hq, hkv, d, dtype, off_all[n_all]);
   rc = check_ws(ws, ws_bytes, need);
   if (rc) return rc;
   rc = clear_status(ws, s);
@@ -107,6 +116,9 @@ int phase1_common(const void* q, const void* k, const void* v, int dtype, int64_
   a.rope_theta = rope_theta;
   a.sel = sel;
   a.ht = ht;
+  a.rope_L = (int64_t)host_end * block;
+  a.ret_lo = (int64_t)host_begin * block;
+  a.ret_hi = (int64_t)host_end * block;
   a.o = o; a.lse = lse_opt; a.k_ret = k_ret; a.v_ret = v_ret;
   char* w = static_cast<char*>(ws);
   a.status = reinterpret_cast<DeviceStatus*>(w);
@@ -116,8 +128,8 @@ int phase1_common(const void* q, const void* k, const void* v, int dtype, int64_
   const size_t qk_elem = dtype == PA_BF16 ? 2 : 4;
   a.qr = w + off;
   off += align_up(qk_elem * (size_t)L * hq * d);
-  a.kr = nullptr;
-  if (dtype == PA_BF16) a.kr = w + off;
+  a.kr = w + off;
+  if (n == 0) return PA_OK;
   a.wait_limit_ns = wait_limit_ns;
   a.stall = stall;
   return launch_phase1(a, s);
@@ -292,6 +304,27 @@ int star_phase1_encode(const void* q, const void* k, const void* v, int dtype, i
                        size_t ws_bytes, void* stream) {
   return phase1_common(q, k, v, dtype, L, hq, hkv, d, rope_theta, block, 0, 16, 0, nullptr, 1,
                        o, lse_opt, k_ret, v_ret, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int pulsar_phase1_encode_hosts(const void* q, const void* k, const void* v, int dtype, int64_t L,
+                               int32_t hq, int32_t hkv, int32_t d, double rope_theta, int32_t block,
+                               int32_t sink, int32_t chunk, int32_t k_chunks, const int32_t* sel,
+                               int32_t host_begin, int32_t host_end, void* o, float* lse_opt,
+                               void* k_ret, void* v_ret, void* ws, size_t ws_bytes, void* stream) {
+  if (host_end < 0) return PA_ERR_INVALID;
+  return phase1_common(q, k, v, dtype, L, hq, hkv, d, rope_theta, block, sink, chunk, k_chunks,
+                       sel, 0, o, lse_opt, k_ret, v_ret, ws, ws_bytes,
+                       static_cast<cudaStream_t>(stream), 1000000000ull, 0, host_begin, host_end);
+}
+
+int star_phase1_encode_hosts(const void* q, const void* k, const void* v, int dtype, int64_t L,
+                             int32_t hq, int32_t hkv, int32_t d, double rope_theta, int32_t block,
+                             int32_t host_begin, int32_t host_end, void* o, float* lse_opt,
+                             void* k_ret, void* v_ret, void* ws, size_t ws_bytes, void* stream) {
+  if (host_end < 0) return PA_ERR_INVALID;
+  return phase1_common(q, k, v, dtype, L, hq, hkv, d, rope_theta, block, 0, 16, 0, nullptr, 1,
+                       o, lse_opt, k_ret, v_ret, ws, ws_bytes, static_cast<cudaStream_t>(stream),
+                       1000000000ull, 0, host_begin, host_end);
 }
 
 size_t pa_phase2_workspace_size(int32_t B, int32_t Tq, int64_t T, int32_t n_shards, int32_t hq,

@@ -48,7 +48,8 @@ struct RopeFreqs {
 
 // Phase-1 host layout shared by the kernels (small, passed by value).
 struct HostTable {
-  int32_t n_hosts;
+  int32_t n_hosts;                   // hosts in this table (a contiguous range)
+  int32_t host0;                     // sequence index of the table's first host
   int32_t star;
   int32_t block, sink, chunk, k_chunks;
   int64_t row_off[kMaxBlocks + 1];   // packed output row offsets
@@ -69,7 +70,10 @@ struct Phase1Args {
   // workspace carve
   int32_t* rowpos;              // [R] original position of every packed row
   void* qr;                     // [L][hq][d] rotated, scaled Q (fp16 or fp32)
-  void* kr;                     // [L][hkv][d] rotated K in QK type (fp16) or == k_ret (fp32)
+  void* kr;                     // [L][hkv][d] rotated K in the QK type (fp16 or fp32)
+  // positions [0, rope_L) are rotated; k_ret / v_ret hold positions
+  // [ret_lo, ret_hi) (the blocks of the table's hosts)
+  int64_t rope_L = 0, ret_lo = 0, ret_hi = 0;
   DeviceStatus* status;
   // bounded-wait limit of the tensor-core kernel and a test-only stall
   uint64_t wait_limit_ns = 1000000000ull;

@@ -26,9 +26,10 @@ __global__ void rowpos_kernel(HostTable ht, const int32_t* __restrict__ sel,
   const int C = ht.chunk > 0 ? ht.block / ht.chunk : 0;
   for (int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r < R;
        r += (int64_t)gridDim.x * blockDim.x) {
-    int i = 0;
-    while (i + 1 < ht.n_hosts && r >= ht.row_off[i + 1]) ++i;
-    const int64_t u = r - ht.row_off[i];
+    int li = 0;
+    while (li + 1 < ht.n_hosts && r >= ht.row_off[li + 1]) ++li;
+    const int64_t u = r - ht.row_off[li];
+    const int i = ht.host0 + li;                     // the host's index in the sequence
     int64_t p;
     if (i == 0) {
       p = u;                                         // host 0: B_0 alone
@@ -67,7 +68,7 @@ template <typename IT, typename QT, int POS>
 __global__ void __launch_bounds__(256) rope_qk_kernel(
     const IT* __restrict__ q, const IT* __restrict__ k, int64_t L, int hq, int hkv, int d,
     RopeFreqs f, float qscale, QT* __restrict__ qr, QT* __restrict__ kr, IT* __restrict__ k_ret,
-    DeviceStatus* st) {
+    int64_t ret_lo, int64_t ret_hi, DeviceStatus* st) {
   constexpr int VEC = 16 / sizeof(IT);          // input elements per 16-byte vector
   __shared__ float2 cs[POS][kMaxHalfDim];
   const int half = d / 2;
@@ -114,15 +115,18 @@ __global__ void __launch_bounds__(256) rope_qk_kernel(
       *reinterpret_cast<Vec<QT, VEC>*>(qr + base + m0) = o1;
       *reinterpret_cast<Vec<QT, VEC>*>(qr + base + m0 + half) = o2;
     } else {
-      Vec<IT, VEC> r1, r2;
+      if (p >= ret_lo && p < ret_hi) {   // retained: the blocks of the encoded hosts
+        Vec<IT, VEC> r1, r2;
 #pragma unroll
-      for (int i = 0; i < VEC; ++i) {
-        r1.v[i] = from_f32<IT>(y1[i]);
-        r2.v[i] = from_f32<IT>(y2[i]);
+        for (int i = 0; i < VEC; ++i) {
+          r1.v[i] = from_f32<IT>(y1[i]);
+          r2.v[i] = from_f32<IT>(y2[i]);
+        }
+        const int64_t rb = base - ret_lo * hkv * (int64_t)d;
+        *reinterpret_cast<Vec<IT, VEC>*>(k_ret + rb + m0) = r1;
+        *reinterpret_cast<Vec<IT, VEC>*>(k_ret + rb + m0 + half) = r2;
       }
-      *reinterpret_cast<Vec<IT, VEC>*>(k_ret + base + m0) = r1;
-      *reinterpret_cast<Vec<IT, VEC>*>(k_ret + base + m0 + half) = r2;
-      if (kr != nullptr) {
+      {
         Vec<QT, VEC> o1, o2;
 #pragma unroll
         for (int i = 0; i < VEC; ++i) {
@@ -245,7 +249,7 @@ size_t phase1_workspace_bytes(int64_t L, int32_t hq, int32_t hkv, int32_t d, int
   size_t b = kStatusBytes;
   b += align_up(sizeof(int32_t) * (size_t)total_rows);
   b += align_up(qk_elem * (size_t)L * hq * d);
-  if (dtype == PA_BF16) b += align_up(qk_elem * (size_t)L * hkv * d);
+  b += align_up(qk_elem * (size_t)L * hkv * d);
   return b;
 }
 
@@ -263,18 +267,21 @@ static int launch_phase1_t(const Phase1Args& a, cudaStream_t s) {
     f.omega[m] = (m < a.d / 2) ? pow(a.rope_theta, -2.0 * m / a.d) : 0.0;
   const float qscale = (float)(kLog2e / sqrt((double)a.d));
   constexpr int POS = 8;
-  if (a.L > 0) {
-    rope_qk_kernel<IT, QT, POS><<<(unsigned)((a.L + POS - 1) / POS), 256, 0, s>>>(
-        static_cast<const IT*>(a.q), static_cast<const IT*>(a.k), a.L, a.hq, a.hkv, a.d, f,
-        qscale, static_cast<QT*>(a.qr), static_cast<QT*>(a.kr), static_cast<IT*>(a.k_ret),
-        a.status);
+  if (a.rope_L > 0) {
+    rope_qk_kernel<IT, QT, POS><<<(unsigned)((a.rope_L + POS - 1) / POS), 256, 0, s>>>(
+        static_cast<const IT*>(a.q), static_cast<const IT*>(a.k), a.rope_L, a.hq, a.hkv, a.d, f,
+        qscale, static_cast<QT*>(a.qr), static_cast<QT*>(a.kr), static_cast<IT*>(a.k_ret), a.ret_lo,
+        a.ret_hi, a.status);
   }
-  if (a.v_ret != a.v && a.L > 0) {
-    if (cudaMemcpyAsync(a.v_ret, a.v, sizeof(IT) * (size_t)a.L * a.hkv * a.d,
-                        cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+  const size_t vrow = sizeof(IT) * (size_t)a.hkv * a.d;
+  if (a.ret_hi > a.ret_lo) {
+    const void* vsrc = static_cast<const char*>(a.v) + vrow * (size_t)a.ret_lo;
+    if (a.v_ret != vsrc &&
+        cudaMemcpyAsync(a.v_ret, vsrc, vrow * (size_t)(a.ret_hi - a.ret_lo), cudaMemcpyDeviceToDevice, s) !=
+            cudaSuccess)
       return PA_ERR_CUDA;
   }
-  const QT* kq = a.kr ? static_cast<const QT*>(a.kr) : static_cast<const QT*>(a.k_ret);
+  const QT* kq = static_cast<const QT*>(a.kr);
   const dim3 grid(a.ht.tile_off[a.ht.n_hosts], a.hq);
   int rc = PA_OK;
   profile_begin(s);

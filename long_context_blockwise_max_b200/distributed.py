@@ -1,7 +1,15 @@
-"""Phase 2 across GPUs: the exchange step of the query phase.
+"""The multi-GPU layout of the method: one host (block) per GPU.
 
-The Pulsar Attention page (§2.2) and the Star Attention review
-(key_machinery) describe the only communication of the method.
+The Pulsar Attention page (§2.1, §2.2) and the Star Attention review
+(key_machinery) spread the hosts of one sequence over devices.
+
+Phase 1 needs no communication: every host encodes its own input (sink,
+summaries of the earlier blocks, its own block) from the whole sequence's
+ids and Q / K / V, and keeps its own block's KV.  ``phase1_encode_distributed``
+gives each rank a contiguous range of hosts and runs
+``pulsar_phase1_encode_hosts`` (or the Star variant) on it.
+
+Phase 2 has the method's one exchange step:
 
 1. The query is broadcast.
 2. Each host attends over the retained cache it holds.
@@ -9,10 +17,10 @@ The Pulsar Attention page (§2.2) and the Star Attention review
    are all-gathered.
 4. An exact online-softmax merge follows.
 
-Here every rank holds a contiguous range of shards. It computes their
-partials with ``star_phase2_attend`` and all-gathers the packed partials
-with ``torch.distributed`` (NCCL on GPUs). Every rank then merges all of them
-with ``pa_lse_merge``. The partial and merge steps can be replaced by other
+``phase2_attend_distributed`` computes a rank's shard partials with
+``star_phase2_attend``, all-gathers the packed partials with
+``torch.distributed`` (NCCL on GPUs), and merges all of them with
+``pa_lse_merge`` on every rank.  The per-rank steps can be replaced by other
 functions of the same contract, which the CPU tests use with the gloo
 backend.
 """
@@ -27,6 +35,34 @@ def shard_ranges(n_shards: int, world: int) -> list[tuple[int, int]]:
     last ranks possibly shorter or empty."""
     per = -(-n_shards // world)
     return [(min(r * per, n_shards), min((r + 1) * per, n_shards)) for r in range(world)]
+
+
+def _gpu_encode_hosts(q, k, v, rope_theta, block, sink, chunk, k_chunks, sel, star, h0, h1):
+    from . import pulsar
+    if star:
+        o, lse, k_ret, v_ret, _, _ = pulsar.star_phase1_encode_hosts(q, k, v, rope_theta, block, h0, h1)
+    else:
+        o, lse, k_ret, v_ret, _, _ = pulsar.pulsar_phase1_encode_hosts(q, k, v, rope_theta, block, sink, chunk,
+                                                                       k_chunks, sel, h0, h1)
+    return o, lse, k_ret, v_ret
+
+
+def phase1_encode_distributed(q, k, v, rope_theta: float, block: int, sink: int = 64, chunk: int = 32,
+                              k_chunks: int = 0, sel=None, star: bool = False, group=None, encode_fn=None):
+    """Phase 1 of one sequence with its N = L / block hosts spread over the
+    ranks: rank r encodes hosts shard_ranges(N, world)[r] (no collective).
+
+    q [L][hq][d], k, v [L][hkv][d] and sel [N][k_chunks] are the whole
+    sequence's, the same on every rank.  Returns (o, lse, k_ret, v_ret,
+    (host_begin, host_end)): the range's Phase-1 rows and retained blocks,
+    which are this rank's shards for ``phase2_attend_distributed``."""
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    n_hosts = q.shape[0] // block
+    h0, h1 = shard_ranges(n_hosts, world)[rank]
+    fn = encode_fn or _gpu_encode_hosts
+    o, lse, k_ret, v_ret = fn(q, k, v, rope_theta, block, sink, chunk, k_chunks, sel, star, h0, h1)
+    return o, lse, k_ret, v_ret, (h0, h1)
 
 
 def _gpu_partials(q, k_local, v_local, n_local, q_pos0, rope_theta):

@@ -27,6 +27,7 @@ ABI_SYMBOLS = (
     "pa_select_workspace_size", "pulsar_select_summaries", "pulsar_select_summaries_noalloc",
     "pulsar_select_summaries_scored",
     "pa_phase1_layout", "pa_phase1_workspace_size", "pulsar_phase1_encode", "star_phase1_encode",
+    "pulsar_phase1_encode_hosts", "star_phase1_encode_hosts",
     "pa_phase2_workspace_size", "star_phase2_attend", "star_phase2_query_step", "pa_lse_merge",
     "star_phase2_attend_art",
 )
@@ -61,6 +62,10 @@ def _load() -> ctypes.CDLL:
                                                 I32, P, P, P, P, P, P, SZ, P]),
         "star_phase1_encode": (ctypes.c_int, [P, P, P, ctypes.c_int, I64, I32, I32, I32, D, I32, P, P, P, P,
                                               P, SZ, P]),
+        "pulsar_phase1_encode_hosts": (ctypes.c_int, [P, P, P, ctypes.c_int, I64, I32, I32, I32, D, I32, I32,
+                                                      I32, I32, P, I32, I32, P, P, P, P, P, SZ, P]),
+        "star_phase1_encode_hosts": (ctypes.c_int, [P, P, P, ctypes.c_int, I64, I32, I32, I32, D, I32, I32, I32,
+                                                    P, P, P, P, P, SZ, P]),
         "pa_phase2_workspace_size": (SZ, [I32, I32, I64, I32, I32, I32, I32]),
         "star_phase2_attend": (ctypes.c_int, [P, ctypes.c_int, I32, I32, I64, D, P, P, I64, I32, I32, I32,
                                               I32, P, P, P, P, P, SZ, P]),
@@ -252,6 +257,66 @@ def star_phase1_encode(q, k, v, rope_theta, block, o=None, lse=None, k_ret=None,
                                  _ptr(o), _ptr(lse), _ptr(k_ret), _ptr(v_ret), _ptr(ws), ws.numel(),
                                  _stream())
     _check(rc, "star_phase1_encode")
+    return o, lse, k_ret, v_ret, row_off, ws
+
+
+def _phase1_range_outputs(q, k, block, rows, nh, o, lse, k_ret, v_ret, want_lse):
+    _, hq, d = q.shape
+    hkv = k.shape[1]
+    if o is None:
+        o = torch.empty((rows, hq, d), dtype=q.dtype, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((rows, hq), dtype=torch.float32, device=q.device)
+    if k_ret is None:
+        k_ret = torch.empty((nh * block, hkv, d), dtype=q.dtype, device=q.device)
+    if v_ret is None:
+        v_ret = torch.empty((nh * block, hkv, d), dtype=q.dtype, device=q.device)
+    return o, lse, k_ret, v_ret
+
+
+def pulsar_phase1_encode_hosts(q, k, v, rope_theta, block, sink, chunk, k_chunks, sel, host_begin, host_end,
+                               o=None, lse=None, k_ret=None, v_ret=None, ws=None, want_lse=True):
+    """Pulsar Phase 1 of hosts [host_begin, host_end) only (one GPU's share of
+    a sequence's hosts).  Returns (o, lse, k_ret, v_ret, row_off, ws): o / lse
+    hold the range's rows packed from 0, row_off their offsets (starting at
+    0), k_ret / v_ret the range's blocks."""
+    _dev(q, k, v, sel, o, lse, k_ret, v_ret)
+    L, hq, d = q.shape
+    hkv = k.shape[1]
+    dt = _dtype_code(q)
+    full = pa_phase1_layout(L, block, sink, k_chunks * chunk, False)
+    row_off = [r - full[host_begin] for r in full[host_begin:host_end + 1]]
+    nh = max(host_end - host_begin, 0)
+    o, lse, k_ret, v_ret = _phase1_range_outputs(q, k, block, row_off[-1] if row_off else 0, nh, o, lse, k_ret,
+                                                 v_ret, want_lse)
+    need = pa_phase1_workspace_size(L, hq, hkv, d, dt, block, sink, k_chunks * chunk, False)
+    ws = _workspace(need, q.device, ws)
+    rc = _lib.pulsar_phase1_encode_hosts(_ptr(q), _ptr(k), _ptr(v), dt, L, hq, hkv, d, float(rope_theta), block,
+                                         sink, chunk, k_chunks, _ptr(sel), host_begin, host_end, _ptr(o), _ptr(lse),
+                                         _ptr(k_ret), _ptr(v_ret), _ptr(ws), ws.numel(), _stream())
+    _check(rc, "pulsar_phase1_encode_hosts")
+    return o, lse, k_ret, v_ret, row_off, ws
+
+
+def star_phase1_encode_hosts(q, k, v, rope_theta, block, host_begin, host_end, o=None, lse=None, k_ret=None,
+                             v_ret=None, ws=None, want_lse=True):
+    """Star anchor-variant Phase 1 of hosts [host_begin, host_end) only.
+    Returns (o, lse, k_ret, v_ret, row_off, ws) as pulsar_phase1_encode_hosts."""
+    _dev(q, k, v, o, lse, k_ret, v_ret)
+    L, hq, d = q.shape
+    hkv = k.shape[1]
+    dt = _dtype_code(q)
+    full = pa_phase1_layout(L, block, 0, 0, True)
+    row_off = [r - full[host_begin] for r in full[host_begin:host_end + 1]]
+    nh = max(host_end - host_begin, 0)
+    o, lse, k_ret, v_ret = _phase1_range_outputs(q, k, block, row_off[-1] if row_off else 0, nh, o, lse, k_ret,
+                                                 v_ret, want_lse)
+    need = pa_phase1_workspace_size(L, hq, hkv, d, dt, block, 0, 0, True)
+    ws = _workspace(need, q.device, ws)
+    rc = _lib.star_phase1_encode_hosts(_ptr(q), _ptr(k), _ptr(v), dt, L, hq, hkv, d, float(rope_theta), block,
+                                       host_begin, host_end, _ptr(o), _ptr(lse), _ptr(k_ret), _ptr(v_ret), _ptr(ws),
+                                       ws.numel(), _stream())
+    _check(rc, "star_phase1_encode_hosts")
     return o, lse, k_ret, v_ret, row_off, ws
 
 

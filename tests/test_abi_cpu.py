@@ -29,7 +29,7 @@ def _header_functions():
 
 def test_library_exports_every_declared_symbol(lib):
     names = _header_functions()
-    assert len(names) == 17
+    assert len(names) == 19
     assert sorted(lib.ABI_SYMBOLS) == names
     so = ctypes.CDLL(lib.LIB_PATH)
     for n in names:
@@ -83,6 +83,14 @@ def test_host_validation_rejects_before_launch(lib):
     args = (dummy, dummy, dummy, 0, 2048, 4, 2, 64, 10000.0, 512, dummy, None, ctypes.c_void_p(4098), dummy,
             ws, 1 << 30, None)
     assert so.star_phase1_encode(*args) == -2
+    # host ranges: begin after end, end past the last host (4 hosts of 512), negative end
+    for hb, he in ((3, 2), (0, 5), (0, -1)):
+        args = (dummy, dummy, dummy, 0, 2048, 4, 2, 64, 10000.0, 512, 64, 32, 2, dummy, hb, he, dummy, None,
+                dummy, dummy, ws, 1 << 30, None)
+        assert so.pulsar_phase1_encode_hosts(*args) == -1, (hb, he)
+        args = (dummy, dummy, dummy, 0, 2048, 4, 2, 64, 10000.0, 512, hb, he, dummy, None, dummy, dummy, ws,
+                1 << 30, None)
+        assert so.star_phase1_encode_hosts(*args) == -1, (hb, he)
     # phase 2: zero shards
     assert so.star_phase2_attend(dummy, 1, 1, 1, 0, 0.0, dummy, dummy, 100, 0, 32, 8, 128, dummy, dummy, None,
                                  None, ws, 1 << 30, None) == -1

@@ -1,8 +1,10 @@
-"""The Phase-2 exchange across ranks (Pulsar page §2.2: partials are
-all-gathered, then merged exactly), on CPU with the gloo backend and world
-size 2: per-rank partials and the merge come from the oracle, so this
-checks the shard partition, packing, gather order and padding of
-long_context_blockwise_max_b200.distributed against dense attention."""
+"""The multi-GPU layout across ranks, on CPU with the gloo backend: Phase 1
+with the hosts spread over ranks (Pulsar page §2.1: no communication), and
+the Phase-2 exchange (§2.2: partials are all-gathered, then merged exactly).
+The per-rank compute steps come from the oracle, so these tests check the
+host and shard partitions, packing, gather order and padding of
+long_context_blockwise_max_b200.distributed against the oracle run on one
+process."""
 import os
 import socket
 import sys
@@ -86,3 +88,79 @@ def test_shard_ranges():
     assert shard_ranges(8, 4) == [(0, 2), (2, 4), (4, 6), (6, 8)]
     assert shard_ranges(3, 2) == [(0, 2), (2, 3)]
     assert shard_ranges(1, 3) == [(0, 1), (1, 1), (1, 1)]
+
+
+# --------------------------------------------------------------------------
+# Phase 1 spread over ranks, then the Phase-2 exchange over the ranks' blocks
+# --------------------------------------------------------------------------
+L1, BLK1, SINK1, CH1, K1, HQ1, HKV1, D1, TH1 = 256, 64, 16, 16, 1, 4, 2, 16, 10000.0
+
+
+def _pipeline_inputs():
+    g = torch.Generator().manual_seed(11)
+    q = torch.randn(L1, HQ1, D1, generator=g, dtype=torch.float64)
+    k = torch.randn(L1, HKV1, D1, generator=g, dtype=torch.float64)
+    v = torch.randn(L1, HKV1, D1, generator=g, dtype=torch.float64)
+    sel = torch.tensor([[2], [0], [3], [1]], dtype=torch.int64)
+    qq = torch.randn(1, 3, HQ1, D1, generator=g, dtype=torch.float64)
+    return q, k, v, sel, qq
+
+
+def _oracle_encode_hosts(q, k, v, theta, block, sink, chunk, k_chunks, sel, star, h0, h1):
+    import oracle
+    pos = oracle.host_positions(q.shape[0], block, sink, chunk, sel.numpy(), star=star)
+    outs = oracle.phase1_encode(q.numpy(), k.numpy(), v.numpy(), pos, theta)[h0:h1]
+    kr, vr = oracle.retained_kv(k.numpy(), v.numpy(), theta)
+    o = np.concatenate([x[0] for x in outs]) if outs else np.zeros((0, q.shape[1], q.shape[2]))
+    lse = np.concatenate([x[1] for x in outs]) if outs else np.zeros((0, q.shape[1]))
+    return (torch.from_numpy(o), torch.from_numpy(lse), torch.from_numpy(kr[h0 * block:h1 * block]),
+            torch.from_numpy(vr[h0 * block:h1 * block]))
+
+
+def _pipeline_worker(rank, world, port, star, out):
+    sys.path.insert(0, ROOT)
+    from long_context_blockwise_max_b200 import distributed as D
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        q, k, v, sel, qq = _pipeline_inputs()
+        o, lse, kr, vr, (h0, h1) = D.phase1_encode_distributed(q, k, v, TH1, BLK1, SINK1, CH1, K1, sel, star,
+                                                               encode_fn=_oracle_encode_hosts)
+        og, lg = D.phase2_attend_distributed(qq, kr[None], vr[None], h1 - h0, L1 // BLK1, L1, TH1,
+                                             partials_fn=_oracle_partials, merge_fn=_oracle_merge)
+        out[rank] = (h0, h1, o.numpy(), lse.numpy(), og.numpy(), lg.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+def _pipeline(world, star):
+    import oracle
+    port = _free_port()
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_pipeline_worker, args=(world, port, star, out), nprocs=world, join=True)
+        res = [out[r] for r in range(world)]
+    q, k, v, sel, qq = _pipeline_inputs()
+    n = L1 // BLK1
+    # the ranks' host ranges tile [0, n) in order
+    assert [(r[0], r[1]) for r in res] == __import__(
+        "long_context_blockwise_max_b200.distributed", fromlist=["x"]).shard_ranges(n, world)
+    # Phase 1: the ranks' rows, in rank order, are the one-process encoding
+    pos = oracle.host_positions(L1, BLK1, SINK1, CH1, sel.numpy(), star=star)
+    full = oracle.phase1_encode(q.numpy(), k.numpy(), v.numpy(), pos, TH1)
+    np.testing.assert_array_equal(np.concatenate([r[2] for r in res]), np.concatenate([x[0] for x in full]))
+    np.testing.assert_array_equal(np.concatenate([r[3] for r in res]), np.concatenate([x[1] for x in full]))
+    # Phase 2 over the ranks' retained blocks equals one-process attention
+    kr, vr = oracle.retained_kv(k.numpy(), v.numpy(), TH1)
+    ro, rl, _, _ = oracle.phase2_attend(qq.numpy(), kr[None], vr[None], n, L1, TH1)
+    for r in res:
+        np.testing.assert_allclose(r[4], ro, rtol=0, atol=1e-6)
+        np.testing.assert_allclose(r[5], rl, rtol=0, atol=1e-6)
+
+
+def test_phase1_hosts_over_two_ranks_then_exchange():
+    _pipeline(2, False)
+
+
+def test_star_hosts_over_three_ranks_one_empty():
+    _pipeline(3, True)   # 4 hosts over 3 ranks: (0, 2), (2, 4), (4, 4)

@@ -150,3 +150,34 @@ def test_bad_summary_index_sets_status(P):
     bad = torch.tensor([[9], [0]], dtype=torch.int32, device=DEV)   # 128/16 = 8 chunks: 9 is out of range
     *_, ws = P.pulsar_phase1_encode(q.to(DEV), k.to(DEV), v.to(DEV), 1e4, block, 16, 16, 1, bad)
     assert P.pa_workspace_status(ws) == -1
+
+
+@pytest.mark.parametrize("star,dtype,splits", [
+    (False, torch.bfloat16, [(0, 2), (2, 5), (5, 6), (3, 3)]),   # tensor-core kernel; an empty range
+    (True, torch.bfloat16, [(0, 1), (1, 6)]),
+    (False, torch.float32, [(0, 4), (4, 6)]),                    # SIMT kernel
+])
+def test_host_ranges_equal_full_encode(P, star, dtype, splits):
+    # one GPU's share of a sequence's hosts (the multi-GPU layout of the
+    # Pulsar page §2.1 / §2.2): the rows and retained blocks of every range
+    # are bit-identical to the same rows of the all-host call
+    L, block, sink, chunk, kc = 6 * 256, 256, 64, 32, 2
+    hq, hkv, d = (8, 2, 128) if dtype == torch.bfloat16 else (4, 2, 64)
+    q, k, v = _inputs(L, hq, hkv, d, dtype, seed=30)
+    sel = np.array([[1, 5], [0, 7], [2, 3], [4, 6], [1, 2], [0, 3]], dtype=np.int32)
+    o, lse, kr, vr, off = _run(P, q, k, v, 5e5, block, sink, chunk, kc, sel, star)
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    seld = torch.from_numpy(sel).to(DEV)
+    for h0, h1 in splits:
+        if star:
+            o2, lse2, kr2, vr2, off2, ws = P.star_phase1_encode_hosts(qd, kd, vd, 5e5, block, h0, h1)
+        else:
+            o2, lse2, kr2, vr2, off2, ws = P.pulsar_phase1_encode_hosts(qd, kd, vd, 5e5, block, sink, chunk, kc,
+                                                                        seld, h0, h1)
+        assert P.pa_workspace_status(ws) == 0
+        assert off2 == [r - off[h0] for r in off[h0:h1 + 1]]
+        rows = slice(off[h0], off[h1])
+        assert torch.equal(o2, o[rows]), (h0, h1)
+        assert torch.equal(lse2, lse[rows]), (h0, h1)
+        assert torch.equal(kr2, kr[h0 * block:h1 * block]), (h0, h1)
+        assert torch.equal(vr2, vr[h0 * block:h1 * block]), (h0, h1)
