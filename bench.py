@@ -183,18 +183,28 @@ class Step:
                                dtype=torch.uint8, device=dev)
         self.attn_events = None
         self.p2_events = None
+        self.stage_events = None   # 4 events: before selection, after it, after Phase 1, after Phase 2
 
     def run(self):
         P, w = self.P, self.w
+        ev = self.stage_events
+        if ev:
+            ev[0].record()
         P.pulsar_select_summaries(self.ids, w.vocab, w.block, w.chunk, w.k_chunks, sel=self.sel, ws=self.ws_sel)
+        if ev:
+            ev[1].record()
         P.pa_set_profile_events(*(self.attn_events or (None, None)))
         P.pulsar_phase1_encode(self.q, self.k, self.v, w.rope_theta, w.block, w.sink, w.chunk, w.k_chunks,
                                self.sel, o=self.o1, lse=self.lse1, k_ret=self.k_ret, v_ret=self.v_ret,
                                ws=self.ws1)
+        if ev:
+            ev[2].record()
         P.pa_set_profile_events(*(self.p2_events or (None, None)))
         P.star_phase2_attend(self.query, self.k_ret[None], self.v_ret[None], w.n_blocks, q_pos0=w.L,
                              rope_theta=w.rope_theta, o=self.o2, lse=self.lse2, ws=self.ws2)
         P.pa_set_profile_events(None, None)
+        if ev:
+            ev[3].record()
 
     # kernels of ours launched by one step (selection 3, Phase 1 3, Phase 2 3)
     LAUNCHES = 9
@@ -252,9 +262,13 @@ def run_ours(args, rank, world, local_rank, dist_on):
     K = args.steps
     ev_attn = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     ev_p2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    ev_stage = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(4)) for _ in range(K)]
     for a, b in ev_attn + ev_p2:      # torch creates the CUDA event on its first record
         a.record()
         b.record()
+    for evs in ev_stage:
+        for e in evs:
+            e.record()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sync_all(dist_on)
     with ClockSampler(local_rank) as clk:
@@ -262,15 +276,20 @@ def run_ours(args, rank, world, local_rank, dist_on):
         for i in range(K):
             step.attn_events = ev_attn[i]
             step.p2_events = ev_p2[i]
+            step.stage_events = ev_stage[i]
             step.run()
         t1.record()
         torch.cuda.synchronize()
     step.attn_events = None
     step.p2_events = None
+    step.stage_events = None
     sync_all(dist_on)
     ms = max_over_ranks(t0.elapsed_time(t1), dist_on) / K
     attn_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_attn)
     p2_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_p2)
+    sel_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev_stage)
+    enc_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev_stage)
+    p2_call_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in ev_stage)
 
     flops = attn_flops(w)
     tokens_per_s = whole_job_rate(w.L, world, ms)
@@ -476,6 +495,10 @@ def run_ours(args, rank, world, local_rank, dist_on):
         extra["selection_us"] = sc
 
     q2_bytes = 2.0 * w.L * w.hkv * w.d * 2
+    # the query's roofline: the slower of streaming K/V at the measured copy
+    # bandwidth and its QK^T + PV work at the measured sustained bf16 peak
+    q2_roof_ms = max(q2_bytes / (peaks["hbm_gbs"] * 1e9),
+                     4.0 * w.d * w.hq * w.q_tokens * w.L / (peaks["bf16_tflops_sustained"] * 1e12)) * 1e3
     clocks = clk.summary()
     line = {
         "metric": METRIC, "value": round(tokens_per_s, 1), "unit": "tokens/s", "n_gpus": world,
@@ -495,13 +518,19 @@ def run_ours(args, rank, world, local_rank, dist_on):
                      "peak_kind": f"{peak_kind} bf16 sustained",
                      "traffic": recorded_traffic("phase1_tc_kernel", w.name),
                      "kernel_ms": round(attn_ms, 3), "flop_per_launch": flops},
+        "phase1_encode": {"selection_ms": round(sel_ms, 4), "encode_ms": round(enc_ms, 3),
+                          "tokens_per_s": round(w.L / (enc_ms * 1e-3), 1),
+                          "with_selection_tokens_per_s": round(w.L / ((sel_ms + enc_ms) * 1e-3), 1),
+                          "note": "encode = position map + RoPE + attention over all hosts"},
         "phase1": {"attn_ms": round(attn_ms, 3), "tflop": round(flops / 1e12, 3),
                    "tflop_s": round(attn_tf, 1)},
         "phase2_query": {"kernel": "phase2_tc_kernel", "kernel_ms": round(p2_ms, 4), "kv_bytes": q2_bytes,
                          "traffic": recorded_traffic("phase2_tc_kernel", w.name + ":query64"),
                          "gb_s": round(q2_bytes / (p2_ms * 1e-3) / 1e9, 1),
                          "frac_hbm": round(q2_bytes / (p2_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
-                         "tflop_s": round(4.0 * w.d * w.hq * w.q_tokens * w.L / (p2_ms * 1e-3) / 1e12, 1)},
+                         "tflop_s": round(4.0 * w.d * w.hq * w.q_tokens * w.L / (p2_ms * 1e-3) / 1e12, 1),
+                         "roofline_ms": round(q2_roof_ms, 4), "frac_roofline": round(q2_roof_ms / p2_ms, 4),
+                         "call_ms": round(p2_call_ms, 4)},
     }
     line.update(extra)
     return line

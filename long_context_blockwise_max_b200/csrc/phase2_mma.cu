@@ -434,200 +434,284 @@ __global__ void __launch_bounds__(kWarps * 32) phase2_mma_rows_kernel(Phase2Args
 }
 
 // ---------------------------------------------------------------------------
-// ART (run-time early termination, ART review page): one warp per (batch,
-// kv head) walks the cache from the newest key backwards in 32-key tiles
-// through an 8-stage cp.async ring; after every block of `block_keys` keys
-// it compares the normalised running output of each query row with the
-// previous block's (magnitude change <= tau * |x_prev|, 1 - cos <= phi) and
-// stops once `patience` consecutive blocks were stable for every row.
+// ART (run-time early termination, ART review page): the cache of each
+// (batch, kv head) is walked from the newest key backwards in blocks of
+// `block_keys` keys; after every block the normalised running output of
+// each query row is compared with the previous block's (magnitude change
+// <= tau * |x_prev|, 1 - cos <= phi), and the walk stops once `patience`
+// consecutive blocks were stable for every row.
+//
+// CTA = one (batch, kv head), 5 warps.  Warps 0-3 compute, in rounds of four
+// blocks, the partial (m, l, A) of one block each (32-key tiles through a
+// private 3-stage cp.async ring, hi/lo query MMAs as in the decode kernel)
+// into a double-buffered shared-memory slot.  Warp 4 folds the partials into
+// the running result in block order (the exact log-sum-exp merge) and runs
+// the stability test after each block, while the compute warps work on the
+// next round.  A stop discards the rest of the round and the round computed
+// ahead; the result is attention over the blocks folded.
 // ---------------------------------------------------------------------------
-constexpr int kArtStages = 8;
+constexpr int kArtWarps = 4;       // compute warps
+constexpr int kArtStages = 3;      // cp.async stages per compute warp
 
 template <int D>
-__global__ void __launch_bounds__(32) phase2_art_kernel(Phase2Args a, ArtArgs art) {
+struct ArtCfg {
+  static constexpr int RING = kArtStages * P2Cfg<D>::STAGE;        // per compute warp
+  static constexpr int OFF_PART = kArtWarps * RING;
+  static constexpr int PART_O = 8 * D;                             // floats per warp slot
+  static constexpr int PART = PART_O + 16;                         // + m[8], l[8]
+  static constexpr int SMEM = OFF_PART + 2 * kArtWarps * PART * 4 + 16;
+};
+
+template <int D>
+__global__ void __launch_bounds__((kArtWarps + 1) * 32) phase2_art_kernel(Phase2Args a, ArtArgs art) {
   using C = P2Cfg<D>;
+  using AC = ArtCfg<D>;
   extern __shared__ __align__(128) uint8_t smem[];
-  const int lane = threadIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.x, kvh = blockIdx.y;
   const int g = a.hq / a.hkv;
   const int R = a.Tq * g;
   const int qi = lane >> 2, qc = (lane & 3) * 2;
   const bool row_ok = qi < R;
-  const int t_row = row_ok ? qi / g : 0;
-  const int head = kvh * g + (row_ok ? qi % g : 0);
-  uint32_t qa[D / 16][4];
-  {
-    const float* qp = a.qr + (((int64_t)b * a.Tq + t_row) * a.hq + head) * D;
-#pragma unroll
-    for (int ks = 0; ks < D / 16; ++ks) {
-      float x[4];
-      x[0] = row_ok ? qp[16 * ks + qc] : 0.f;
-      x[1] = row_ok ? qp[16 * ks + qc + 1] : 0.f;
-      x[2] = row_ok ? qp[16 * ks + qc + 8] : 0.f;
-      x[3] = row_ok ? qp[16 * ks + qc + 9] : 0.f;
-      float h[4], l[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        h[e] = __bfloat162float(__float2bfloat16_rn(x[e]));
-        l[e] = x[e] - h[e];
-      }
-      qa[ks][0] = pack_bf16(h[0], h[1]);
-      qa[ks][1] = pack_bf16(l[0], l[1]);
-      qa[ks][2] = pack_bf16(h[2], h[3]);
-      qa[ks][3] = pack_bf16(l[2], l[3]);
-    }
-  }
   const int64_t T = a.T;
   const int n_tiles = static_cast<int>((T + kKT - 1) / kKT);
-  const int tiles_per_block = art.block_keys / kKT;
-  const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
-  const __nv_bfloat16* Kg = static_cast<const __nv_bfloat16*>(a.k_ret);
-  const __nv_bfloat16* Vg = static_cast<const __nv_bfloat16*>(a.v_ret);
-  const int64_t key_stride = (int64_t)a.hkv * D;
-  const int64_t base_off = ((int64_t)b * T) * key_stride + (int64_t)kvh * D;
-  // tile s covers keys [T - 32 (s + 1), T - 32 s), clipped at 0
-  auto issue = [&](int it) {
-    if (it < n_tiles) {
-      const int64_t key0 = T - (int64_t)kKT * (it + 1);
-      const uint32_t sbase = base + (it % kArtStages) * C::STAGE;
+  const int tpb = art.block_keys / kKT;                       // tiles per block
+  const int n_blocks = (n_tiles + tpb - 1) / tpb;
+  const int n_rounds = (n_blocks + kArtWarps - 1) / kArtWarps;
+  float* part = reinterpret_cast<float*>(smem + AC::OFF_PART);  // [2][warp][PART]
+  // round in which the folder decided to stop (n_rounds: not yet).  Every
+  // warp runs the same barriers: one per round, after the round's partials
+  // are published; after barrier r all warps leave the loop together when
+  // the stop was decided in a round < r (written before that barrier, so
+  // every warp sees it), and a value written during round r's fold never
+  // passes the test in round r.
+  volatile int* stop_round =
+      reinterpret_cast<volatile int*>(smem + AC::OFF_PART + 2 * kArtWarps * AC::PART * 4);
+  if (threadIdx.x == 0) *stop_round = n_rounds;
+  __syncthreads();
+
+  if (warp < kArtWarps) {
+    // ------------------------------------------------------- compute warp
+    const int t_row = row_ok ? qi / g : 0;
+    const int head = kvh * g + (row_ok ? qi % g : 0);
+    uint32_t qa[D / 16][4];
+    {
+      const float* qp = a.qr + (((int64_t)b * a.Tq + t_row) * a.hq + head) * D;
 #pragma unroll
-      for (int e = 0; e < (kKT * C::CH) / 32; ++e) {
-        const int idx = e * 32 + lane;
-        const int key = idx / C::CH, ch = idx % C::CH;
-        const int64_t kg = key0 + key;
-        const bool valid = kg >= 0;
-        const int64_t off = base_off + (valid ? kg : 0) * key_stride + ch * 8;
-        cp_async16(sbase + swz<D>(key, ch), Kg + off, valid);
-        cp_async16(sbase + C::TILE + swz<D>(key, ch), Vg + off, valid);
+      for (int ks = 0; ks < D / 16; ++ks) {
+        float x[4];
+        x[0] = row_ok ? qp[16 * ks + qc] : 0.f;
+        x[1] = row_ok ? qp[16 * ks + qc + 1] : 0.f;
+        x[2] = row_ok ? qp[16 * ks + qc + 8] : 0.f;
+        x[3] = row_ok ? qp[16 * ks + qc + 9] : 0.f;
+        float h[4], l[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          h[e] = __bfloat162float(__float2bfloat16_rn(x[e]));
+          l[e] = x[e] - h[e];
+        }
+        qa[ks][0] = pack_bf16(h[0], h[1]);
+        qa[ks][1] = pack_bf16(l[0], l[1]);
+        qa[ks][2] = pack_bf16(h[2], h[3]);
+        qa[ks][3] = pack_bf16(l[2], l[3]);
       }
     }
-    cp_async_commit();
-  };
-  float o[D / 8][4];
+    const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(smem)) + warp * AC::RING;
+    const __nv_bfloat16* Kg = static_cast<const __nv_bfloat16*>(a.k_ret);
+    const __nv_bfloat16* Vg = static_cast<const __nv_bfloat16*>(a.v_ret);
+    const int64_t key_stride = (int64_t)a.hkv * D;
+    const int64_t base_off = ((int64_t)b * T) * key_stride + (int64_t)kvh * D;
+    // this warp's k-th tile: tile (4 * (k / tpb) + warp) * tpb + k % tpb of
+    // the walk; walk tile s covers keys [T - 32 (s + 1), T - 32 s), clipped at 0
+    auto walk_tile = [&](int k) { return ((k / tpb) * kArtWarps + warp) * tpb + k % tpb; };
+    auto issue = [&](int k) {
+      const int it = walk_tile(k);
+      if (k < n_rounds * tpb && it < n_tiles && ((k / tpb) * kArtWarps + warp) < n_blocks) {
+        const int64_t key0 = T - (int64_t)kKT * (it + 1);
+        const uint32_t sbase = base + (k % kArtStages) * C::STAGE;
 #pragma unroll
-  for (int j = 0; j < D / 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
-  float prev[D / 8][2];
+        for (int e = 0; e < (kKT * C::CH) / 32; ++e) {
+          const int idx = e * 32 + lane;
+          const int key = idx / C::CH, ch = idx % C::CH;
+          const int64_t kg = key0 + key;
+          const bool valid = kg >= 0;
+          const int64_t off = base_off + (valid ? kg : 0) * key_stride + ch * 8;
+          cp_async16(sbase + swz<D>(key, ch), Kg + off, valid);
+          cp_async16(sbase + C::TILE + swz<D>(key, ch), Vg + off, valid);
+        }
+      }
+      cp_async_commit();
+    };
 #pragma unroll
-  for (int j = 0; j < D / 8; ++j) prev[j][0] = prev[j][1] = 0.f;
-  float prev_sq = 0.f;
-  float m_run = -INFINITY, l_run = 0.f;
-  int run = 0, blocks = 0;
+    for (int s2 = 0; s2 < kArtStages - 1; ++s2) issue(s2);
+    int k = 0;
+    for (int r = 0; r < n_rounds; ++r) {
+      const int blk = r * kArtWarps + warp;
+      float o[D / 8][4];
 #pragma unroll
-  for (int s2 = 0; s2 < kArtStages - 1; ++s2) issue(s2);
-  int it = 0;
-  for (; it < n_tiles; ++it) {
-    issue(it + kArtStages - 1);
-    cp_async_wait<kArtStages - 1>();
-    __syncwarp();
-    const uint32_t sK = base + (it % kArtStages) * C::STAGE;
-    const uint32_t sV = sK + C::TILE;
-    const int64_t key0 = T - (int64_t)kKT * (it + 1);
-    float sc[4][4];
+      for (int j = 0; j < D / 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+      float m_b = -INFINITY, l_b = 0.f;
+      for (int t = 0; t < tpb; ++t, ++k) {
+        issue(k + kArtStages - 1);
+        cp_async_wait<kArtStages - 1>();
+        __syncwarp();
+        const int it = walk_tile(k);
+        if (blk < n_blocks && it < n_tiles) {
+          const uint32_t sK = base + (k % kArtStages) * C::STAGE;
+          const uint32_t sV = sK + C::TILE;
+          const int64_t key0 = T - (int64_t)kKT * (it + 1);
+          float sc[4][4];
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+          for (int nt = 0; nt < 4; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt) {
+          for (int nt = 0; nt < 4; ++nt) {
 #pragma unroll
-      for (int kk = 0; kk < D / 32; ++kk) {
-        uint32_t b0, b1, b2, b3;
-        const int key = nt * 8 + (lane & 7);
-        const int ch = kk * 4 + (lane >> 3);
-        ldsm_x4(sK + swz<D>(key, ch), b0, b1, b2, b3);
-        mma_bf16(sc[nt], qa[2 * kk][0], qa[2 * kk][1], qa[2 * kk][2], qa[2 * kk][3], b0, b1);
-        mma_bf16(sc[nt], qa[2 * kk + 1][0], qa[2 * kk + 1][1], qa[2 * kk + 1][2], qa[2 * kk + 1][3], b2, b3);
+            for (int kk = 0; kk < D / 32; ++kk) {
+              uint32_t b0, b1, b2, b3;
+              const int key = nt * 8 + (lane & 7);
+              const int ch = kk * 4 + (lane >> 3);
+              ldsm_x4(sK + swz<D>(key, ch), b0, b1, b2, b3);
+              mma_bf16(sc[nt], qa[2 * kk][0], qa[2 * kk][1], qa[2 * kk][2], qa[2 * kk][3], b0, b1);
+              mma_bf16(sc[nt], qa[2 * kk + 1][0], qa[2 * kk + 1][1], qa[2 * kk + 1][2], qa[2 * kk + 1][3], b2, b3);
+            }
+          }
+          float sv[4][2];
+          float mt = -INFINITY;
+#pragma unroll
+          for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int64_t kg = key0 + nt * 8 + qc + e;
+              const float x = (kg >= 0) ? sc[nt][e] + sc[nt][e + 2] : -INFINITY;
+              sv[nt][e] = x;
+              mt = fmaxf(mt, x);
+            }
+          mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
+          mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
+          const float m_new = fmaxf(m_b, mt);
+          const float alpha = fast_exp2(m_b - m_new);
+          m_b = m_new;
+          l_b *= alpha;
+#pragma unroll
+          for (int j = 0; j < D / 8; ++j) {
+            o[j][0] *= alpha;
+            o[j][1] *= alpha;
+          }
+          uint32_t pa_[4];
+#pragma unroll
+          for (int nt = 0; nt < 4; ++nt) {
+            const float p0 = fast_exp2(sv[nt][0] - m_new), p1 = fast_exp2(sv[nt][1] - m_new);
+            l_b += p0 + p1;
+            pa_[nt] = pack_bf16(p0, p1);
+          }
+#pragma unroll
+          for (int k2 = 0; k2 < 2; ++k2) {
+#pragma unroll
+            for (int cj = 0; cj < D / 16; ++cj) {
+              uint32_t b0, b1, b2, b3;
+              const int mtx = lane >> 3;
+              const int key = k2 * 16 + (mtx & 1) * 8 + (lane & 7);
+              const int ch = cj * 2 + (mtx >> 1);
+              ldsm_x4_t(sV + swz<D>(key, ch), b0, b1, b2, b3);
+              mma_bf16(o[2 * cj], pa_[2 * k2], 0u, pa_[2 * k2 + 1], 0u, b0, b1);
+              mma_bf16(o[2 * cj + 1], pa_[2 * k2], 0u, pa_[2 * k2 + 1], 0u, b2, b3);
+            }
+          }
+        }
+        __syncwarp();   // the stage is refilled by a later issue
+      }
+      // the block's partial (unnormalised A, m, l) into the round's slot
+      l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
+      l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
+      float* slot = part + ((r & 1) * kArtWarps + warp) * AC::PART;
+#pragma unroll
+      for (int j = 0; j < D / 8; ++j)
+        *reinterpret_cast<float2*>(slot + qi * D + 8 * j + qc) = make_float2(o[j][0], o[j][1]);
+      if ((lane & 3) == 0) {
+        slot[AC::PART_O + qi] = m_b;
+        slot[AC::PART_O + 8 + qi] = l_b;
+      }
+      __syncthreads();   // round r published; the folder takes it while this warp goes on
+      if (*stop_round < r) break;
+    }
+    cp_async_wait<0>();
+  } else {
+    // ------------------------------------------------------------- folder
+    float O[D / 8][2];
+#pragma unroll
+    for (int j = 0; j < D / 8; ++j) O[j][0] = O[j][1] = 0.f;
+    float prev[D / 8][2];
+#pragma unroll
+    for (int j = 0; j < D / 8; ++j) prev[j][0] = prev[j][1] = 0.f;
+    float prev_sq = 0.f;
+    float m_run = -INFINITY, l_run = 0.f;
+    int run = 0, blocks = 0;
+    bool done = false;
+    for (int r = 0; r < n_rounds; ++r) {
+      __syncthreads();   // round r published
+      if (*stop_round < r) break;
+      for (int w = 0; w < kArtWarps && !done; ++w) {
+        const int blk = r * kArtWarps + w;
+        if (blk >= n_blocks) break;
+        const float* slot = part + ((r & 1) * kArtWarps + w) * AC::PART;
+        const float mb = slot[AC::PART_O + qi], lb = slot[AC::PART_O + 8 + qi];
+        const float m_new = fmaxf(m_run, mb);
+        const float ca = (m_run == -INFINITY) ? 0.f : fast_exp2(m_run - m_new);
+        const float cb = (mb == -INFINITY) ? 0.f : fast_exp2(mb - m_new);
+#pragma unroll
+        for (int j = 0; j < D / 8; ++j) {
+          const float2 v = *reinterpret_cast<const float2*>(slot + qi * D + 8 * j + qc);
+          O[j][0] = O[j][0] * ca + v.x * cb;
+          O[j][1] = O[j][1] * ca + v.y * cb;
+        }
+        l_run = l_run * ca + lb * cb;
+        m_run = m_new;
+        // stability of the normalised output after this block
+        ++blocks;
+        const float inv = 1.f / l_run;
+        float sq = 0.f, dot = 0.f;
+#pragma unroll
+        for (int j = 0; j < D / 8; ++j) {
+          const float x0 = O[j][0] * inv, x1 = O[j][1] * inv;
+          sq = fmaf(x0, x0, fmaf(x1, x1, sq));
+          dot = fmaf(x0, prev[j][0], fmaf(x1, prev[j][1], dot));
+          prev[j][0] = x0;
+          prev[j][1] = x1;
+        }
+        sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+        sq += __shfl_xor_sync(0xffffffffu, sq, 2);
+        dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+        dot += __shfl_xor_sync(0xffffffffu, dot, 2);
+        bool stable = true;
+        if (blocks >= 2 && row_ok) {
+          const float nx = sqrtf(sq), np = sqrtf(prev_sq);
+          stable = fabsf(nx - np) <= art.tau * np && 1.f - dot / (nx * np) <= art.phi;
+        } else if (row_ok) {
+          stable = false;
+        }
+        prev_sq = sq;
+        run = __all_sync(0xffffffffu, stable) ? run + 1 : 0;
+        if (run >= art.patience) done = true;
+      }
+      if (done) {
+        if (lane == 0) *stop_round = r;
+        __syncwarp();
       }
     }
-    float sv[4][2];
-    float mt = -INFINITY;
+    if (lane == 0 && art.visited) art.visited[(int64_t)b * a.hkv + kvh] = blocks;
+    if (row_ok) {
+      const int t_row = qi / g;
+      const int head = kvh * g + qi % g;
+      const bool empty = (m_run == -INFINITY) || !(l_run > 0.f);
+      const float inv = empty ? 0.f : 1.f / l_run;
+      const int64_t orow = ((int64_t)b * a.Tq + t_row) * a.hq + head;
+      __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.o) + orow * D;
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int64_t kg = key0 + nt * 8 + qc + e;
-        const float x = (kg >= 0) ? sc[nt][e] + sc[nt][e + 2] : -INFINITY;
-        sv[nt][e] = x;
-        mt = fmaxf(mt, x);
-      }
-    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
-    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
-    const float m_new = fmaxf(m_run, mt);
-    const float alpha = fast_exp2(m_run - m_new);
-    m_run = m_new;
-    l_run *= alpha;
-#pragma unroll
-    for (int j = 0; j < D / 8; ++j) {
-      o[j][0] *= alpha;
-      o[j][1] *= alpha;
-    }
-    uint32_t pa_[4];
-#pragma unroll
-    for (int nt = 0; nt < 4; ++nt) {
-      const float p0 = fast_exp2(sv[nt][0] - m_new), p1 = fast_exp2(sv[nt][1] - m_new);
-      l_run += p0 + p1;
-      pa_[nt] = pack_bf16(p0, p1);
-    }
-#pragma unroll
-    for (int k2 = 0; k2 < 2; ++k2) {
-#pragma unroll
-      for (int cj = 0; cj < D / 16; ++cj) {
-        uint32_t b0, b1, b2, b3;
-        const int mtx = lane >> 3;
-        const int key = k2 * 16 + (mtx & 1) * 8 + (lane & 7);
-        const int ch = cj * 2 + (mtx >> 1);
-        ldsm_x4_t(sV + swz<D>(key, ch), b0, b1, b2, b3);
-        mma_bf16(o[2 * cj], pa_[2 * k2], 0u, pa_[2 * k2 + 1], 0u, b0, b1);
-        mma_bf16(o[2 * cj + 1], pa_[2 * k2], 0u, pa_[2 * k2 + 1], 0u, b2, b3);
-      }
-    }
-    __syncwarp();
-    // end of a block (or of the cache): stability of the normalised output
-    if ((it + 1) % tiles_per_block == 0 || it + 1 == n_tiles) {
-      ++blocks;
-      float l_tot = l_run;
-      l_tot += __shfl_xor_sync(0xffffffffu, l_tot, 1);
-      l_tot += __shfl_xor_sync(0xffffffffu, l_tot, 2);
-      const float inv = 1.f / l_tot;
-      float sq = 0.f, dot = 0.f;
-#pragma unroll
-      for (int j = 0; j < D / 8; ++j) {
-        const float x0 = o[j][0] * inv, x1 = o[j][1] * inv;
-        sq = fmaf(x0, x0, fmaf(x1, x1, sq));
-        dot = fmaf(x0, prev[j][0], fmaf(x1, prev[j][1], dot));
-        prev[j][0] = x0;
-        prev[j][1] = x1;
-      }
-      sq += __shfl_xor_sync(0xffffffffu, sq, 1);
-      sq += __shfl_xor_sync(0xffffffffu, sq, 2);
-      dot += __shfl_xor_sync(0xffffffffu, dot, 1);
-      dot += __shfl_xor_sync(0xffffffffu, dot, 2);
-      bool stable = true;
-      if (blocks >= 2 && row_ok) {
-        const float nx = sqrtf(sq), np = sqrtf(prev_sq);
-        stable = fabsf(nx - np) <= art.tau * np && 1.f - dot / (nx * np) <= art.phi;
-      } else if (row_ok) {
-        stable = false;
-      }
-      prev_sq = sq;
-      run = __all_sync(0xffffffffu, stable) ? run + 1 : 0;
-      if (run >= art.patience) {
-        ++it;
-        break;
-      }
+      for (int j = 0; j < D / 8; ++j)
+        *reinterpret_cast<__nv_bfloat162*>(dst + 8 * j + qc) = __floats2bfloat162_rn(O[j][0] * inv, O[j][1] * inv);
+      if ((lane & 3) == 0) a.lse[orow] = empty ? -INFINITY : (m_run + __log2f(l_run)) * kLn2f;
     }
   }
-  cp_async_wait<0>();
-  l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
-  l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
-  if (lane == 0 && art.visited) art.visited[(int64_t)b * a.hkv + kvh] = blocks;
-  if (!row_ok) return;
-  const bool empty = (m_run == -INFINITY);
-  const float inv = empty ? 0.f : 1.f / l_run;
-  const int64_t orow = ((int64_t)b * a.Tq + t_row) * a.hq + head;
-  __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.o) + orow * D;
-#pragma unroll
-  for (int j = 0; j < D / 8; ++j)
-    *reinterpret_cast<__nv_bfloat162*>(dst + 8 * j + qc) = __floats2bfloat162_rn(o[j][0] * inv, o[j][1] * inv);
-  if ((lane & 3) == 0) a.lse[orow] = empty ? -INFINITY : (m_run + __log2f(l_run)) * kLn2f;
 }
 
 template <int D>
@@ -668,17 +752,17 @@ int launch_phase2_art(const Phase2Args& a, const ArtArgs& art, cudaStream_t s) {
   const dim3 grid(a.B, a.hkv);
   if (a.B <= 0) return PA_OK;
   if (a.d == 128) {
-    const int sm = kArtStages * P2Cfg<128>::STAGE;
+    const int sm = ArtCfg<128>::SMEM;
     if (cudaFuncSetAttribute(phase2_art_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm) !=
         cudaSuccess)
       return PA_ERR_CUDA;
-    phase2_art_kernel<128><<<grid, 32, sm, s>>>(a, art);
+    phase2_art_kernel<128><<<grid, (kArtWarps + 1) * 32, sm, s>>>(a, art);
   } else {
-    const int sm = kArtStages * P2Cfg<64>::STAGE;
+    const int sm = ArtCfg<64>::SMEM;
     if (cudaFuncSetAttribute(phase2_art_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm) !=
         cudaSuccess)
       return PA_ERR_CUDA;
-    phase2_art_kernel<64><<<grid, 32, sm, s>>>(a, art);
+    phase2_art_kernel<64><<<grid, (kArtWarps + 1) * 32, sm, s>>>(a, art);
   }
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
