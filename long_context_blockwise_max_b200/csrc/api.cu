@@ -481,4 +481,33 @@ int pa_testing_phase1_stall(const void* q, const void* k, const void* v, int64_t
                        static_cast<uint64_t>(wait_limit_us) * 1000ull, 1);
 }
 
+int pa_testing_phase2_stall(const void* q, const void* k_ret, const void* v_ret, int32_t B, int32_t Tq,
+                            int64_t T, int32_t n_shards, int32_t hq, int32_t hkv, int32_t d, void* o,
+                            float* lse, void* ws, size_t ws_bytes, int32_t wait_limit_us, void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (wait_limit_us <= 0 || wait_limit_us > 10000000) return PA_ERR_INVALID;
+  int rc = check_heads(hq, hkv, d, PA_BF16);
+  if (rc) return rc;
+  if (B < 1 || Tq < 1 || T < 1 || n_shards < 1 || n_shards > 4096) return PA_ERR_INVALID;
+  if (!q || !k_ret || !v_ret || !o || !lse) return PA_ERR_INVALID;
+  const size_t need = phase2_workspace_bytes(B, Tq, T, n_shards, hq, hkv, d);
+  rc = check_ws(ws, ws_bytes, need);
+  if (rc) return rc;
+  Phase2Args a;
+  a.dtype = PA_BF16;
+  a.q = q; a.B = B; a.Tq = Tq; a.q_pos0 = 0; a.rope_theta = 0.0;
+  a.k_ret = k_ret; a.v_ret = v_ret; a.T = T;
+  a.n_shards = n_shards;
+  a.n_split = phase2_split(B, Tq, T, n_shards, hq, hkv);
+  a.hq = hq; a.hkv = hkv; a.d = d;
+  a.o = o; a.lse = lse; a.part_o_opt = nullptr; a.part_lse_opt = nullptr;
+  a.wait_limit_ns = static_cast<uint64_t>(wait_limit_us) * 1000ull;
+  a.stall = 1;
+  if (!phase2_tc_supported(a)) return PA_ERR_UNSUPPORTED;   // tensor-core query path only
+  rc = clear_status(ws, s);
+  if (rc) return rc;
+  carve_phase2(a, ws);
+  return launch_phase2(a, s);
+}
+
 }  // extern "C"

@@ -109,6 +109,9 @@ struct Phase2Args {
   const void* v_self = nullptr;
   int64_t self_cap = 0, self_len = 0;
   int has_self = 0;
+  // bounded-wait limit of the tensor-core query kernel and a test-only stall
+  uint64_t wait_limit_ns = 1000000000ull;
+  int stall = 0;
 };
 
 // One Phase-2 work unit: a split of a context shard, or (the last unit, when

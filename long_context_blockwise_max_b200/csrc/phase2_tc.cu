@@ -32,8 +32,8 @@
 //               own cache, past the row's causal limit); lazy rescale of O.
 // Output: the unit's normalised partial A and its lse per row, the same
 // contract as the other Phase-2 kernels, merged by merge_kernel.
-// Every wait is bounded (1 s); on expiry the CTA records PA_ERR_TIMEOUT,
-// drains its copies and MMAs, frees TMEM and returns.
+// Every wait is bounded (1 s by default); on expiry the CTA records
+// PA_ERR_TIMEOUT, drains its copies and MMAs, frees TMEM and returns.
 #include <cuda_fp16.h>
 #include <cudaTypedefs.h>
 
@@ -48,7 +48,6 @@ namespace {
 constexpr int kKT = 128;           // keys per tile
 constexpr int kMaxStages = 4;
 constexpr int kConvThreads = 64;   // warps 2-3
-constexpr uint64_t kWaitNs = 1000000000ull;
 
 template <int D>
 struct QtCfg {
@@ -118,6 +117,7 @@ __global__ void __launch_bounds__(384, 1) phase2_tc_kernel(const __grid_constant
   uint8_t* sV = smem + C::OFF_V;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const Phase2Args& a = p.a;
+  const uint64_t wait_ns = a.wait_limit_ns;   // limit of every bounded wait
 
   // work item: pair fastest (CTAs that share a unit's K / V run together)
   int idx = blockIdx.x;
@@ -179,7 +179,7 @@ __global__ void __launch_bounds__(384, 1) phase2_tc_kernel(const __grid_constant
       // Q: row tile t covers tokens [mt * 128 / g, +128 / g) of batch b; the
       // box (64 x g heads x 128 / g tokens) lands as rows token * g + head
       const int tpt = 128 / g;
-      mbar_arrive_expect_tx(&bars->q_full, 2 * C::TILE);
+      mbar_arrive_expect_tx(&bars->q_full, 2 * C::TILE + (a.stall ? 16 : 0));
       for (int t = 0; t < 2; ++t) {
         const int tok = b * a.Tq + (2 * pair + t) * tpt;
         for (int kb = 0; kb < C::NKB; ++kb)
@@ -192,12 +192,12 @@ __global__ void __launch_bounds__(384, 1) phase2_tc_kernel(const __grid_constant
       for (int j = 0; j < nkv; ++j) {
         const int row = row_base + j * kKT;
         const int sk = j % KST, sv = j % VST;
-        if (!mbar_wait(&bars->k_empty[sk], ((j / KST) & 1) ^ 1, abort, kWaitNs, gabort)) { fail(1); break; }
+        if (!mbar_wait(&bars->k_empty[sk], ((j / KST) & 1) ^ 1, abort, wait_ns, gabort)) { fail(1); break; }
         mbar_arrive_expect_tx(&bars->k_full[sk], C::TILE);
         for (int kb = 0; kb < C::NKB; ++kb)
           tma_load_3d(sK + sk * C::TILE + kb * C::KB_BYTES, mk, &bars->k_full[sk], kb * 64, kvh, row);
         ++armed_k[sk];
-        if (!mbar_wait(&bars->v_empty[sv], ((j / VST) & 1) ^ 1, abort, kWaitNs, gabort)) { fail(2); break; }
+        if (!mbar_wait(&bars->v_empty[sv], ((j / VST) & 1) ^ 1, abort, wait_ns, gabort)) { fail(2); break; }
         mbar_arrive_expect_tx(&bars->v_full[sv], C::TILE);
         for (int kb = 0; kb < C::NKB; ++kb)
           tma_load_3d(sV + sv * C::TILE + kb * C::KB_BYTES, mv, &bars->v_full[sv], kb * 64, kvh, row);
@@ -205,11 +205,11 @@ __global__ void __launch_bounds__(384, 1) phase2_tc_kernel(const __grid_constant
       }
       // Drain: every copy this thread started has landed before the CTA ends.
       int zero = 0;
-      mbar_wait(&bars->q_full, 0, &zero, kWaitNs);
+      mbar_wait(&bars->q_full, 0, &zero, wait_ns);
       for (int s = 0; s < KST; ++s)
-        if (armed_k[s]) mbar_wait(&bars->k_full[s], (armed_k[s] - 1) & 1, &zero, kWaitNs);
+        if (armed_k[s]) mbar_wait(&bars->k_full[s], (armed_k[s] - 1) & 1, &zero, wait_ns);
       for (int s = 0; s < VST; ++s)
-        if (armed_v[s]) mbar_wait(&bars->v_full[s], (armed_v[s] - 1) & 1, &zero, kWaitNs);
+        if (armed_v[s]) mbar_wait(&bars->v_full[s], (armed_v[s] - 1) & 1, &zero, wait_ns);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
@@ -234,14 +234,14 @@ __global__ void __launch_bounds__(384, 1) phase2_tc_kernel(const __grid_constant
           mma_ts(d_tmem, tmem + t * 256 + ks * 8, db, C::IDESC_PV, (acc | ks) != 0);
         }
       };
-      bool ok = mbar_wait(&bars->q_full, 0, abort, kWaitNs, gabort);
+      bool ok = mbar_wait(&bars->q_full, 0, abort, wait_ns, gabort);
       if (!ok) fail(3);
       for (int j = 0; ok && j < nkv; ++j) {
         const int sv = j % VST;
         const int sk1 = (j + 1) % KST;
         const uint32_t pk1 = ((j + 1) / KST) & 1;
         if (j == 0) {
-          if (!mbar_wait(&bars->k_conv[0], 0, abort, kWaitNs, gabort)) { fail(4); break; }
+          if (!mbar_wait(&bars->k_conv[0], 0, abort, wait_ns, gabort)) { fail(4); break; }
           tc_fence_after();
           qk(0, 0);
           mma_commit(&bars->s_full[0]);
@@ -250,19 +250,19 @@ __global__ void __launch_bounds__(384, 1) phase2_tc_kernel(const __grid_constant
           mma_commit(&bars->k_empty[0]);
         }
         // tile 0: O0 += P0 V_j, then S0 = Q0 K_{j+1}
-        if (!mbar_wait(&bars->p_full[0], j & 1, abort, kWaitNs, gabort)) { fail(5); break; }
-        if (!mbar_wait(&bars->v_full[sv], (j / VST) & 1, abort, kWaitNs, gabort)) { fail(6); break; }
+        if (!mbar_wait(&bars->p_full[0], j & 1, abort, wait_ns, gabort)) { fail(5); break; }
+        if (!mbar_wait(&bars->v_full[sv], (j / VST) & 1, abort, wait_ns, gabort)) { fail(6); break; }
         tc_fence_after();
         pv(0, sv, j > 0);
         if (j == nkv - 1) mma_commit(&bars->o_final[0]);
         if (j + 1 < nkv) {
-          if (!mbar_wait(&bars->k_conv[sk1], pk1, abort, kWaitNs, gabort)) { fail(7); break; }
+          if (!mbar_wait(&bars->k_conv[sk1], pk1, abort, wait_ns, gabort)) { fail(7); break; }
           tc_fence_after();
           qk(0, sk1);
           mma_commit(&bars->s_full[0]);
         }
         // tile 1: O1 += P1 V_j, then S1 = Q1 K_{j+1}
-        if (!mbar_wait(&bars->p_full[1], j & 1, abort, kWaitNs, gabort)) { fail(8); break; }
+        if (!mbar_wait(&bars->p_full[1], j & 1, abort, wait_ns, gabort)) { fail(8); break; }
         tc_fence_after();
         pv(1, sv, j > 0);
         if (j == nkv - 1) mma_commit(&bars->o_final[1]);
@@ -276,7 +276,7 @@ __global__ void __launch_bounds__(384, 1) phase2_tc_kernel(const __grid_constant
       // Drain: all MMAs issued by this thread complete before TMEM is freed.
       int zero = 0;
       mma_commit(&bars->drain);
-      mbar_wait(&bars->drain, 0, &zero, kWaitNs);
+      mbar_wait(&bars->drain, 0, &zero, wait_ns);
     }
   } else if (warp < 4) {
     // ------------------------------------------------------- K converters
@@ -284,7 +284,7 @@ __global__ void __launch_bounds__(384, 1) phase2_tc_kernel(const __grid_constant
     bool bad = false;
     for (int j = 0; j < nkv; ++j) {
       const int sk = j % KST;
-      if (!mbar_wait(&bars->k_full[sk], (j / KST) & 1, abort, kWaitNs, gabort)) { fail(12); break; }
+      if (!mbar_wait(&bars->k_full[sk], (j / KST) & 1, abort, wait_ns, gabort)) { fail(12); break; }
       uint4* tile = reinterpret_cast<uint4*>(sK + sk * C::TILE);
       constexpr int N16 = C::TILE / 16;   // 16-byte chunks per tile
 #pragma unroll 4
@@ -313,7 +313,7 @@ __global__ void __launch_bounds__(384, 1) phase2_tc_kernel(const __grid_constant
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
-      if (!mbar_wait(&bars->s_full[t], j & 1, abort, kWaitNs, gabort)) { fail(9); ok = false; break; }
+      if (!mbar_wait(&bars->s_full[t], j & 1, abort, wait_ns, gabort)) { fail(9); ok = false; break; }
       tc_fence_after();
       uint32_t sr[kKT];
       tmem_ld_x128(s_tmem, sr);
@@ -391,7 +391,7 @@ __global__ void __launch_bounds__(384, 1) phase2_tc_kernel(const __grid_constant
         for (int c = 0; c < D / 4; ++c) reinterpret_cast<float4*>(dst)[c] = make_float4(0.f, 0.f, 0.f, 0.f);
         a.unit_lse[orow] = -INFINITY;
       }
-    } else if (ok && mbar_wait(&bars->o_final[t], 0, abort, kWaitNs, gabort)) {
+    } else if (ok && mbar_wait(&bars->o_final[t], 0, abort, wait_ns, gabort)) {
       tc_fence_after();
       const bool empty = !(l_run > 0.f);
       const float inv = empty ? 0.f : 1.f / l_run;

@@ -77,6 +77,8 @@ def _load() -> ctypes.CDLL:
     }
     # test hook (include/pulsar_testing.h)
     sig["pa_testing_phase1_stall"] = (ctypes.c_int, [P, P, P, I64, I32, I32, I32, I32, P, P, P, P, SZ, I32, P])
+    sig["pa_testing_phase2_stall"] = (ctypes.c_int, [P, P, P, I32, I32, I64, I32, I32, I32, I32, P, P, P, SZ, I32,
+                                                     P])
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
         fn.restype, fn.argtypes = res, args
@@ -421,4 +423,21 @@ def pa_testing_phase1_stall(q, k, v, block, wait_limit_us):
     rc = _lib.pa_testing_phase1_stall(_ptr(q), _ptr(k), _ptr(v), L, hq, hkv, d, block, _ptr(o), _ptr(k_ret),
                                       _ptr(v_ret), _ptr(ws), ws.numel(), int(wait_limit_us), _stream())
     _check(rc, "pa_testing_phase1_stall")
+    return ws
+
+
+def pa_testing_phase2_stall(q, k_ret, v_ret, n_shards, wait_limit_us):
+    """Test hook: Phase-2 attention (no RoPE) through the tensor-core query
+    kernel with one unsatisfiable barrier and waits limited to
+    ``wait_limit_us``; the workspace status then reads PA_ERR_TIMEOUT.
+    Returns the workspace."""
+    _dev(q, k_ret, v_ret)
+    B, Tq, hq, d = q.shape
+    T, hkv = k_ret.shape[1], k_ret.shape[2]
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Tq, hq), dtype=torch.float32, device=q.device)
+    ws = _workspace(pa_phase2_workspace_size(B, Tq, T, n_shards, hq, hkv, d), q.device)
+    rc = _lib.pa_testing_phase2_stall(_ptr(q), _ptr(k_ret), _ptr(v_ret), B, Tq, T, n_shards, hq, hkv, d, _ptr(o),
+                                      _ptr(lse), _ptr(ws), ws.numel(), int(wait_limit_us), _stream())
+    _check(rc, "pa_testing_phase2_stall")
     return ws

@@ -1,7 +1,8 @@
 """Failure detection on the GPU without a fault: a barrier that can never
-complete makes every bounded wait of the tensor-core Phase-1 kernel run
-out; the kernel records PA_ERR_TIMEOUT, frees its resources and returns,
-and the next call on the same context computes correct results."""
+complete makes every bounded wait of a tensor-core kernel (Phase 1, and the
+Phase-2 query kernel) run out; the kernel records PA_ERR_TIMEOUT, frees its
+resources and returns, and the next call on the same context computes
+correct results."""
 import time
 
 import numpy as np
@@ -34,3 +35,22 @@ def test_stalled_barrier_times_out_and_context_survives():
     for i, (ro, rl) in enumerate(oracle.phase1_encode(f64(q), f64(k), f64(v), pos, 10000.0)):
         assert_close(f64(o[off[i]:off[i + 1]].cpu()), ro, O_TOL[torch.bfloat16], "O")
         assert_close(lse[off[i]:off[i + 1]].cpu().double().numpy(), rl, LSE_TOL, "lse")
+
+
+
+def test_stalled_query_kernel_times_out_and_context_survives():
+    from long_context_blockwise_max_b200 import pulsar as P
+    B, Tq, hq, hkv, d, T, S = 1, 64, 8, 2, 128, 1000, 3   # 256 query rows per kv head
+    q = workloads.normal((B, Tq, hq, d), 93, torch.bfloat16)
+    kc = workloads.normal((B, T, hkv, d), 94, torch.bfloat16)
+    vc = workloads.normal((B, T, hkv, d), 95, torch.bfloat16)
+    qd, kd, vd = q.to(DEV), kc.to(DEV), vc.to(DEV)
+    t0 = time.time()
+    ws = P.pa_testing_phase2_stall(qd, kd, vd, S, wait_limit_us=20000)
+    assert P.pa_workspace_status(ws) == -5          # PA_ERR_TIMEOUT
+    assert time.time() - t0 < 30.0
+    o, lse, _, _, ws2 = P.star_phase2_attend(qd, kd, vd, S, q_pos0=T, rope_theta=0.0)
+    assert P.pa_workspace_status(ws2) == 0
+    ro, rl, _, _ = oracle.phase2_attend(f64(q), f64(kc), f64(vc), S, T, 0.0)
+    assert_close(f64(o.cpu()), ro, O_TOL[torch.bfloat16], "O")
+    assert_close(lse.cpu().double().numpy(), rl, LSE_TOL, "lse")

@@ -149,3 +149,23 @@ def test_query_kernel_range_status(P, where):
         q[0, 5, 3, 9] = 1.0
     *_, ws = P.star_phase2_attend(q.to(DEV), kc.to(DEV), vc.to(DEV), S, q_pos0=T, rope_theta=0.0)
     assert P.pa_workspace_status(ws) == 0
+
+
+def test_query_32k_sampled_groups(P):
+    # the 32K workload's 64-token query over its 4 retained blocks (the
+    # tensor-core query kernel: 256 rows per kv head, 4 splits per shard)
+    w = workloads.LLAMA_32K
+    q = w.query(device=DEV)
+    kc = workloads.normal((1, w.L, w.hkv, w.d), workloads.SEED_KC, w.dtype, DEV)
+    vc = workloads.normal((1, w.L, w.hkv, w.d), workloads.SEED_VC, w.dtype, DEV)
+    o, lse, po, pl, ws = P.star_phase2_attend(q, kc, vc, w.n_blocks, q_pos0=w.L, rope_theta=w.rope_theta,
+                                              want_partials=True)
+    assert P.pa_workspace_status(ws) == 0
+    g = w.hq // w.hkv
+    for kvh in (1, 7):
+        ro, rl, ra, rs = _oracle_group(q, kc, vc, 0, kvh, g, w.n_blocks, w.L, w.rope_theta)
+        hs = slice(kvh * g, (kvh + 1) * g)
+        assert_close(f64(o[:, :, hs].cpu()), ro, O_TOL[torch.bfloat16], "O")
+        assert_close(lse[:, :, hs].cpu().double().numpy(), rl, LSE_TOL, "lse")
+        assert_close(f64(po[:, :, :, hs].cpu()), ra, O_TOL[torch.bfloat16], "A_h")
+        assert_close(pl[:, :, :, hs].cpu().double().numpy(), rs, LSE_TOL, "s_h")
