@@ -78,7 +78,8 @@ def test_tiny_fp32_all_rows(P, star):
 BF16_CASES = [
     # (L, block, hq, hkv, d, sink, chunk, k, theta)
     (4 * 640, 640, 8, 2, 128, 64, 32, 3, 500000.0),     # ragged host lengths 640/800/896/992
-    (3 * 384, 384, 4, 4, 64, 32, 16, 5, 10000.0),       # d = 64, MHA, 16-token chunks
+    (3 * 384, 384, 4, 4, 64, 32, 16, 5, 10000.0),       # d = 64, MHA (g = 1: SIMT kernel), 16-token chunks
+    (3 * 384, 384, 8, 2, 64, 32, 16, 5, 10000.0),       # d = 64, g = 4: tensor-core kernel
     (1024, 1024, 8, 1, 128, 64, 32, 4, 10000.0),        # N = 1: plain causal attention
 ]
 
