@@ -1,0 +1,96 @@
+"""GPU parity on seeded random shapes: Phase-1 encoding (Pulsar and Star) and
+Phase-2 attention against the fp64 oracle, for sizes drawn around every
+kernel's boundaries (ragged hosts and tiles, row counts on both sides of the
+tensor-core query path, GQA ratios that do and do not divide 128, empty and
+one-key shards, fp32 and bf16, d = 64 and 128).  Every case is small enough
+for the oracle to check all outputs."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from helpers import LSE_TOL, O_TOL, assert_close, f64
+from long_context_blockwise_max_b200 import workloads
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda:0")
+
+
+@pytest.fixture(scope="module")
+def P():
+    from long_context_blockwise_max_b200 import pulsar
+    return pulsar
+
+
+def _phase1_case(seed):
+    rng = np.random.default_rng(1000 + seed)
+    dtype = torch.bfloat16 if seed % 3 else torch.float32
+    d = int(rng.choice([64, 128]))
+    hkv = int(rng.choice([1, 2, 4]))
+    g = int(rng.choice([1, 2, 4])) if dtype == torch.float32 else int(rng.choice([1, 2, 3, 4, 8]))
+    chunk = int(rng.choice([16, 32]))
+    block = chunk * int(rng.integers(4, 13))
+    n = int(rng.integers(1, 5))
+    sink = 16 * int(rng.integers(0, min(block // 16, 5) + 1))
+    k = int(rng.integers(0, block // chunk // 2 + 1))
+    star = bool(rng.integers(0, 2))
+    return dict(dtype=dtype, d=d, hq=g * hkv, hkv=hkv, chunk=chunk, block=block, n=n, sink=sink, k=k, star=star,
+                theta=float(rng.choice([1e4, 5e5])))
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_phase1_random_shape(P, seed):
+    c = _phase1_case(seed)
+    L = c["n"] * c["block"]
+    q = workloads.normal((L, c["hq"], c["d"]), 200 + seed, c["dtype"])
+    k = workloads.normal((L, c["hkv"], c["d"]), 300 + seed, c["dtype"])
+    v = workloads.normal((L, c["hkv"], c["d"]), 400 + seed, c["dtype"])
+    rng = np.random.default_rng(seed)
+    C = c["block"] // c["chunk"]
+    sel = np.sort(np.stack([rng.choice(C, c["k"], replace=False) for _ in range(c["n"])]), axis=1).astype(np.int32)
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    if c["star"]:
+        o, lse, kr, vr, off, ws = P.star_phase1_encode(qd, kd, vd, c["theta"], c["block"])
+        pos = oracle.host_positions(L, c["block"], 0, 16, np.zeros((c["n"], 0), dtype=np.int64), star=True)
+    else:
+        o, lse, kr, vr, off, ws = P.pulsar_phase1_encode(qd, kd, vd, c["theta"], c["block"], c["sink"], c["chunk"],
+                                                         c["k"], torch.from_numpy(sel).to(DEV))
+        pos = oracle.host_positions(L, c["block"], c["sink"], c["chunk"], sel.astype(np.int64), star=False)
+    assert P.pa_workspace_status(ws) == 0, c
+    assert off == oracle.host_row_offsets(pos).tolist()
+    ref = oracle.phase1_encode(f64(q), f64(k), f64(v), pos, c["theta"])
+    o_c, lse_c = o.cpu(), lse.cpu()
+    for i, (ro, rl) in enumerate(ref):
+        assert_close(f64(o_c[off[i]:off[i + 1]]), ro, O_TOL[c["dtype"]], f"{c} host {i} O")
+        assert_close(lse_c[off[i]:off[i + 1]].double().numpy(), rl, LSE_TOL, f"{c} host {i} lse")
+    assert torch.equal(vr.cpu(), v)
+
+
+def _phase2_case(seed):
+    rng = np.random.default_rng(2000 + seed)
+    dtype = torch.bfloat16 if seed % 4 else torch.float32
+    d = int(rng.choice([64, 128]))
+    g = int(rng.choice([1, 2, 3, 4, 8, 16]))
+    hkv = int(rng.choice([1, 2])) if g >= 8 else int(rng.choice([1, 2, 4, 8]))
+    # row counts on both sides of the tensor-core path (>= 64 rows per kv head)
+    Tq = int(rng.choice([1, 2, 5, max(1, 64 // g - 1), max(1, 64 // g), int(rng.integers(1, 130))]))
+    B = int(rng.integers(1, 4))
+    T = int(rng.choice([0, 1, 37, 128, 700, int(rng.integers(129, 4000))]))
+    S = int(rng.integers(1, 12))
+    return dict(dtype=dtype, d=d, hq=g * hkv, hkv=hkv, Tq=Tq, B=B, T=T, S=S, theta=float(rng.choice([0.0, 5e5])))
+
+
+@pytest.mark.parametrize("seed", range(16))
+def test_phase2_random_shape(P, seed):
+    c = _phase2_case(seed)
+    q = workloads.normal((c["B"], c["Tq"], c["hq"], c["d"]), 500 + seed, c["dtype"])
+    kc = workloads.normal((c["B"], c["T"], c["hkv"], c["d"]), 600 + seed, c["dtype"])
+    vc = workloads.normal((c["B"], c["T"], c["hkv"], c["d"]), 700 + seed, c["dtype"])
+    o, lse, po, pl, ws = P.star_phase2_attend(q.to(DEV), kc.to(DEV), vc.to(DEV), c["S"], q_pos0=c["T"],
+                                              rope_theta=c["theta"], want_partials=True)
+    assert P.pa_workspace_status(ws) == 0, c
+    ro, rl, ra, rs = oracle.phase2_attend(f64(q), f64(kc), f64(vc), c["S"], c["T"], c["theta"])
+    assert_close(f64(o.cpu()), ro, O_TOL[c["dtype"]], f"{c} O")
+    assert_close(lse.cpu().double().numpy(), rl, LSE_TOL, f"{c} lse")
+    assert_close(po.cpu().double().numpy(), ra, O_TOL[c["dtype"]], f"{c} A_h")
+    assert_close(pl.cpu().double().numpy(), rs, LSE_TOL, f"{c} s_h")
