@@ -480,6 +480,25 @@ def run_ours(args, rank, world, local_rank, dist_on):
         del dq, dk, dv, dk2
         torch.cuda.empty_cache()
 
+        # the 1M-token decode: batch 4 over a 16 GiB cache in 32 shards
+        SC = workloads.SCALE_1M
+        sq, sk, sv = SC.decode_inputs(device=dev)
+        B1, T1, S1 = SC.decode_batch, SC.decode_T, SC.decode_shards
+        so_ = torch.empty_like(sq)
+        sl_ = torch.empty((B1, 1, SC.hq), dtype=torch.float32, device=dev)
+        sws = torch.empty(P.pa_phase2_workspace_size(B1, 1, T1, S1, SC.hq, SC.hkv, SC.d), dtype=torch.uint8,
+                          device=dev)
+
+        def dec1m():
+            P.star_phase2_attend(sq, sk, sv, S1, q_pos0=T1, rope_theta=SC.rope_theta, o=so_, lse=sl_, ws=sws)
+        dec1m_ms, _ = timed(dec1m)
+        kv1m = 2.0 * B1 * T1 * SC.hkv * SC.d * 2
+        extra["phase2_decode_1m"] = {
+            "workload": SC.name, "ms": round(dec1m_ms, 4), "gb_s": round(kv1m / (dec1m_ms * 1e-3) / 1e9, 1),
+            "frac_hbm": round(kv1m / (dec1m_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4), "bytes_per_call": kv1m}
+        del sq, sk, sv
+        torch.cuda.empty_cache()
+
         # generation loop on the query host: the 64-token query, then 128
         # tokens generated one at a time over the retained 128K cache
         gen = 128
@@ -509,10 +528,29 @@ def run_ours(args, rank, world, local_rank, dist_on):
         g1.record()
         torch.cuda.synchronize()
         gen_ms = g0.elapsed_time(g1) / gen
+        # the same 128 steps captured once in a CUDA graph and replayed (each
+        # replay rewrites the same own-cache rows): GPU time per token without
+        # the Python / ctypes cost of the per-token call
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for i, (a_q, a_k, a_v) in enumerate(toks):
+                t = w.q_tokens + i
+                P.star_phase2_query_step(a_q, a_k, a_v, kr1, vr1, w.n_blocks, ks, vs, t, w.L + t, w.rope_theta,
+                                         o=go, lse=gl, ws=gws)
+        graph.replay()
+        torch.cuda.synchronize()
+        g0.record()
+        graph.replay()
+        g1.record()
+        torch.cuda.synchronize()
+        gen_graph_ms = g0.elapsed_time(g1) / gen
+        del graph
         cache_bytes = 2.0 * w.L * w.hkv * w.d * 2
         extra["generation"] = {"context": w.L, "query_tokens": w.q_tokens, "generated": gen,
                                "ms_per_token": round(gen_ms, 4), "tokens_per_s": round(1e3 / gen_ms, 1),
-                               "cache_gb_s": round(cache_bytes / (gen_ms * 1e-3) / 1e9, 1)}
+                               "cache_gb_s": round(cache_bytes / (gen_ms * 1e-3) / 1e9, 1),
+                               "graph_ms_per_token": round(gen_graph_ms, 4),
+                               "graph_cache_gb_s": round(cache_bytes / (gen_graph_ms * 1e-3) / 1e9, 1)}
         del gq, gk, gv, ks, vs, toks
 
         # summary scorers on the 128K and 1M token ids (selection alone)
@@ -536,6 +574,21 @@ def run_ours(args, rank, world, local_rank, dist_on):
                 a1.record()
                 torch.cuda.synchronize()
                 sc[f"{wl.name}:{name}_us"] = round(a0.elapsed_time(a1) / 10 * 1e3, 1)
+                # the same call captured once in a CUDA graph and replayed: the
+                # GPU time without the Python / ctypes enqueue cost per call
+                graph = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(graph):
+                    sel_call()
+                for _ in range(3):
+                    graph.replay()
+                torch.cuda.synchronize()
+                a0.record()
+                for _ in range(20):
+                    graph.replay()
+                a1.record()
+                torch.cuda.synchronize()
+                sc[f"{wl.name}:{name}_graph_us"] = round(a0.elapsed_time(a1) / 20 * 1e3, 1)
+                del graph
         extra["selection_us"] = sc
 
     q2_bytes = 2.0 * w.L * w.hkv * w.d * 2
@@ -655,8 +708,9 @@ def run_profile_case(name, steps, warmup):
     """One kernel family on a small workload, for ncu captures:
     phase1-32k (Pulsar Phase 1 incl. its RoPE prepass, 32K shape),
     decode-128k / decode-16k (Phase-2 decode, 16 queries over a 128K / 16K
-    cache in 8 shards), query-128k (Phase-2 64-token query).  Prints one JSON
-    line with the mean call time."""
+    cache in 8 shards), query-128k (Phase-2 64-token query), select-1m
+    (Max-IDF selection over the 1M-token ids).  Prints one JSON line with the
+    mean call time."""
     from long_context_blockwise_max_b200 import pulsar as P
     dev = torch.device("cuda", 0)
     if name == "phase1-32k":
@@ -689,6 +743,15 @@ def run_profile_case(name, steps, warmup):
 
         def call():
             P.star_phase2_attend(q, kc, vc, w.n_blocks, w.L, w.rope_theta, o=o, lse=lse, ws=ws)
+    elif name == "select-1m":
+        w = workloads.SCALE_1M
+        idd = torch.from_numpy(w.token_ids()).to(dev)
+        sel, _, _, _ = P.pulsar_select_summaries(idd, w.vocab, w.block, w.chunk, w.k_chunks)
+        sws = torch.empty(P.pa_select_workspace_size(w.L, w.vocab, w.block, w.chunk), dtype=torch.uint8,
+                          device=dev)
+
+        def call():
+            P.pulsar_select_summaries(idd, w.vocab, w.block, w.chunk, w.k_chunks, sel=sel, ws=sws)
     else:
         raise SystemExit(f"unknown profile case {name}")
     for _ in range(warmup):
@@ -712,7 +775,7 @@ def main():
     ap.add_argument("--headline-only", action="store_true", help="skip the side measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-case", default=None,
-                    help="run one kernel family on a small workload (phase1-32k, decode-128k, query-128k)")
+                    help="run one kernel family on a small workload (phase1-32k, decode-16k, decode-128k, query-128k, select-1m)")
     args = ap.parse_args()
     if args.profile_case:
         run_profile_case(args.profile_case, args.steps, args.warmup)

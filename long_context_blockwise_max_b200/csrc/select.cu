@@ -6,8 +6,10 @@
 // minimum document frequency, with identical ties.  Everything here is
 // integer arithmetic and bit-exact.
 //
-//  presence_mask_kernel : mask[t] |= 1 << j for every token t of block j
-//                         (blocks are the documents); df(t) = popc(mask[t]).
+//  presence_tile_kernel : mask[t] |= 1 << j for every token t of block j
+//                         (blocks are the documents); df(t) = popc(mask[t]);
+//                         per-tile dedupe in shared memory (presence_mask_kernel
+//                         for vocabularies above 2^20 ids).
 //  chunk_mindf_kernel   : one warp per chunk, min over its tokens of df.
 //  topk_kernel          : one CTA per block; histogram of min-df values
 //                         (1..N) -> threshold -> ordered compaction that keeps
@@ -37,6 +39,49 @@ __global__ void presence_mask_kernel(const int32_t* __restrict__ ids, int64_t L,
     const unsigned peers = __match_any_sync(0xffffffffu, key);
     if (ok && lane == __ffs(peers) - 1) {
       const unsigned long long bit = 1ull << j;
+      if (!(ld_cg_u64(mask + t) & bit)) atomicOr(mask + t, bit);
+    }
+  }
+}
+
+// Presence with a per-CTA dedupe: CTA = one tile of up to `tile` consecutive
+// ids inside one block (512 .. 4096 ids, about four CTAs per SM).  The tile's distinct ids are first
+// collected in a shared-memory bitmap of the vocabulary, then each distinct
+// id sets the block's bit in global memory once.  With Zipf-distributed ids
+// the frequent ids would otherwise send most of the tile's requests to the
+// same few global words.
+constexpr size_t kPresenceSmemMax = 128 * 1024;   // vocabularies up to 2^20 ids
+
+__global__ void __launch_bounds__(256) presence_tile_kernel(const int32_t* __restrict__ ids, int64_t L,
+                                                            int32_t vocab, int32_t block, int32_t tile,
+                                                            unsigned long long* __restrict__ mask,
+                                                            DeviceStatus* st) {
+  extern __shared__ uint32_t bm[];   // [ceil(vocab / 32)]
+  const int words = (vocab + 31) >> 5;
+  const int tiles_per_block = (block + tile - 1) / tile;
+  const int j = blockIdx.x / tiles_per_block;
+  const int64_t i0 = (int64_t)j * block + (int64_t)(blockIdx.x % tiles_per_block) * tile;
+  const int64_t i1 = min(min(i0 + tile, (int64_t)(j + 1) * block), L);
+  for (int w = threadIdx.x; w < words; w += blockDim.x) bm[w] = 0u;
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  // warp-uniform loop: lanes with equal ids elect one leader (__match_any_sync)
+  for (int64_t base = i0 + (threadIdx.x & ~31); base < i1; base += blockDim.x) {
+    const int64_t i = base + lane;
+    const bool valid = i < i1;
+    const int t = valid ? ids[i] : 0;
+    const bool ok = valid && t >= 0 && t < vocab;
+    if (valid && !ok) set_status(st, PA_ERR_INVALID, (int)(i & 0x7fffffff), t);
+    const unsigned peers = __match_any_sync(0xffffffffu, ok ? t : -1);
+    if (ok && lane == __ffs(peers) - 1) atomicOr(&bm[t >> 5], 1u << (t & 31));
+  }
+  __syncthreads();
+  const unsigned long long bit = 1ull << j;
+  for (int w = threadIdx.x; w < words; w += blockDim.x) {
+    uint32_t x = bm[w];
+    while (x) {
+      const int t = (w << 5) + __ffs(x) - 1;
+      x &= x - 1u;
       if (!(ld_cg_u64(mask + t) & bit)) atomicOr(mask + t, bit);
     }
   }
@@ -208,6 +253,32 @@ __global__ void evenly_spaced_kernel(int32_t n_blocks, int32_t C, int32_t k, int
   }
 }
 
+// mask[t] = the set of blocks containing t (zeroed first)
+static int launch_presence(const SelectArgs& a, cudaStream_t s) {
+  if (cudaMemsetAsync(a.mask, 0, sizeof(unsigned long long) * (size_t)a.vocab, s) != cudaSuccess)
+    return PA_ERR_CUDA;
+  if (a.L <= 0) return PA_OK;
+  const int threads = 256;
+  const size_t bm_bytes = sizeof(uint32_t) * (size_t)((a.vocab + 31) / 32);
+  if (bm_bytes <= kPresenceSmemMax) {
+    int64_t tile = a.L / (4 * 148);
+    tile = tile < 512 ? 512 : (tile > 4096 ? 4096 : (tile + 255) / 256 * 256);
+    const int tiles_per_block = (int)((a.block + tile - 1) / tile);
+    const int64_t n_tiles = (int64_t)(a.L / a.block) * tiles_per_block;
+    if (bm_bytes > 48 * 1024 &&
+        cudaFuncSetAttribute(presence_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bm_bytes) !=
+            cudaSuccess)
+      return PA_ERR_CUDA;
+    presence_tile_kernel<<<(unsigned)n_tiles, threads, bm_bytes, s>>>(a.ids, a.L, a.vocab, a.block, (int)tile,
+                                                                     a.mask, a.status);
+  } else {
+    const int64_t want = (a.L + threads - 1) / threads;
+    presence_mask_kernel<<<(int)(want < 148 * 16 ? want : 148 * 16), threads, 0, s>>>(a.ids, a.L, a.vocab,
+                                                                                      a.block, a.mask, a.status);
+  }
+  return PA_OK;
+}
+
 int launch_select_scored(const SelectArgs& a, int method, const FixedIdf& tab, long long* score,
                          cudaStream_t s) {
   const int64_t n_chunks = a.L / a.chunk;
@@ -220,12 +291,9 @@ int launch_select_scored(const SelectArgs& a, int method, const FixedIdf& tab, l
     }
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
   }
-  if (cudaMemsetAsync(a.mask, 0, sizeof(unsigned long long) * (size_t)a.vocab, s) != cudaSuccess)
-    return PA_ERR_CUDA;
+  int rc = launch_presence(a, s);
+  if (rc) return rc;
   const int threads = 256;
-  const int64_t want = (a.L + threads - 1) / threads;
-  presence_mask_kernel<<<(int)(want < 148 * 16 ? want : 148 * 16), threads, 0, s>>>(
-      a.ids, a.L, a.vocab, a.block, a.mask, a.status);
   const int64_t wgrid = (n_chunks * 32 + threads - 1) / threads;
   chunk_fixed_score_kernel<<<(int)(wgrid < 148 * 32 ? wgrid : 148 * 32), threads, 0, s>>>(
       a.ids, n_chunks, a.chunk, a.vocab, a.mask, tab, score);
@@ -257,13 +325,10 @@ int launch_select(const SelectArgs& a, cudaStream_t s) {
   const int64_t n_chunks = a.L / a.chunk;
   const int C = a.block / a.chunk;
   const int n_blocks = (int)(a.L / a.block);
-  if (cudaMemsetAsync(a.mask, 0, sizeof(unsigned long long) * (size_t)a.vocab, s) != cudaSuccess)
-    return PA_ERR_CUDA;
+  int rc = launch_presence(a, s);
+  if (rc) return rc;
   if (a.L > 0) {
     const int threads = 256;
-    const int64_t want = (a.L + threads - 1) / threads;
-    const int grid = (int)(want < 148 * 16 ? want : 148 * 16);
-    presence_mask_kernel<<<grid, threads, 0, s>>>(a.ids, a.L, a.vocab, a.block, a.mask, a.status);
     const int64_t wwarps = n_chunks;
     const int64_t wgrid = (wwarps * 32 + threads - 1) / threads;
     chunk_mindf_kernel<<<(int)(wgrid < 148 * 32 ? wgrid : 148 * 32), threads, 0, s>>>(
