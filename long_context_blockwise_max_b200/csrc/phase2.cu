@@ -257,7 +257,10 @@ static void launch_merge_kernel(const Phase2Args& a, cudaStream_t s) {
 // Splits per shard so that small batches still fill the GPU.  Independent of
 // the dtype, so that the workspace size does not depend on it.
 //  - Few rows per kv head (decode, <= 8): work units are (batch, shard split,
-//    kv head); aim for 4 units per SM, with at least 512 keys per split.
+//    kv head), one CTA per SM; pick the split count w that minimises
+//    waves x (fixed cost + keys per split), waves = ceil(units x w / 148),
+//    the fixed cost of a unit taken as 140 keys' streaming, with at least 512
+//    keys per split.
 //  - Many rows: units are (batch, shard split, kv head, 256 query rows), one
 //    CTA per SM, keys in tiles of 128; pick the split count w that minimises
 //    waves x (fixed cost + tiles per split), waves = ceil(units x w / 148),
@@ -273,10 +276,17 @@ int32_t phase2_split(int32_t B, int32_t Tq, int64_t T, int32_t n_shards, int32_t
   if (cap < 1) cap = 1;
   if (R <= 8) {
     const int64_t base = (int64_t)B * n_shards * hkv;
-    int64_t want = base > 0 ? (4 * 148 + base - 1) / base : 1;
-    if (want > cap) want = cap;
-    if (want < 1) want = 1;
-    return (int32_t)want;
+    if (base <= 0) return 1;
+    int64_t best = 1, best_cost = 0;
+    for (int64_t w = 1; w <= cap; ++w) {
+      const int64_t waves = (base * w + 147) / 148;
+      const int64_t cost = waves * (140 + (shard_len + w - 1) / w);
+      if (w == 1 || cost < best_cost) {
+        best = w;
+        best_cost = cost;
+      }
+    }
+    return (int32_t)best;
   }
   const int64_t base = (int64_t)B * n_shards * hkv * ((R + 255) / 256);
   if (base <= 0) return 1;
