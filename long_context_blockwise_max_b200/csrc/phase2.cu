@@ -3,10 +3,16 @@
 // summary "Fase 2"; Star Attention review, key_machinery and the referee's
 // correction of Algorithm 2: O = sum_h exp(s_h - s_global) A_h).
 //
-// Work unit = (batch element, shard, split, kv head, tile of 128 query rows).
+// Work unit = (batch element, shard split, kv head) and a group of query rows.
 // A shard may be cut into `n_split` contiguous splits so that small batches
 // still fill the GPU; the merge is associative, so splits and shards merge
-// with the same algebra.
+// with the same algebra.  Kernels by case:
+//   bf16, >= 64 query rows per kv head   phase2_tc_kernel (phase2_tc.cu)
+//   bf16, <= 8 rows (decode)             phase2_mma_kernel (phase2_mma.cu)
+//   bf16, other row counts               phase2_mma_rows_kernel (phase2_mma.cu)
+//   fp32                                 phase2_simt_kernel (below)
+// followed by merge_kernel; this file also holds the query RoPE, the split
+// heuristic and the own-cache append of the query-host step.
 #include "pa_internal.h"
 
 namespace pa {
