@@ -41,6 +41,9 @@ METRIC = "Phase-1 encode tokens/s (%bf16 TC peak); Phase-2 query attn GB/s (%HBM
 WORKLOAD = workloads.LLAMA_128K
 DECODE = workloads.DECODE_128K
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# NVIDIA's nominal B200 figures, reported beside the measured denominators
+NOMINAL_BF16_TFLOPS = 2250.0   # dense
+NOMINAL_HBM_GBS = 8000.0
 
 
 def load_peaks():
@@ -410,6 +413,7 @@ def run_ours(args, rank, world, local_rank, dist_on):
             "gb_s": round(kv_bytes / (dec_ms * 1e-3) / 1e9, 1),
             "kernel_gb_s": round(kv_bytes / (dec_kernel_ms * 1e-3) / 1e9, 1),
             "frac_hbm": round(kv_bytes / (dec_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+            "frac_of_nominal_hbm": round(kv_bytes / (dec_ms * 1e-3) / 1e9 / NOMINAL_HBM_GBS, 4),
             "bytes_per_call": kv_bytes}
         # ART early termination on the same decode (the page's defaults)
         ao = torch.empty_like(dq)
@@ -614,7 +618,9 @@ def run_ours(args, rank, world, local_rank, dist_on):
                      "peak": peak_tf, "unit": "TFLOP/s", "frac": round(attn_tf / peak_tf, 4),
                      "peak_kind": f"{peak_kind} bf16 sustained",
                      "traffic": recorded_traffic("phase1_tc_kernel", w.name),
-                     "kernel_ms": round(attn_ms, 3), "flop_per_launch": flops},
+                     "kernel_ms": round(attn_ms, 3), "flop_per_launch": flops,
+                     "frac_of_nominal_dense_bf16": round(attn_tf / NOMINAL_BF16_TFLOPS, 4),
+                     "frac_of_burst": round(attn_tf / peaks["bf16_tflops"], 4)},
         "phase1_encode": {"selection_ms": round(sel_ms, 4), "encode_ms": round(enc_ms, 3),
                           "tokens_per_s": round(w.L / (enc_ms * 1e-3), 1),
                           "with_selection_tokens_per_s": round(w.L / ((sel_ms + enc_ms) * 1e-3), 1),
