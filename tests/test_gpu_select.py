@@ -44,6 +44,9 @@ CASES = [
     (1024, 64, 256, 1, 17, 0.8),            # one-token chunks
     (24 * 1000, 300, 1000, 40, 7, 1.3),     # blocks not a multiple of 32
     (8 * 32768, 2000, 32768, 32, 512, 1.1), # 1024 chunks per block, several tiles of the compaction
+    (4 * 8192, 1 << 20, 8192, 32, 16, 1.1), # vocabulary of 2^20 ids: the largest shared-memory bitmap
+    (4 * 1024, 1500000, 1024, 32, 4, 1.1),  # vocabulary above 2^20 ids: the per-warp dedupe kernel
+    (7 * 640, 500, 640, 32, 3, 0.3),        # tiles end at block ends inside the per-tile kernel
 ]
 
 
