@@ -41,7 +41,11 @@ Parity pins (tests/test_oracle_*.py): brute-force top-k and a Figure-2
 analogue (selection); N = 1 reduces to library causal attention, full-budget
 / zero-sink hosts equal dense causal attention rows, the uniform-score closed
 form lse = ln(r+1), and complex-multiplication RoPE (Phase 1); the shard merge
-equals library dense attention over the concatenated cache (Phase 2).
+equals library dense attention over the concatenated cache (Phase 2).  Added
+rows: mean-IDF against hand-worked Figure-2 means and brute force, evenly
+spaced chunks against their closed form; the query-host step against masked
+library attention; ART with zero thresholds against library attention and
+its stop block against a closed form where the weights underflow.
 """
 from __future__ import annotations
 
