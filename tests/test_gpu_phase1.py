@@ -118,6 +118,30 @@ def test_bf16_zero_sink_zero_budget(P):
     _parity(P, q, k, v, 10000.0, block, 0, 32, 0, sel, False)
 
 
+@pytest.mark.parametrize("star", [False, True])
+def test_bf16_running_max_jumps_mid_sequence(P, star):
+    # Rows at positions >= 128 with p = 1 (mod 4), and rows at positions >= 256
+    # with p = 3 (mod 4), score the keys before that point about 7 nat lower
+    # through sixteen of the slowest-turning RoPE dimensions.  Their running
+    # max therefore jumps by more than 2^8 at key tile 1 or 2, which takes the
+    # lazy-rescale branch (half a tile recomputed, O rescaled) for some rows of
+    # every warp while the others keep their max.  The jump comes from pushing
+    # early keys down, so the dominant scores stay small and the fp16 operand
+    # rounding stays well inside the lse tolerance.
+    L, block, theta, a = 2 * 512, 512, 500000.0, 5.0
+    q, k, v = _inputs(L, 4, 2, 128, torch.bfloat16, seed=77)
+    pos = np.arange(L)
+    rng = np.random.default_rng(5)
+    for dims, start, rem in ((np.r_[48:56, 112:120], 128, 1), (np.r_[56:64, 120:128], 256, 3)):
+        idx = torch.from_numpy(dims)
+        kx = (pos < start)[:, None, None] * -a * (1.0 + 0.25 * rng.standard_normal((L, 2, 16)))
+        qx = ((pos % 4 == rem) & (pos >= start))[:, None, None] * (1.0 + 0.25 * rng.standard_normal((L, 4, 16)))
+        k[:, :, idx] = torch.from_numpy(kx).to(torch.bfloat16)
+        q[:, :, idx] = torch.from_numpy(qx).to(torch.bfloat16)
+    sel = np.array([[1, 9], [3, 14]])
+    _parity(P, q, k, v, theta, block, 64, 32, 2, sel, star)
+
+
 @pytest.mark.parametrize("wname", ["llama3.1-8b_attn_32k", "llama3.1-8b_attn_128k"])
 @pytest.mark.parametrize("star", [False, True])
 def test_llama_shapes_sampled_rows(P, wname, star):

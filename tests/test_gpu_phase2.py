@@ -78,6 +78,34 @@ def test_bf16_small_full(P, case):
     assert_close(pl.cpu().double().numpy(), rs, LSE_TOL, "s_h")
 
 
+def test_query_kernel_running_max_jumps(P):
+    # A 64-token query with g = 4 (256 rows per kv head: the tensor-core
+    # kernel) over two 512-key shards, one unit each.  For the odd query heads
+    # the first 128 keys of each shard score about 7 nat lower, so those rows'
+    # running max jumps by more than 2^8 at the unit's second key tile (the
+    # lazy-rescale branch), while the even heads' rows, in the same warps, keep
+    # theirs.  No RoPE, so the shifted dimensions stay as written.
+    B, Tq, T, S, hq, hkv, d = 1, 64, 1024, 2, 8, 2, 128
+    q = workloads.normal((B, Tq, hq, d), 63, torch.bfloat16)
+    kc = workloads.normal((B, T, hkv, d), 64, torch.bfloat16)
+    vc = workloads.normal((B, T, hkv, d), 65, torch.bfloat16)
+    rng = np.random.default_rng(6)
+    idx = torch.arange(96, 128)
+    t = np.arange(T)
+    kx = ((t % 512) < 128)[None, :, None, None] * -2.5 * (1.0 + 0.25 * rng.standard_normal((B, T, hkv, 32)))
+    qx = (np.arange(hq) % 2 == 1)[None, None, :, None] * (1.0 + 0.25 * rng.standard_normal((B, Tq, hq, 32)))
+    kc[..., idx] = torch.from_numpy(kx).to(torch.bfloat16)
+    q[..., idx] = torch.from_numpy(qx).to(torch.bfloat16)
+    o, lse, po, pl, ws = P.star_phase2_attend(q.to(DEV), kc.to(DEV), vc.to(DEV), S, q_pos0=T, rope_theta=0.0,
+                                              want_partials=True)
+    assert P.pa_workspace_status(ws) == 0
+    ro, rl, ra, rs = oracle.phase2_attend(f64(q), f64(kc), f64(vc), S, T, 0.0)
+    assert_close(f64(o.cpu()), ro, O_TOL[torch.bfloat16], "O")
+    assert_close(lse.cpu().double().numpy(), rl, LSE_TOL, "lse")
+    assert_close(po.cpu().double().numpy(), ra, O_TOL[torch.bfloat16], "A_h")
+    assert_close(pl.cpu().double().numpy(), rs, LSE_TOL, "s_h")
+
+
 @pytest.mark.parametrize("wname,groups", [
     ("decode_128k_b16", [(0, 0), (9, 5), (15, 7)]),
     ("scale_1m", [(0, 3), (3, 7)]),
