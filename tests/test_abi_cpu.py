@@ -94,3 +94,54 @@ def test_host_validation_rejects_before_launch(lib):
     # phase 2: zero shards
     assert so.star_phase2_attend(dummy, 1, 1, 1, 0, 0.0, dummy, dummy, 100, 0, 32, 8, 128, dummy, dummy, None,
                                  None, ws, 1 << 30, None) == -1
+
+
+def test_host_validation_of_the_other_entry_points(lib):
+    # argument checks of the scorer, ART, merge and query-step entry points
+    # and the status text, all decided on the host before any launch
+    so = lib._lib
+    ws = ctypes.c_void_p(256)
+    dummy = ctypes.c_void_p(4096)
+    texts = {c: so.pa_status_string(c).decode() for c in range(-6, 1)}
+    assert len(set(texts.values())) == 7 and all(texts.values())
+    assert so.pa_status_string(-99).decode() == "unknown status"
+    assert so.pa_abi_version() >= 1
+    assert so.pa_set_profile_events(dummy, None) == -1
+    assert so.pa_set_profile_events(None, dummy) == -1
+    assert so.pa_set_profile_events(None, None) == 0
+    # scorer: unknown method; missing ids for a scorer that reads them; mean-IDF beyond 8192 chunks per block
+    assert so.pulsar_select_summaries_scored(dummy, 1024, 100, 512, 32, 2, 3, dummy, None, ws, 1 << 20,
+                                             None) == -1
+    assert so.pulsar_select_summaries_scored(None, 1024, 100, 512, 32, 2, 1, dummy, None, ws, 1 << 20,
+                                             None) == -1
+    assert so.pulsar_select_summaries_scored(dummy, 16384, 100, 16384, 1, 1, 1, dummy, None, ws, 1 << 30,
+                                             None) == -2
+
+    def art(dtype=1, Tq=1, hq=32, hkv=8, block_keys=128, tau=1e-5, phi=1e-3, patience=5, theta=5e5):
+        return so.star_phase2_attend_art(dummy, dtype, 2, Tq, 1000, theta, dummy, dummy, 1000, hq, hkv, 128,
+                                         block_keys, tau, phi, patience, dummy, dummy, None, ws, 1 << 30, None)
+    assert art(dtype=0) == -2                      # bf16 only
+    assert art(block_keys=48) == -1                # a multiple of 32
+    assert art(block_keys=0) == -1
+    assert art(patience=0) == -1
+    assert art(tau=float("nan")) == -1
+    assert art(phi=-1.0) == -1
+    assert art(theta=float("inf")) == -1
+    assert art(Tq=3) == -2                         # 3 tokens x 4 heads = 12 decode rows > 8
+
+    def merge(S=4, d=128, dtype=1, part_o=dummy):
+        return so.pa_lse_merge(part_o, dummy, 1, S, 2, 8, d, dtype, dummy, dummy, None)
+    assert merge(S=0) == -1
+    assert merge(d=96) == -2
+    assert merge(dtype=5) == -2
+    assert merge(part_o=ctypes.c_void_p(4100)) == -1   # partials must be 16-byte aligned
+
+    def step(n_shards=8, self_cap=64, self_len=0, Tq=4, theta=5e5):
+        return so.star_phase2_query_step(dummy, dummy, dummy, 1, 1, Tq, 1000, theta, dummy, dummy, 1000,
+                                         n_shards, dummy, dummy, self_cap, self_len, 32, 8, 128, dummy, dummy,
+                                         ws, 1 << 30, None)
+    assert step(n_shards=0) == -1
+    assert step(n_shards=4097) == -1
+    assert step(self_len=62) == -1                 # 62 + 4 new tokens > capacity 64
+    assert step(self_len=-1) == -1
+    assert step(theta=float("nan")) == -1
