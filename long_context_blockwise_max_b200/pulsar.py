@@ -118,6 +118,26 @@ def _dev(*ts):
                 raise ValueError("tensors must be contiguous")
 
 
+def _need(t, name: str, dtype, numel: int):
+    """A caller-supplied tensor (None: skipped) must have ``dtype`` and at
+    least ``numel`` elements: the library reads or writes that many through
+    the raw pointer, so a smaller or differently typed buffer is refused
+    here rather than overrun on the device."""
+    if t is None:
+        return
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if t.numel() < numel:
+        raise ValueError(f"{name}: {t.numel()} elements, at least {numel} needed")
+
+
+def _same(ref, *named):
+    """Tensors that must match ``ref`` in dtype and shape (K and V of one cache)."""
+    for name, t in named:
+        if t is not None and (t.dtype != ref.dtype or t.shape != ref.shape):
+            raise ValueError(f"{name}: {t.dtype} {tuple(t.shape)}, expected {ref.dtype} {tuple(ref.shape)}")
+
+
 def _workspace(nbytes: int, device, ws=None):
     if ws is not None:
         return ws
@@ -152,16 +172,20 @@ def pulsar_select_summaries(ids: torch.Tensor, vocab: int, block: int, chunk: in
                             sel=None, df=None, chunk_mindf=None, ws=None, want_df=False,
                             want_mindf=False):
     """Max-IDF summary selection. Returns (sel [N][k] int32, df or None, mindf or None, ws)."""
-    _dev(ids)
+    _dev(ids, sel, df, chunk_mindf)
     L = ids.numel()
     n = L // block if block > 0 else 0
+    _need(ids, "ids", torch.int32, L)
+    _need(sel, "sel", torch.int32, n * k_chunks)
+    _need(df, "df", torch.int32, vocab)
+    _need(chunk_mindf, "chunk_mindf", torch.int32, L // chunk if chunk > 0 else 0)
     dev = ids.device
     if sel is None:
         sel = torch.empty((n, k_chunks), dtype=torch.int32, device=dev)
     if want_df and df is None:
         df = torch.empty(vocab, dtype=torch.int32, device=dev)
     if want_mindf and chunk_mindf is None:
-        chunk_mindf = torch.empty(L // chunk, dtype=torch.int32, device=dev)
+        chunk_mindf = torch.empty(L // chunk if chunk > 0 else 0, dtype=torch.int32, device=dev)
     need = pa_select_workspace_size(L, vocab, block, chunk)
     ws = _workspace(need, dev, ws)
     rc = _lib.pulsar_select_summaries(_ptr(ids), L, vocab, block, chunk, k_chunks, _ptr(sel),
@@ -176,6 +200,11 @@ def pulsar_select_summaries_noalloc(ids: torch.Tensor, vocab: int, block: int, c
     memory: writes into the caller's preallocated ``sel`` (and optional
     ``df`` / ``chunk_mindf``) and allocates nothing.  Returns ``sel``."""
     _dev(ids, sel, df, chunk_mindf)
+    L = ids.numel()
+    _need(ids, "ids", torch.int32, L)
+    _need(sel, "sel", torch.int32, (L // block if block > 0 else 0) * k_chunks)
+    _need(df, "df", torch.int32, vocab)
+    _need(chunk_mindf, "chunk_mindf", torch.int32, L // chunk if chunk > 0 else 0)
     rc = _lib.pulsar_select_summaries_noalloc(_ptr(ids), ids.numel(), vocab, block, chunk, k_chunks, _ptr(sel),
                                               _ptr(df), _ptr(chunk_mindf), _stream())
     _check(rc, "pulsar_select_summaries_noalloc")
@@ -190,9 +219,11 @@ def pulsar_select_summaries_scored(ids, vocab: int, block: int, chunk: int, k_ch
     L = ids.numel() if ids is not None else int(L)
     dev = ids.device if ids is not None else torch.device("cuda", torch.cuda.current_device())
     n = L // block if block > 0 else 0
+    _need(ids, "ids", torch.int32, L)
+    _need(sel, "sel", torch.int32, n * k_chunks)
     if sel is None:
         sel = torch.empty((n, k_chunks), dtype=torch.int32, device=dev)
-    scores = torch.empty(L // chunk, dtype=torch.int64, device=dev) if want_scores else None
+    scores = torch.empty(L // chunk if chunk > 0 else 0, dtype=torch.int64, device=dev) if want_scores else None
     ws = _workspace(pa_select_workspace_size(L, vocab, block, chunk), dev, ws)
     rc = _lib.pulsar_select_summaries_scored(_ptr(ids), L, vocab, block, chunk, k_chunks, int(method), _ptr(sel),
                                              _ptr(scores), _ptr(ws), ws.numel() * ws.element_size(), _stream())
@@ -210,6 +241,23 @@ def pa_phase1_layout(L, block, sink, summary_tokens, star) -> list[int]:
 
 def pa_phase1_workspace_size(L, hq, hkv, d, dtype, block, sink, summary_tokens, star) -> int:
     return _lib.pa_phase1_workspace_size(L, hq, hkv, d, dtype, block, sink, summary_tokens, int(star))
+
+
+def _phase1_check(q, k, v, rows, ret_rows, o, lse, k_ret, v_ret, sel=None, n_sel=0):
+    """Inputs [L][h][d] of one dtype (K and V alike); caller-supplied outputs
+    large enough for ``rows`` output rows and ``ret_rows`` retained rows."""
+    if q.dim() != 3 or k.dim() != 3:
+        raise ValueError("q, k, v must be [L][heads][d]")
+    L, hq, d = q.shape
+    hkv = k.shape[1]
+    if k.shape[0] != L or k.shape[2] != d or k.dtype != q.dtype:
+        raise ValueError(f"k: {k.dtype} {tuple(k.shape)} does not match q {q.dtype} {tuple(q.shape)}")
+    _same(k, ("v", v))
+    _need(sel, "sel", torch.int32, n_sel)
+    _need(o, "o", q.dtype, rows * hq * d)
+    _need(lse, "lse", torch.float32, rows * hq)
+    _need(k_ret, "k_ret", q.dtype, ret_rows * hkv * d)
+    _need(v_ret, "v_ret", q.dtype, ret_rows * hkv * d)
 
 
 def _phase1_outputs(q, k, rows, o, lse, k_ret, v_ret, want_lse):
@@ -234,6 +282,7 @@ def pulsar_phase1_encode(q, k, v, rope_theta, block, sink, chunk, k_chunks, sel,
     hkv = k.shape[1]
     dt = _dtype_code(q)
     row_off = pa_phase1_layout(L, block, sink, k_chunks * chunk, False)
+    _phase1_check(q, k, v, row_off[-1], L, o, lse, k_ret, v_ret, sel, (L // block if block > 0 else 0) * k_chunks)
     o, lse, k_ret, v_ret = _phase1_outputs(q, k, row_off[-1], o, lse, k_ret, v_ret, want_lse)
     need = pa_phase1_workspace_size(L, hq, hkv, d, dt, block, sink, k_chunks * chunk, False)
     ws = _workspace(need, q.device, ws)
@@ -252,6 +301,7 @@ def star_phase1_encode(q, k, v, rope_theta, block, o=None, lse=None, k_ret=None,
     hkv = k.shape[1]
     dt = _dtype_code(q)
     row_off = pa_phase1_layout(L, block, 0, 0, True)
+    _phase1_check(q, k, v, row_off[-1], L, o, lse, k_ret, v_ret)
     o, lse, k_ret, v_ret = _phase1_outputs(q, k, row_off[-1], o, lse, k_ret, v_ret, want_lse)
     need = pa_phase1_workspace_size(L, hq, hkv, d, dt, block, 0, 0, True)
     ws = _workspace(need, q.device, ws)
@@ -289,6 +339,8 @@ def pulsar_phase1_encode_hosts(q, k, v, rope_theta, block, sink, chunk, k_chunks
     full = pa_phase1_layout(L, block, sink, k_chunks * chunk, False)
     row_off = [r - full[host_begin] for r in full[host_begin:host_end + 1]]
     nh = max(host_end - host_begin, 0)
+    _phase1_check(q, k, v, row_off[-1] if row_off else 0, nh * block, o, lse, k_ret, v_ret, sel,
+                  (L // block if block > 0 else 0) * k_chunks)
     o, lse, k_ret, v_ret = _phase1_range_outputs(q, k, block, row_off[-1] if row_off else 0, nh, o, lse, k_ret,
                                                  v_ret, want_lse)
     need = pa_phase1_workspace_size(L, hq, hkv, d, dt, block, sink, k_chunks * chunk, False)
@@ -311,6 +363,7 @@ def star_phase1_encode_hosts(q, k, v, rope_theta, block, host_begin, host_end, o
     full = pa_phase1_layout(L, block, 0, 0, True)
     row_off = [r - full[host_begin] for r in full[host_begin:host_end + 1]]
     nh = max(host_end - host_begin, 0)
+    _phase1_check(q, k, v, row_off[-1] if row_off else 0, nh * block, o, lse, k_ret, v_ret)
     o, lse, k_ret, v_ret = _phase1_range_outputs(q, k, block, row_off[-1] if row_off else 0, nh, o, lse, k_ret,
                                                  v_ret, want_lse)
     need = pa_phase1_workspace_size(L, hq, hkv, d, dt, block, 0, 0, True)
@@ -322,6 +375,19 @@ def star_phase1_encode_hosts(q, k, v, rope_theta, block, host_begin, host_end, o
     return o, lse, k_ret, v_ret, row_off, ws
 
 
+def _phase2_check(q, k_ret, v_ret, o, lse):
+    """q [B][Tq][hq][d]; caches [B][T][hkv][d] in q's dtype (K and V alike);
+    caller-supplied o / lse large enough."""
+    if q.dim() != 4 or k_ret.dim() != 4:
+        raise ValueError("q must be [B][Tq][hq][d] and the caches [B][T][hkv][d]")
+    B, Tq, hq, d = q.shape
+    if k_ret.shape[0] != B or k_ret.shape[3] != d or k_ret.dtype != q.dtype:
+        raise ValueError(f"k_ret: {k_ret.dtype} {tuple(k_ret.shape)} does not match q {q.dtype} {tuple(q.shape)}")
+    _same(k_ret, ("v_ret", v_ret))
+    _need(o, "o", q.dtype, B * Tq * hq * d)
+    _need(lse, "lse", torch.float32, B * Tq * hq)
+
+
 def pa_phase2_workspace_size(B, Tq, T, n_shards, hq, hkv, d) -> int:
     return _lib.pa_phase2_workspace_size(B, Tq, T, n_shards, hq, hkv, d)
 
@@ -331,8 +397,11 @@ def star_phase2_attend(q, k_ret, v_ret, n_shards, q_pos0=0, rope_theta=0.0, o=No
     """Phase-2 split-KV attention + exact merge. q [B][Tq][hq][d]; caches [B][T][hkv][d].
     Returns (o, lse, part_o, part_lse, ws)."""
     _dev(q, k_ret, v_ret, o, lse, part_o, part_lse)
+    _phase2_check(q, k_ret, v_ret, o, lse)
     B, Tq, hq, d = q.shape
     T, hkv = k_ret.shape[1], k_ret.shape[2]
+    _need(part_o, "part_o", torch.float32, B * n_shards * Tq * hq * d)
+    _need(part_lse, "part_lse", torch.float32, B * n_shards * Tq * hq)
     dt = _dtype_code(q)
     if o is None:
         o = torch.empty_like(q)
@@ -357,6 +426,7 @@ def star_phase2_attend_art(q, k_ret, v_ret, q_pos0=0, rope_theta=0.0, block_keys
     """Phase 2 with run-time early termination of the key walk (newest keys
     first).  bf16; Tq * hq / hkv <= 8.  Returns (o, lse, visited_blocks [B][hkv], ws)."""
     _dev(q, k_ret, v_ret, o, lse)
+    _phase2_check(q, k_ret, v_ret, o, lse)
     B, Tq, hq, d = q.shape
     T, hkv = k_ret.shape[1], k_ret.shape[2]
     if o is None:
@@ -377,7 +447,13 @@ def pa_lse_merge(part_o, part_lse, dtype=torch.bfloat16, o=None, lse=None):
     """Exact merge of partials part_o [B][S][Tq][hq][d], part_lse [B][S][Tq][hq]
     (float32, on the GPU).  Returns (o in ``dtype``, lse)."""
     _dev(part_o, part_lse, o, lse)
+    if part_o.dim() != 5:
+        raise ValueError("part_o must be [B][S][Tq][hq][d]")
     B, S, Tq, hq, d = part_o.shape
+    _need(part_o, "part_o", torch.float32, B * S * Tq * hq * d)
+    _need(part_lse, "part_lse", torch.float32, B * S * Tq * hq)
+    _need(o, "o", o.dtype if o is not None else dtype, B * Tq * hq * d)
+    _need(lse, "lse", torch.float32, B * Tq * hq)
     if o is None:
         o = torch.empty((B, Tq, hq, d), dtype=dtype, device=part_o.device)
     if lse is None:
@@ -395,8 +471,14 @@ def star_phase2_query_step(q, k_new, v_new, k_ret, v_ret, n_shards, k_self, v_se
     0..self_len + j, causal).  q/k_new/v_new [B][Tq][h][d]; caches
     [B][T][hkv][d]; k_self/v_self [B][cap][hkv][d].  Returns (o, lse, ws)."""
     _dev(q, k_new, v_new, k_ret, v_ret, k_self, v_self, o, lse)
+    _phase2_check(q, k_ret, v_ret, o, lse)
+    _phase2_check(q, k_self, v_self, None, None)
     B, Tq, hq, d = q.shape
     T, hkv = k_ret.shape[1], k_ret.shape[2]
+    if k_self.shape[2] != hkv:
+        raise ValueError(f"k_self: {k_self.shape[2]} kv heads, the shards have {hkv}")
+    _need(k_new, "k_new", q.dtype, B * Tq * hkv * d)
+    _same(k_new, ("v_new", v_new))
     if o is None:
         o = torch.empty_like(q)
     if lse is None:

@@ -6,6 +6,7 @@ import os
 import re
 
 import numpy as np
+import torch
 import pytest
 
 import oracle
@@ -145,3 +146,54 @@ def test_host_validation_of_the_other_entry_points(lib):
     assert step(self_len=62) == -1                 # 62 + 4 new tokens > capacity 64
     assert step(self_len=-1) == -1
     assert step(theta=float("nan")) == -1
+
+
+def test_binding_refuses_mismatched_tensors_before_the_library(lib, monkeypatch):
+    # the binding hands raw pointers to the library, so it checks dtypes and
+    # sizes first; these calls must all stop there (CPU tensors, with the
+    # CUDA-residency check stubbed out, never reach a launch)
+    P = lib
+    monkeypatch.setattr(P, "_dev", lambda *ts: None)
+    bf, f32, i32 = torch.bfloat16, torch.float32, torch.int32
+    L, hq, hkv, d, block = 1024, 8, 2, 64, 256
+    q = torch.zeros((L, hq, d), dtype=bf)
+    k = torch.zeros((L, hkv, d), dtype=bf)
+    sel = torch.zeros((4, 2), dtype=i32)
+    with pytest.raises(ValueError, match="ids"):
+        P.pulsar_select_summaries(torch.zeros(L, dtype=torch.int64), 100, block, 32, 2)
+    with pytest.raises(ValueError, match="sel"):
+        P.pulsar_select_summaries(torch.zeros(L, dtype=i32), 100, block, 32, 2, sel=torch.zeros((4, 1), dtype=i32))
+    with pytest.raises(ValueError, match="df"):
+        P.pulsar_select_summaries_noalloc(torch.zeros(L, dtype=i32), 100, block, 32, 2, sel,
+                                          df=torch.zeros(99, dtype=i32))
+    with pytest.raises(ValueError, match="k:"):
+        P.pulsar_phase1_encode(q, k.float(), k, 1e4, block, 64, 32, 2, sel)
+    with pytest.raises(ValueError, match="v:"):
+        P.pulsar_phase1_encode(q, k, torch.zeros((L, hkv, d + 64), dtype=bf), 1e4, block, 64, 32, 2, sel)
+    with pytest.raises(ValueError, match="sel"):
+        P.pulsar_phase1_encode(q, k, k, 1e4, block, 64, 32, 2, sel.long())
+    with pytest.raises(ValueError, match="o:"):
+        P.star_phase1_encode(q, k, k, 1e4, block, o=torch.zeros((10, hq, d), dtype=bf))
+    with pytest.raises(ValueError, match="lse"):
+        P.star_phase1_encode(q, k, k, 1e4, block, lse=torch.zeros((L, hq), dtype=bf))
+    with pytest.raises(ValueError, match="k_ret"):
+        P.star_phase1_encode_hosts(q, k, k, 1e4, block, 0, 2, k_ret=torch.zeros((block, hkv, d), dtype=bf))
+    qq = torch.zeros((2, 3, hq, d), dtype=bf)
+    kc = torch.zeros((2, 500, hkv, d), dtype=bf)
+    with pytest.raises(ValueError, match="k_ret"):
+        P.star_phase2_attend(qq, kc.float(), kc.float(), 4)
+    with pytest.raises(ValueError, match="v_ret"):
+        P.star_phase2_attend(qq, kc, kc[:, :400].contiguous(), 4)
+    with pytest.raises(ValueError, match="part_o"):
+        P.star_phase2_attend(qq, kc, kc, 4, want_partials=True, part_o=torch.zeros((2, 3, 3, hq, d), dtype=f32))
+    with pytest.raises(ValueError, match="o:"):
+        P.star_phase2_attend_art(qq, kc, kc, o=torch.zeros_like(qq, dtype=f32))
+    with pytest.raises(ValueError, match="part_lse"):
+        P.pa_lse_merge(torch.zeros((2, 4, 3, hq, d)), torch.zeros((2, 4, 3, hq), dtype=bf))
+    ks = torch.zeros((2, 16, hkv, d), dtype=bf)
+    kn = torch.zeros((2, 3, hkv, d), dtype=bf)
+    with pytest.raises(ValueError, match="v_new"):
+        P.star_phase2_query_step(qq, kn, kn[:, :2].contiguous(), kc, kc, 4, ks, ks, 0, 500, 5e5)
+    with pytest.raises(ValueError, match="k_self"):
+        P.star_phase2_query_step(qq, kn, kn, kc, kc, 4, torch.zeros((2, 16, 1, d), dtype=bf),
+                                 torch.zeros((2, 16, 1, d), dtype=bf), 0, 500, 5e5)
