@@ -34,7 +34,7 @@ def _worker(rank, world, port, out):
 
 def test_max_over_ranks_and_weak_scaling_rate():
     world, port = 2, _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
         res = dict(out)

@@ -62,7 +62,7 @@ def _worker(rank, world, port, n_shards, out):
 def _run(n_shards):
     import oracle
     world, port = 2, _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.spawn(_worker, args=(world, port, n_shards, out), nprocs=world, join=True)
         res = dict(out)
@@ -136,7 +136,7 @@ def _pipeline_worker(rank, world, port, star, out):
 def _pipeline(world, star):
     import oracle
     port = _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.spawn(_pipeline_worker, args=(world, port, star, out), nprocs=world, join=True)
         res = [out[r] for r in range(world)]
