@@ -1,17 +1,23 @@
-"""A randomized model of the synchronisation of phase1_tc_kernel (csrc/phase1_tc.cu),
-checked on the CPU for the failures that would hang or corrupt the GPU kernel:
+"""A randomized model of the synchronisation of the two tcgen05 attention
+kernels, phase1_tc_kernel (csrc/phase1_tc.cu) and phase2_tc_kernel
+(csrc/phase2_tc.cu), checked on the CPU for the failures that would hang or
+corrupt the GPU kernel:
 a waiter that misses an mbarrier phase (the hardware parity wait would then
 spin until its time limit), a deadlock, or an MMA / TMA copy / softmax step
 that touches data out of order.
 
-The model follows the kernel's roles and barriers one to one:
-  producer   Q once (q_full), then K(j) and V(j) into stage j & 1 after the
-             stage's *_empty barrier (2-stage ring);
+The model follows the kernels' roles and barriers one to one:
+  producer   Q once (q_full), then K(j) into stage j % KST and V(j) into stage
+             j % VST after the stage's *_empty barrier (Phase 1: 2 and 2
+             stages; Phase 2: 3 and 2 at d = 128, 4 and 4 at d = 64);
+  converter  (Phase 2 only) after K(j) lands, convert the stage to fp16 in
+             place and arrive k_conv; the issuer's QK^T waits for that;
   issuer     QK_t(0) for both heads; per key tile j: wait P0(j) (p_full0) and
              V(j) (v_full), PV0(j), wait K(j+1), QK0(j+1); wait P1(j), PV1(j),
              release V(j), QK1(j+1), release K(j+1); MMAs run in issue order on
              one pipe and a commit arrives once every earlier MMA has finished;
-  softmax t  wait S_t(j) (s_full_t), read S, write P over S, arrive p_full_t.
+  softmax t  wait S_t(j) (s_full_t), read S, write P over S, arrive p_full_t
+             (t is the head in Phase 1 and the 128-row tile in Phase 2).
 mbarriers keep an arrival count and a transaction count per phase; a parity
 wait for phase k succeeds when the completed-phase count has the other parity
 than k, exactly as mbarrier.try_wait.parity.  Copy latencies, MMA durations
@@ -54,19 +60,28 @@ class Bar:
 
 
 class Model:
-    def __init__(self, seed, nkv, mutation=None):
+    def __init__(self, seed, nkv, mutation=None, kst=2, vst=2, convert=False):
         self.rng = random.Random(seed)
         self.nkv, self.mutation = nkv, mutation
+        self.kst, self.vst, self.convert = kst, vst, convert
         self.t, self.events, self.pipe_free = 0, [], 0
         self.bars = {"q_full": Bar("q_full", 1)}
-        for s in (0, 1):
-            for name in ("k_full", "k_empty", "v_full", "v_empty", "s_full", "o_final"):
+        for s in range(kst):
+            for name in ("k_full", "k_empty"):
                 self.bars[f"{name}{s}"] = Bar(f"{name}{s}", 1)
-            self.bars[f"p_full{s}"] = Bar(f"p_full{s}", 128)
-        self.k_stage = [None, None]     # key tile held (landed) by each K stage
-        self.v_stage = [None, None]
-        self.k_readers = [0, 0]         # MMA groups in flight reading a stage
-        self.v_readers = [0, 0]
+            self.bars[f"k_conv{s}"] = Bar(f"k_conv{s}", 64)
+        for s in range(vst):
+            for name in ("v_full", "v_empty"):
+                self.bars[f"{name}{s}"] = Bar(f"{name}{s}", 1)
+        for t in (0, 1):
+            for name in ("s_full", "o_final"):
+                self.bars[f"{name}{t}"] = Bar(f"{name}{t}", 1)
+            self.bars[f"p_full{t}"] = Bar(f"p_full{t}", 128)
+        self.k_stage = [None] * kst     # key tile held (landed) by each K stage
+        self.k_ready = [None] * kst     # key tile whose stage is ready for QK^T (converted in Phase 2)
+        self.v_stage = [None] * vst
+        self.k_readers = [0] * kst      # MMA groups in flight reading a stage
+        self.v_readers = [0] * vst
         self.S = [None, None]           # TMEM S_t / P_t: ("S", j) or ("P", j)
         self.s_users = [0, 0]           # MMA groups in flight using S_t / P_t
         self.o_users = [0, 0]           # PV groups in flight accumulating into O_t
@@ -77,8 +92,12 @@ class Model:
     def copy(self, stage_list, st, j, bar):
         def land():
             stage_list[st] = j
+            if stage_list is self.k_stage and not self.convert:
+                self.k_ready[st] = j
             self.bars[bar].complete_tx(1)
         stage_list[st] = None
+        if stage_list is self.k_stage:
+            self.k_ready[st] = None
         self.bars[bar].arrive(expect_tx=1)
         self.at(self.t + self.rng.randint(1, 600), land)
 
@@ -97,20 +116,32 @@ class Model:
         b["q_full"].arrive(expect_tx=1)
         self.at(self.t + self.rng.randint(1, 100), lambda: b["q_full"].complete_tx(1))
         for j in range(self.nkv):
-            st = j & 1
-            if j >= 2:
-                yield (f"k_empty{st}", (j >> 1) - 1)
-            assert self.k_readers[st] == 0, f"K stage {st} refilled while an MMA reads it (tile {j})"
-            self.copy(self.k_stage, st, j, f"k_full{st}")
-            if j >= 2 and self.mutation != "v_no_empty_wait":
-                yield (f"v_empty{st}", (j >> 1) - 1)
-            assert self.v_readers[st] == 0, f"V stage {st} refilled while an MMA reads it (tile {j})"
-            self.copy(self.v_stage, st, j, f"v_full{st}")
+            sk, sv = j % self.kst, j % self.vst
+            if j >= self.kst:
+                yield (f"k_empty{sk}", j // self.kst - 1)
+            assert self.k_readers[sk] == 0, f"K stage {sk} refilled while an MMA reads it (tile {j})"
+            self.copy(self.k_stage, sk, j, f"k_full{sk}")
+            if j >= self.vst and self.mutation != "v_no_empty_wait":
+                yield (f"v_empty{sv}", j // self.vst - 1)
+            assert self.v_readers[sv] == 0, f"V stage {sv} refilled while an MMA reads it (tile {j})"
+            self.copy(self.v_stage, sv, j, f"v_full{sv}")
+
+    def converter(self):
+        for j in range(self.nkv):
+            sk = j % self.kst
+            if self.mutation != "convert_before_landing":
+                yield (f"k_full{sk}", j // self.kst)
+            assert self.k_stage[sk] == j, f"converter({j}) converts stage {sk} holding {self.k_stage[sk]}"
+            assert self.k_readers[sk] == 0, f"converter({j}) rewrites stage {sk} while an MMA reads it"
+            yield ("sleep", self.rng.randint(1, 200))
+            assert self.k_stage[sk] == j and self.k_readers[sk] == 0
+            self.k_ready[sk] = j
+            self.bars[f"k_conv{sk}"].arrive(64)
 
     def issuer(self):
         def qk(t, st, j):
             def start():
-                assert self.k_stage[st] == j, f"QK{t}({j}) reads K stage {st} holding {self.k_stage[st]}"
+                assert self.k_ready[st] == j, f"QK{t}({j}) reads K stage {st} holding {self.k_ready[st]}"
                 self.k_readers[st] += 1
                 self.s_users[t] += 1
 
@@ -134,8 +165,9 @@ class Model:
                 self.o_users[t] -= 1
             self.mma_group(start, finish)
 
+        kbar = "k_conv" if self.convert else "k_full"
         yield ("q_full", 0)
-        yield ("k_full0", 0)
+        yield (f"{kbar}0", 0)
         qk(0, 0, 0)
         self.commit("s_full0")
         qk(1, 0, 0)
@@ -143,26 +175,26 @@ class Model:
         self.commit("k_empty0")
         nkv = self.nkv
         for j in range(nkv):
-            st, st1 = j & 1, (j + 1) & 1
+            sv, sk1 = j % self.vst, (j + 1) % self.kst
             yield ("p_full0", j)
-            yield (f"v_full{st}", j >> 1)
-            pv(0, st, j)
+            yield (f"v_full{sv}", j // self.vst)
+            pv(0, sv, j)
             if j == nkv - 1:
                 self.commit("o_final0")
             if j + 1 < nkv:
-                yield (f"k_full{st1}", (j + 1) >> 1)
-                qk(0, st1, j + 1)
+                yield (f"{kbar}{sk1}", (j + 1) // self.kst)
+                qk(0, sk1, j + 1)
                 self.commit("s_full0")
             if self.mutation != "pv1_without_p1":
                 yield ("p_full1", j)
-            pv(1, st, j)
+            pv(1, sv, j)
             if j == nkv - 1:
                 self.commit("o_final1")
-            self.commit(f"v_empty{st}")
+            self.commit(f"v_empty{sv}")
             if j + 1 < nkv:
-                qk(1, st1, j + 1)
+                qk(1, sk1, j + 1)
                 self.commit("s_full1")
-                self.commit(f"k_empty{st1}")
+                self.commit(f"k_empty{sk1}")
 
     def softmax(self, t):
         for j in range(self.nkv):
@@ -182,6 +214,8 @@ class Model:
     def run(self):
         actors = {"producer": self.producer(), "issuer": self.issuer(),
                   "softmax0": self.softmax(0), "softmax1": self.softmax(1)}
+        if self.convert:
+            actors["converter"] = self.converter()
         waits = {a: None for a in actors}
         for _ in range(10 ** 6):
             if not actors:
@@ -212,18 +246,27 @@ class Model:
         raise AssertionError("no progress")
 
 
+KERNELS = {
+    "phase1_tc": dict(kst=2, vst=2, convert=False),
+    "phase2_tc_d128": dict(kst=3, vst=2, convert=True),
+    "phase2_tc_d64": dict(kst=4, vst=4, convert=True),
+}
+
+
+@pytest.mark.parametrize("kernel", sorted(KERNELS))
 @pytest.mark.parametrize("nkv", [1, 2, 3, 4, 7])
-def test_kernel_protocol_has_no_missed_phase_deadlock_or_race(nkv):
-    for seed in range(400):
-        Model(seed, nkv).run()
+def test_kernel_protocol_has_no_missed_phase_deadlock_or_race(kernel, nkv):
+    for seed in range(300):
+        Model(seed, nkv, **KERNELS[kernel]).run()
 
 
-@pytest.mark.parametrize("mutation", ["v_no_empty_wait", "pv1_without_p1"])
-def test_the_model_catches_planted_protocol_mistakes(mutation):
+@pytest.mark.parametrize("kernel,mutation", [("phase1_tc", "v_no_empty_wait"), ("phase1_tc", "pv1_without_p1"),
+                                             ("phase2_tc_d128", "convert_before_landing")])
+def test_the_model_catches_planted_protocol_mistakes(kernel, mutation):
     caught = 0
     for seed in range(300):
         try:
-            Model(seed, 5, mutation).run()
+            Model(seed, 5, mutation, **KERNELS[kernel]).run()
         except AssertionError:
             caught += 1
     assert caught > 0
