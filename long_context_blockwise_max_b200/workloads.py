@@ -52,6 +52,28 @@ def zipf_token_ids(L: int, vocab: int, s: float = 1.1, seed: int = SEED_IDS,
     return ids.astype(np.int32)
 
 
+def windowed_token_ids(n_blocks: int, block: int, spans=(1, 2, 3, 4, 8, 9, 16), seed: int = 0) -> np.ndarray:
+    """Token ids whose set of blocks is fixed by construction: for every
+    span v in ``spans`` (v <= n_blocks) and start block i there is one id
+    that occurs exactly once in each of the v cyclically consecutive blocks
+    i, i + 1, .., i + v - 1 (mod n_blocks) and nowhere else; id 0 fills the
+    other positions of every block.  Every block therefore holds sum(spans)
+    such ids, at positions shuffled by numpy's PCG64 stream seeded with
+    ``seed``.  Id 1 + s * n_blocks + i is span number s starting at block i
+    (vocabulary 1 + len(spans) * n_blocks)."""
+    spans = [v for v in spans if v <= n_blocks]
+    if sum(spans) > block:
+        raise ValueError("block too short for the requested spans")
+    rng = np.random.Generator(np.random.PCG64(seed))
+    ids = np.zeros(n_blocks * block, dtype=np.int64)
+    for j in range(n_blocks):
+        toks = [1 + s * n_blocks + (j - o) % n_blocks for s, v in enumerate(spans) for o in range(v)]
+        row = np.zeros(block, dtype=np.int64)
+        row[rng.choice(block, size=len(toks), replace=False)] = toks
+        ids[j * block:(j + 1) * block] = row
+    return ids.astype(np.int32)
+
+
 def normal(shape, seed: int, dtype: torch.dtype = torch.float32,
            device: str | torch.device = "cpu") -> torch.Tensor:
     """N(0, 1) tensor of ``shape`` from torch's generator seeded with ``seed``."""

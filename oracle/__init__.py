@@ -25,9 +25,8 @@ from .pulsar_oracle import (  # noqa: F401
     lse_merge,
     phase2_attend,
     phase1_flops,
-    idf_fixed_table,
     chunk_mean_idf,
-    chunk_mean_idf_fixed,
+    chunk_df_product,
     select_evenly_spaced,
     select_summaries_mean_idf,
     phase2_attend_with_self,

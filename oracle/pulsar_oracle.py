@@ -42,8 +42,9 @@ analogue (selection); N = 1 reduces to library causal attention, full-budget
 / zero-sink hosts equal dense causal attention rows, the uniform-score closed
 form lse = ln(r+1), and complex-multiplication RoPE (Phase 1); the shard merge
 equals library dense attention over the concatenated cache (Phase 2).  Added
-rows: mean-IDF against hand-worked Figure-2 means and brute force, evenly
-spaced chunks against their closed form; the query-host step against masked
+rows: mean-IDF against hand-worked Figure-2 means, a hand-worked tie at
+N = 16 and brute force over a high-precision evaluation of the real mean
+IDF; evenly spaced chunks against their closed form; the query-host step against masked
 library attention; ART with zero thresholds against library attention and
 its stop block against a closed form where the weights underflow.
 """
@@ -141,21 +142,9 @@ def select_summaries(ids: np.ndarray, block: int, chunk: int, k: int, vocab: int
 # scores and the non-statistical baselines; [P] §2.1 contrasts max with mean)
 # ----------------------------------------------------------------------------
 
-FIXED_BITS = 24
-
-
-def idf_fixed_table(n_blocks: int) -> list:
-    """q[df] = nearest integer to ln(N / df) * 2^24 for df = 1..N (q[0] = 0).
-    Mean-IDF ranks chunks by a sum of IDF values; the decision is taken on
-    this fixed-point scale (the precision the CUDA path uses), so that equal
-    multisets of df give equal sums whatever the summation order."""
-    return [0] + [int(round(math.log(float(n_blocks) / df) * (1 << FIXED_BITS)))
-                  for df in range(1, n_blocks + 1)]
-
-
 def chunk_mean_idf(ids: np.ndarray, block: int, chunk: int, idf: np.ndarray) -> np.ndarray:
     """Mean IDF over each chunk's tokens (exactly rounded sum / chunk),
-    float64 [N][C]."""
+    float64 [N][C].  Reported score only: the ranking below is exact."""
     blocks = _blocks(ids, block)
     C = block // chunk
     out = np.empty((len(blocks), C), dtype=np.float64)
@@ -165,16 +154,24 @@ def chunk_mean_idf(ids: np.ndarray, block: int, chunk: int, idf: np.ndarray) -> 
     return out
 
 
-def chunk_mean_idf_fixed(ids: np.ndarray, block: int, chunk: int, df: np.ndarray) -> np.ndarray:
-    """Sum over each chunk's tokens of q[df(t)] (see idf_fixed_table),
-    int64 [N * C] in sequence order."""
+def chunk_df_product(ids: np.ndarray, block: int, chunk: int, df: np.ndarray) -> list:
+    """Product of df(t) over each chunk's tokens, as exact Python integers
+    [N * C] in sequence order.
+
+    With every chunk holding the same number c of tokens,
+        mean IDF = (1/c) sum_t ln(N / df(t)) = ln N - (1/c) ln prod_t df(t),
+    so a higher mean IDF is exactly a smaller product, and equal means are
+    exactly equal products: the real-valued order of the definition, with
+    its ties, and no rounding anywhere."""
     blocks = _blocks(ids, block)
-    q = idf_fixed_table(len(blocks))
     C = block // chunk
-    out = np.empty(len(blocks) * C, dtype=np.int64)
-    for j, blk in enumerate(blocks):
+    out = []
+    for blk in blocks:
         for c in range(C):
-            out[j * C + c] = sum(q[int(df[t])] for t in blk[c * chunk:(c + 1) * chunk].tolist())
+            prod = 1
+            for t in blk[c * chunk:(c + 1) * chunk].tolist():
+                prod *= int(df[t])
+            out.append(prod)
     return out
 
 
@@ -186,18 +183,30 @@ def select_evenly_spaced(n_blocks: int, block: int, chunk: int, k: int) -> np.nd
     return np.tile(np.array(row, dtype=np.int64), (n_blocks, 1)).reshape(n_blocks, k)
 
 
-def select_summaries_mean_idf(ids: np.ndarray, block: int, chunk: int, k: int, vocab: int):
-    """Top-k chunks per block by mean IDF (on the fixed-point scale of
-    idf_fixed_table), kept in original order; ties go to the lower index."""
+def select_summaries_mean_idf(ids: np.ndarray, block: int, chunk: int, k: int, vocab: int,
+                              return_rank: bool = False):
+    """Top-k chunks per block by mean IDF ([P] §3.1, Table 1; §2.1 contrasts
+    the maximum with the mean), kept in original order; equal means go to the
+    lower chunk index.  The order is the exact real-valued one: ascending
+    product of df over the chunk (chunk_df_product).
+
+    Returns int64 [N][k] local chunk indices, ascending (and, when
+    ``return_rank``, int64 [N * C]: each chunk's 0-based position in its
+    block's order, best first)."""
     n_blocks = len(ids) // block
     C = block // chunk
+    if not 0 <= k <= C:
+        raise ValueError("k must be in [0, block/chunk]")
     df = document_frequency(ids, block, vocab)
-    sc = chunk_mean_idf_fixed(ids, block, chunk, df).reshape(n_blocks, C)
+    prod = chunk_df_product(ids, block, chunk, df)
     sel = np.empty((n_blocks, k), dtype=np.int64)
+    rank = np.empty(n_blocks * C, dtype=np.int64)
     for j in range(n_blocks):
-        order = sorted(range(C), key=lambda c: (-int(sc[j, c]), c))
+        order = sorted(range(C), key=lambda c: (prod[j * C + c], c))
+        for r, c in enumerate(order):
+            rank[j * C + c] = r
         sel[j] = sorted(order[:k])
-    return sel
+    return (sel, rank) if return_rank else sel
 
 
 # ----------------------------------------------------------------------------

@@ -146,7 +146,7 @@ def test_budget_and_prefix_arithmetic():
     assert [len(p) for p in pos] == [4096, 4096 + 64 + 512, 4096 + 64 + 1024, 4096 + 1600]
 
 
-def test_mean_idf_figure2_and_fixed_scale():
+def test_mean_idf_figure2():
     g = json.load(open(os.path.join(GOLDEN, "figure2_toy.json")))
     ids = np.array(g["ids"], dtype=np.int64)
     df = oracle.document_frequency(ids, g["block"], g["vocab"])
@@ -156,24 +156,143 @@ def test_mean_idf_figure2_and_fixed_scale():
     np.testing.assert_allclose(oracle.chunk_mean_idf(ids, g["block"], g["chunk"], idf), want, rtol=0, atol=1e-15)
     assert oracle.select_summaries_mean_idf(ids, g["block"], g["chunk"], 1, g["vocab"]).tolist() == \
         g["expected_mean_idf_selection"]
-    # the fixed-point table: q[df] ~ ln(N/df) * 2^24, q[N] = 0
-    q = oracle.idf_fixed_table(4)
-    assert q[4] == 0 and abs(q[1] - math.log(4.0) * 2 ** 24) <= 0.5 and abs(q[2] - math.log(2.0) * 2 ** 24) <= 0.5
-    fx = oracle.chunk_mean_idf_fixed(ids, g["block"], g["chunk"], df).reshape(4, 4)
-    assert (np.abs(fx / 2.0 ** 24 / g["chunk"] - want) <= 4 * 0.5 / 2 ** 24 / g["chunk"] + 1e-15).all()
 
 
-@pytest.mark.parametrize("seed", range(4))
-def test_mean_idf_brute_force(seed):
-    rng = np.random.default_rng(500 + seed)
-    block, chunk, n, vocab = 32, 4, 4, 14
-    ids = rng.integers(0, vocab, size=block * n)
+def _tie_case(swap: bool):
+    """N = 16 blocks of four 4-token chunks, worked by hand.  Token 0 is in
+    every block (df 16, IDF 0), token 1 in block 0 only (df 1), token 2 in
+    blocks 0..8 (df 9), tokens 3 and 4 in blocks 0..2 (df 3).  In block 0 the
+    chunks {3, 4, 0, 0} and {1, 2, 0, 0} have the same mean IDF:
+    (2 ln(16/3)) / 4 = (ln 16 + ln(16/9)) / 4, since ln 9 = 2 ln 3; the two
+    all-filler chunks have mean 0."""
+    F = 0
+    blocks = []
+    pair_a, pair_b = [3, 4, F, F], [1, 2, F, F]
+    if swap:
+        pair_a, pair_b = pair_b, pair_a
+    blocks.append([F] * 4 + pair_a + pair_b + [F] * 4)
+    for j in range(1, 16):
+        head = [2 if j <= 8 else F, 3 if j <= 2 else F, 4 if j <= 2 else F, F]
+        blocks.append(head + [F] * 12)
+    ids = np.array(sum(blocks, []), dtype=np.int64)
+    df = oracle.document_frequency(ids, 16, 5)
+    assert df.tolist() == [16, 1, 9, 3, 3]
+    return ids
+
+
+@pytest.mark.parametrize("swap", [False, True])
+def test_mean_idf_hand_worked_tie_at_n16(swap):
+    ids = _tie_case(swap)
+    idf = oracle.idf_table(oracle.document_frequency(ids, 16, 5), 16)
+    m = oracle.chunk_mean_idf(ids, 16, 4, idf)[0]
+    assert abs(m[1] - m[2]) < 1e-15 and abs(m[1] - 2 * math.log(16 / 3) / 4) < 1e-15
+    # equal real means: the lower chunk index wins, whichever multiset it holds
+    assert oracle.select_summaries_mean_idf(ids, 16, 4, 1, 5)[0].tolist() == [1]
+    assert oracle.select_summaries_mean_idf(ids, 16, 4, 2, 5)[0].tolist() == [1, 2]
+    _, rank = oracle.select_summaries_mean_idf(ids, 16, 4, 1, 5, return_rank=True)
+    assert rank[:4].tolist() == [2, 0, 1, 3]
+
+
+def _real_mean_idf_resolved(ids, block, chunk, vocab):
+    """The definition evaluated to 60 significant digits: mean over each
+    chunk's tokens of ln(N / df(t)), df counted by brute force over the
+    blocks.  Means of c-token chunks with N <= 64 that differ at all differ
+    by at least ln(1 + 64^-c) / c, above 1e-16 for c <= 8, so values closer
+    than 1e-40 are the same real number; each value is replaced by the
+    smallest value of its group of equals."""
+    from decimal import Decimal, getcontext
+    getcontext().prec = 60
+    n = len(ids) // block
+    sets = [set(ids[j * block:(j + 1) * block].tolist()) for j in range(n)]
+    C = block // chunk
+    rows = []
+    for j in range(n):
+        vals = []
+        for c in range(C):
+            toks = ids[j * block + c * chunk:j * block + (c + 1) * chunk].tolist()
+            tot = sum((Decimal(n) / Decimal(sum(t in s for s in sets))).ln() for t in toks)
+            vals.append(tot / Decimal(chunk))
+        srt = sorted(vals)
+        rep = {}
+        for v in srt:
+            rep[v] = next(w for w in srt if abs(w - v) < Decimal("1e-40"))
+        rows.append([rep[v] for v in vals])
+    return rows
+
+
+def _brute_force_real_order(n_blocks):
+    """Brute force over every k-subset against the real-valued mean IDF
+    (not the oracle's integer products).  Returns the number of exact real
+    ties between chunks with different df multisets."""
+    rng = np.random.default_rng(900 + n_blocks)
+    block, chunk, vocab = 16, 2, 40
+    # every id confined to a random set of blocks whose size is a power of
+    # two, 3 or 9 (so that different df multisets often have equal products,
+    # e.g. {1, 4} and {2, 2}, {1, 9} and {3, 3}); others of any size
+    sizes = [z for z in (1, 2, 3, 4, 8, 9, 16, 32, 64) if z <= n_blocks]
+    home = [rng.choice(n_blocks, size=int(rng.choice(sizes)) if t % 4 else int(rng.integers(1, n_blocks + 1)),
+                       replace=False) for t in range(vocab)]
+    ids = np.empty(n_blocks * block, dtype=np.int64)
+    for j in range(n_blocks):
+        allowed = [t for t in range(vocab) if j in home[t]] or [0]
+        ids[j * block:(j + 1) * block] = rng.choice(allowed, size=block)
+    real = _real_mean_idf_resolved(ids, block, chunk, vocab)
     df = oracle.document_frequency(ids, block, vocab)
-    sc = oracle.chunk_mean_idf_fixed(ids, block, chunk, df).reshape(n, block // chunk)
-    for k in (1, 3, 8):
-        sel = oracle.select_summaries_mean_idf(ids, block, chunk, k, vocab)
-        for j in range(n):
-            assert sel[j].tolist() == _brute_force_topk(sc[j].tolist(), k)
+    prods = oracle.chunk_df_product(ids, block, chunk, df)
+    C = block // chunk
+    cross_ties = 0
+    for j in range(n_blocks):
+        for a in range(C):
+            for b in range(a + 1, C):
+                ma = sorted(int(df[t]) for t in ids[j * block + a * chunk:j * block + (a + 1) * chunk])
+                mb = sorted(int(df[t]) for t in ids[j * block + b * chunk:j * block + (b + 1) * chunk])
+                cross_ties += real[j][a] == real[j][b] and ma != mb
+    for k in (1, 3, 5):
+        sel, rank = oracle.select_summaries_mean_idf(ids, block, chunk, k, vocab, return_rank=True)
+        for j in range(n_blocks):
+            assert sel[j].tolist() == _brute_force_topk(real[j], k)
+            order = sorted(range(C), key=lambda c: (-real[j][c], c))
+            assert [int(rank[j * C + c]) for c in order] == list(range(C))
+    assert len(prods) == n_blocks * C
+    return cross_ties
+
+
+@pytest.mark.parametrize("n_blocks", [16, 32, 64])
+def test_mean_idf_brute_force_real_order(n_blocks):
+    _brute_force_real_order(n_blocks)
+
+
+@pytest.mark.parametrize("n_blocks", [16, 32, 64])
+def test_mean_idf_planted_ties_real_order(n_blocks):
+    """Ids whose df values are fixed by construction (1, 2, 3, 4, 8, 9, 16 and
+    the filler's N), paired into 2-token chunks: many chunks with different
+    df multisets have equal real means ({1, 4} and {2, 2}, {1, 9} and {3, 3},
+    {2, 8} and {4, 4}, ...).  The oracle's full order must be the real-valued
+    order, ties to the lower index."""
+    block, chunk = 64, 2
+    ids = workloads.windowed_token_ids(n_blocks, block, seed=40 + n_blocks).astype(np.int64)
+    vocab = 1 + 7 * n_blocks
+    real = _real_mean_idf_resolved(ids, block, chunk, vocab)
+    df = oracle.document_frequency(ids, block, vocab)
+    C = block // chunk
+    cross = 0
+    for j in range(n_blocks):
+        ms = [sorted(int(df[t]) for t in ids[j * block + c * chunk:j * block + (c + 1) * chunk]) for c in range(C)]
+        cross += sum(real[j][a] == real[j][b] and ms[a] != ms[b] for a in range(C) for b in range(a + 1, C))
+    assert cross >= n_blocks, cross
+    for k in (1, 4, 11):
+        sel, rank = oracle.select_summaries_mean_idf(ids, block, chunk, k, vocab, return_rank=True)
+        for j in range(n_blocks):
+            order = sorted(range(C), key=lambda c: (-real[j][c], c))
+            assert sel[j].tolist() == sorted(order[:k])
+            assert [int(rank[j * C + c]) for c in order] == list(range(C))
+
+
+def test_mean_idf_brute_force_has_cross_multiset_ties():
+    # the brute-force cases must include equal real means reached by
+    # different df multisets (the case a rounded score can get wrong)
+    ties = [_brute_force_real_order(n) for n in (16, 32, 64)]
+    assert sum(ties) > 0, ties
 
 
 def test_evenly_spaced_closed_form():
