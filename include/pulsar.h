@@ -134,13 +134,18 @@ typedef enum {
  * [P] §3.1 (Table 1 compares Max-IDF with other statistical scores and with
  * non-statistical baselines; §2.1 contrasts the maximum with the mean).
  * Same sizes, rules, outputs and tie-break as pulsar_select_summaries.
- *  - PA_SCORE_MEAN_IDF ranks chunks by sum_t q[df(t)] with
- *    q[df] = round(ln(N/df) * 2^24) (the mean times the chunk length, on a
- *    fixed-point scale so that ranking is exact and order-independent);
- *    block / chunk <= 8192 (PA_ERR_UNSUPPORTED otherwise).
+ *  - PA_SCORE_MEAN_IDF ranks chunks by their mean IDF,
+ *    (1/chunk) sum_t ln(N / df(t)), exactly: with a fixed chunk length the
+ *    mean is ln N - ln(prod_t df(t)) / chunk, so the order is that of the
+ *    integer product of df over the chunk (ascending), compared as exact
+ *    256-bit integers; equal means go to the lower chunk index.  Requires
+ *    chunk <= 32 and block / chunk <= 4096 (PA_ERR_UNSUPPORTED otherwise).
  *  - PA_SCORE_EVENLY_SPACED does not read ids (may be NULL).
- *  chunk_score_opt  out [L / chunk] int64: the fixed-point sums (mean-IDF),
- *                   the min df (max-IDF), not written (evenly spaced); or NULL.
+ *  chunk_score_opt  out [L / chunk] int64, or NULL: for PA_SCORE_MEAN_IDF
+ *                   each chunk's rank in its block's order (0 = highest
+ *                   mean IDF; the ranks of a block are a permutation of
+ *                   0 .. block/chunk - 1); for PA_SCORE_MAX_IDF the min df;
+ *                   not written for PA_SCORE_EVENLY_SPACED.
  * Workspace: pa_select_workspace_size.
  */
 int pulsar_select_summaries_scored(const int32_t* ids, int64_t L, int32_t vocab, int32_t block,

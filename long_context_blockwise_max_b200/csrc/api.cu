@@ -189,7 +189,7 @@ size_t pa_select_workspace_size(int64_t L, int32_t vocab, int32_t block, int32_t
   size_t b = kStatusBytes;
   b += align_up(sizeof(unsigned long long) * (size_t)vocab);
   b += align_up(sizeof(int32_t) * (size_t)(L / chunk));
-  b += align_up(sizeof(long long) * (size_t)(L / chunk));   // fixed-point scores (scorer variants)
+  b += align_up(kScoreKeyBytes * (size_t)(L / chunk));      // mean-IDF keys (scorer variants)
   return b;
 }
 
@@ -206,7 +206,8 @@ int pulsar_select_summaries_scored(const int32_t* ids, int64_t L, int32_t vocab,
   if ((ids == nullptr && method != PA_SCORE_EVENLY_SPACED) || (sel == nullptr && k_chunks > 0))
     return PA_ERR_INVALID;
   if (L / block > kMaxBlocks) return PA_ERR_UNSUPPORTED;
-  if (method == PA_SCORE_MEAN_IDF && block / chunk > kMaxScoredChunks) return PA_ERR_UNSUPPORTED;
+  if (method == PA_SCORE_MEAN_IDF && (block / chunk > kMaxScoredChunks || chunk > kMaxScoredChunk))
+    return PA_ERR_UNSUPPORTED;
   const size_t need = pa_select_workspace_size(L, vocab, block, chunk);
   int rc = check_ws(ws, ws_bytes, need);
   if (rc) return rc;
@@ -222,24 +223,17 @@ int pulsar_select_summaries_scored(const int32_t* ids, int64_t L, int32_t vocab,
   off += align_up(sizeof(unsigned long long) * (size_t)vocab);
   int32_t* mindf = reinterpret_cast<int32_t*>(w + off);
   off += align_up(sizeof(int32_t) * (size_t)(L / chunk));
-  long long* score = chunk_score_opt ? reinterpret_cast<long long*>(chunk_score_opt)
-                                     : reinterpret_cast<long long*>(w + off);
+  long long* score = reinterpret_cast<long long*>(chunk_score_opt);
+  a.mindf = mindf;
   if (method == PA_SCORE_MAX_IDF) {
-    a.mindf = mindf;
     rc = launch_select(a, s);
-    if (rc == PA_OK && chunk_score_opt != nullptr) {
+    if (rc == PA_OK && score != nullptr) {
       // widen the min df of every chunk into the caller's int64 array
       rc = launch_widen_i32(mindf, score, L / chunk, s);
     }
     return rc;
   }
-  FixedIdf tab;
-  const int n = (int)(L / block);
-  tab.q[0] = 0;
-  for (int df = 1; df <= kMaxBlocks; ++df)
-    tab.q[df] = df <= n ? llround(std::log((double)n / df) * (double)(1 << 24)) : 0;
-  a.mindf = mindf;
-  return launch_select_scored(a, method, tab, score, s);
+  return launch_select_scored(a, method, w + off, score, s);
 }
 
 int pulsar_select_summaries(const int32_t* ids, int64_t L, int32_t vocab, int32_t block,

@@ -32,13 +32,15 @@ struct SelectArgs {
 };
 int launch_select(const SelectArgs& a, cudaStream_t s);
 
-// q[df] = round(ln(N/df) * 2^24), df = 0..N (q[0] unused)
-struct FixedIdf {
-  long long q[kMaxBlocks + 1];
-};
-constexpr int kMaxScoredChunks = 8192;   // chunks per block for the rank-based top-k
+// Mean-IDF scorer: chunks are ranked by the exact product of df over their
+// tokens, a 256-bit key per chunk (32 bytes of workspace per chunk).
+constexpr int kMaxScoredChunks = 4096;   // chunks per block (keys staged in shared memory)
+constexpr int kMaxScoredChunk = 32;      // tokens per chunk: 64^32 < 2^256
+constexpr size_t kScoreKeyBytes = 32;
 int launch_widen_i32(const int32_t* in, long long* out, int64_t n, cudaStream_t s);
-int launch_select_scored(const SelectArgs& a, int method, const FixedIdf& tab, long long* score,
+// key_ws: [L / chunk] 32-byte keys; a.mindf receives the int32 ranks;
+// rank_out (optional) the int64 ranks.
+int launch_select_scored(const SelectArgs& a, int method, void* key_ws, long long* rank_out,
                          cudaStream_t s);
 
 // Host-computed RoPE frequencies omega_m = theta^(-2m/d), fp64.

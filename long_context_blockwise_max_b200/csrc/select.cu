@@ -188,55 +188,109 @@ __global__ void __launch_bounds__(THREADS) topk_kernel(const int32_t* __restrict
 
 // ---------------------------------------------------------------------------
 // Alternative scorers (Pulsar Attention page §3.1, Table 1).
-//  chunk_fixed_score_kernel: mean-IDF as the sum over the chunk's tokens of
-//    q[df] = round(ln(N/df) * 2^24) (int64, exact and order-independent).
-//  topk_rank_kernel: per block, a chunk is kept when fewer than k chunks
-//    beat it (higher score, or equal score and lower index); ordered
-//    compaction as in topk_kernel.
+//  Mean IDF.  Every chunk holds the same number c of tokens, so
+//    mean IDF = (1/c) sum_t ln(N / df(t)) = ln N - (1/c) ln prod_t df(t):
+//  a higher mean is exactly a smaller product of df, and equal means are
+//  exactly equal products.  The product of at most 32 values in 1..64 is
+//  below 2^193, so it is kept exactly as a 256-bit integer (four 64-bit
+//  limbs, least significant first) and chunks are ranked by it.
+//  chunk_df_product_kernel: one warp per chunk, product tree in 64 bits over
+//    groups of 8 lanes (at most 2^48 each), then four multiword products.
+//  rank_kernel: the rank of a chunk in its block is the number of chunks
+//    with a smaller key, or an equal key and a lower index (a permutation of
+//    0..C-1); a chunk is kept when its rank is below k.  Without a rank
+//    output the count stops at k.
+//  select_by_rank_kernel: ordered compaction of the chunks with rank < k.
 //  evenly_spaced_kernel: chunk floor(m * C / k) in every block.
 // ---------------------------------------------------------------------------
-__global__ void chunk_fixed_score_kernel(const int32_t* __restrict__ ids, int64_t n_chunks,
-                                         int32_t chunk, int32_t vocab,
-                                         const unsigned long long* __restrict__ mask, FixedIdf tab,
-                                         long long* __restrict__ score) {
+struct Key256 {
+  unsigned long long w[4];
+};
+
+__device__ __forceinline__ void key_mul_small(Key256& a, unsigned long long f) {
+  unsigned long long carry = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const unsigned long long lo = a.w[i] * f;
+    const unsigned long long hi = __umul64hi(a.w[i], f);
+    const unsigned long long sum = lo + carry;
+    carry = hi + (sum < lo ? 1ull : 0ull);
+    a.w[i] = sum;
+  }
+}
+
+__device__ __forceinline__ bool key_less(const Key256& a, const Key256& b) {
+#pragma unroll
+  for (int i = 3; i >= 0; --i)
+    if (a.w[i] != b.w[i]) return a.w[i] < b.w[i];
+  return false;
+}
+
+__device__ __forceinline__ bool key_equal(const Key256& a, const Key256& b) {
+  return a.w[0] == b.w[0] && a.w[1] == b.w[1] && a.w[2] == b.w[2] && a.w[3] == b.w[3];
+}
+
+__global__ void chunk_df_product_kernel(const int32_t* __restrict__ ids, int64_t n_chunks, int32_t chunk,
+                                        int32_t vocab, const unsigned long long* __restrict__ mask,
+                                        Key256* __restrict__ key) {
   const int lane = threadIdx.x & 31;
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   for (int64_t c = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; c < n_chunks;
        c += nwarps) {
-    long long acc = 0;
-    const int32_t* tok = ids + c * chunk;
-    for (int u = lane; u < chunk; u += 32) {
-      const int t = tok[u];
-      if (t >= 0 && t < vocab) acc += tab.q[__popcll(mask[t])];
+    unsigned long long f = 1;   // lanes past the chunk, and invalid ids, contribute 1
+    if (lane < chunk) {
+      const int t = ids[c * chunk + lane];
+      if (t >= 0 && t < vocab) f = (unsigned long long)__popcll(mask[t]);
     }
+    // products of 8 consecutive lanes: at most 64^8 = 2^48
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) score[c] = acc;
+    for (int off = 1; off < 8; off <<= 1) f *= __shfl_xor_sync(0xffffffffu, f, off);
+    const unsigned long long p8 = __shfl_sync(0xffffffffu, f, 8);
+    const unsigned long long p16 = __shfl_sync(0xffffffffu, f, 16);
+    const unsigned long long p24 = __shfl_sync(0xffffffffu, f, 24);
+    if (lane == 0) {
+      Key256 k;
+      k.w[0] = f;
+      k.w[1] = k.w[2] = k.w[3] = 0;
+      key_mul_small(k, p8);
+      key_mul_small(k, p16);
+      key_mul_small(k, p24);
+      key[c] = k;
+    }
   }
 }
 
+// grid (ceil(C / 256), n_blocks); the block's keys are staged in shared memory.
+__global__ void __launch_bounds__(256) rank_kernel(const Key256* __restrict__ key, int32_t C, int32_t k,
+                                                   int32_t* __restrict__ rank,
+                                                   long long* __restrict__ rank_out) {
+  extern __shared__ Key256 sk[];
+  const int j = blockIdx.y;
+  const Key256* kb = key + (int64_t)j * C;
+  for (int o = threadIdx.x; o < C; o += blockDim.x) sk[o] = kb[o];
+  __syncthreads();
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= C) return;
+  const Key256 v = sk[c];
+  const int stop = rank_out != nullptr ? C : k;   // the count only decides rank < k
+  int better = 0;
+  for (int o = 0; o < C && better < stop; ++o) {
+    const Key256 w = sk[o];
+    better += key_less(w, v) || (o < c && key_equal(w, v));
+  }
+  rank[(int64_t)j * C + c] = better;
+  if (rank_out != nullptr) rank_out[(int64_t)j * C + c] = better;
+}
+
 template <int THREADS>
-__global__ void __launch_bounds__(THREADS) topk_rank_kernel(const long long* __restrict__ score,
-                                                            int32_t C, int32_t k,
-                                                            int32_t* __restrict__ sel) {
-  extern __shared__ long long sc[];
+__global__ void __launch_bounds__(THREADS) select_by_rank_kernel(const int32_t* __restrict__ rank, int32_t C,
+                                                                 int32_t k, int32_t* __restrict__ sel) {
   __shared__ int warp_tot[THREADS / 32];
   const int j = blockIdx.x;
-  for (int c = threadIdx.x; c < C; c += THREADS) sc[c] = score[(int64_t)j * C + c];
-  __syncthreads();
   int base_sel = 0;
   for (int base = 0; base < C; base += THREADS) {
     const int c = base + threadIdx.x;
-    bool take = false;
-    if (c < C) {
-      const long long v = sc[c];
-      int better = 0;
-      for (int o = 0; o < C && better < k; ++o) {
-        const long long w = sc[o];
-        better += (w > v) || (w == v && o < c);
-      }
-      take = better < k;
-    }
+    const bool take = c < C && rank[(int64_t)j * C + c] < k;
     int tot;
     const int pos = base_sel + block_exclusive_count<THREADS>(take, warp_tot, &tot);
     if (take) sel[(int64_t)j * k + pos] = c;
@@ -279,7 +333,7 @@ static int launch_presence(const SelectArgs& a, cudaStream_t s) {
   return PA_OK;
 }
 
-int launch_select_scored(const SelectArgs& a, int method, const FixedIdf& tab, long long* score,
+int launch_select_scored(const SelectArgs& a, int method, void* key_ws, long long* rank_out,
                          cudaStream_t s) {
   const int64_t n_chunks = a.L / a.chunk;
   const int C = a.block / a.chunk;
@@ -293,17 +347,19 @@ int launch_select_scored(const SelectArgs& a, int method, const FixedIdf& tab, l
   }
   int rc = launch_presence(a, s);
   if (rc) return rc;
+  Key256* key = static_cast<Key256*>(key_ws);
   const int threads = 256;
   const int64_t wgrid = (n_chunks * 32 + threads - 1) / threads;
-  chunk_fixed_score_kernel<<<(int)(wgrid < 148 * 32 ? wgrid : 148 * 32), threads, 0, s>>>(
-      a.ids, n_chunks, a.chunk, a.vocab, a.mask, tab, score);
-  if (a.k > 0) {
-    const size_t sm = sizeof(long long) * (size_t)C;
-    if (cudaFuncSetAttribute(topk_rank_kernel<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)sm) != cudaSuccess)
+  chunk_df_product_kernel<<<(int)(wgrid < 148 * 32 ? wgrid : 148 * 32), threads, 0, s>>>(
+      a.ids, n_chunks, a.chunk, a.vocab, a.mask, key);
+  if (a.k > 0 || rank_out != nullptr) {
+    const size_t sm = sizeof(Key256) * (size_t)C;
+    if (cudaFuncSetAttribute(rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) != cudaSuccess)
       return PA_ERR_CUDA;
-    topk_rank_kernel<1024><<<n_blocks, 1024, sm, s>>>(score, C, a.k, a.sel);
+    const dim3 grid((unsigned)((C + 255) / 256), (unsigned)n_blocks);
+    rank_kernel<<<grid, 256, sm, s>>>(key, C, a.k, a.mindf, rank_out);
   }
+  if (a.k > 0) select_by_rank_kernel<1024><<<n_blocks, 1024, 0, s>>>(a.mindf, C, a.k, a.sel);
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 

@@ -214,7 +214,9 @@ def pulsar_select_summaries_noalloc(ids: torch.Tensor, vocab: int, block: int, c
 def pulsar_select_summaries_scored(ids, vocab: int, block: int, chunk: int, k_chunks: int, method: int,
                                    L: int | None = None, sel=None, want_scores=False, ws=None):
     """Selection with another chunk scorer (PA_SCORE_*).  ``ids`` may be None
-    for PA_SCORE_EVENLY_SPACED (then pass ``L``).  Returns (sel, scores or None, ws)."""
+    for PA_SCORE_EVENLY_SPACED (then pass ``L``).  Returns (sel, scores or
+    None, ws); with ``want_scores`` the int64 scores are each chunk's rank in
+    its block (mean IDF) or its min df (max IDF)."""
     _dev(ids, sel)
     L = ids.numel() if ids is not None else int(L)
     dev = ids.device if ids is not None else torch.device("cuda", torch.cuda.current_device())

@@ -110,12 +110,15 @@ def test_host_validation_of_the_other_entry_points(lib):
     assert so.pa_set_profile_events(dummy, None) == -1
     assert so.pa_set_profile_events(None, dummy) == -1
     assert so.pa_set_profile_events(None, None) == 0
-    # scorer: unknown method; missing ids for a scorer that reads them; mean-IDF beyond 8192 chunks per block
+    # scorer: unknown method; missing ids for a scorer that reads them; mean-IDF beyond 4096 chunks per
+    # block or beyond 32 tokens per chunk (the exact 256-bit product)
     assert so.pulsar_select_summaries_scored(dummy, 1024, 100, 512, 32, 2, 3, dummy, None, ws, 1 << 20,
                                              None) == -1
     assert so.pulsar_select_summaries_scored(None, 1024, 100, 512, 32, 2, 1, dummy, None, ws, 1 << 20,
                                              None) == -1
-    assert so.pulsar_select_summaries_scored(dummy, 16384, 100, 16384, 1, 1, 1, dummy, None, ws, 1 << 30,
+    assert so.pulsar_select_summaries_scored(dummy, 8192, 100, 8192, 1, 1, 1, dummy, None, ws, 1 << 30,
+                                             None) == -2
+    assert so.pulsar_select_summaries_scored(dummy, 4096, 100, 1024, 64, 1, 1, dummy, None, ws, 1 << 30,
                                              None) == -2
 
     def art(dtype=1, Tq=1, hq=32, hkv=8, block_keys=128, tau=1e-5, phi=1e-3, patience=5, theta=5e5):

@@ -1,7 +1,8 @@
 """GPU parity of the alternative summary scorers (Pulsar Attention page
-§3.1, Table 1): mean-IDF on the fixed-point scale and evenly spaced
-sampling, bit-exact against the oracle; Max-IDF through the scored entry
-point equals pulsar_select_summaries."""
+§3.1, Table 1): mean-IDF (exact order, ties to the lower index) and evenly
+spaced sampling, bit-exact against the oracle -- the selection and every
+chunk's rank; Max-IDF through the scored entry point against the oracle's
+selection and min df."""
 import json
 import os
 
@@ -31,24 +32,52 @@ def _cases():
     yield workloads.zipf_token_ids(8 * 4096, 700, 1.1, seed=7), 700, 4096, 32, 16
     w = workloads.LLAMA_32K
     yield w.token_ids(), w.vocab, w.block, w.chunk, w.k_chunks
+    # df fixed by construction (1, 2, 3, 4, 8, 9, 16 and N): many equal real
+    # means from different df multisets ({1, 9} and {3, 3}, {2, 8} and {4, 4})
+    # at N = 16, 32 and 64, in 2-token and 32-token chunks
+    for n in (16, 32, 64):
+        yield workloads.windowed_token_ids(n, 64, seed=40 + n), 1 + 7 * n, 64, 2, 11
+    yield workloads.windowed_token_ids(64, 1024, seed=5), 1 + 7 * 64, 1024, 32, 4   # products up to 2^192
 
 
-@pytest.mark.parametrize("idx", range(5))
+N_CASES = 9
+
+
+@pytest.mark.parametrize("idx", range(N_CASES))
 def test_mean_idf_and_evenly_spaced(P, idx):
     ids, vocab, block, chunk, k = list(_cases())[idx]
     ids = ids.astype(np.int32)
     dev_ids = torch.from_numpy(ids).to(DEV)
-    sel, sc, ws = P.pulsar_select_summaries_scored(dev_ids, vocab, block, chunk, k, P.PA_SCORE_MEAN_IDF,
-                                                  want_scores=True)
+    sel, rank, ws = P.pulsar_select_summaries_scored(dev_ids, vocab, block, chunk, k, P.PA_SCORE_MEAN_IDF,
+                                                    want_scores=True)
     assert P.pa_workspace_status(ws) == 0
-    df = oracle.document_frequency(ids, block, vocab)
-    assert np.array_equal(sc.cpu().numpy(), oracle.chunk_mean_idf_fixed(ids, block, chunk, df))
-    assert np.array_equal(sel.cpu().numpy(), oracle.select_summaries_mean_idf(ids, block, chunk, k, vocab))
+    want_sel, want_rank = oracle.select_summaries_mean_idf(ids, block, chunk, k, vocab, return_rank=True)
+    assert np.array_equal(rank.cpu().numpy(), want_rank)
+    assert np.array_equal(sel.cpu().numpy(), want_sel)
+    sel_nr, none, _ = P.pulsar_select_summaries_scored(dev_ids, vocab, block, chunk, k, P.PA_SCORE_MEAN_IDF)
+    assert none is None and np.array_equal(sel_nr.cpu().numpy(), want_sel)
     sel2, _, _ = P.pulsar_select_summaries_scored(None, vocab, block, chunk, k, P.PA_SCORE_EVENLY_SPACED,
                                                  L=ids.size)
     assert np.array_equal(sel2.cpu().numpy(), oracle.select_evenly_spaced(ids.size // block, block, chunk, k))
     sel3, sc3, _ = P.pulsar_select_summaries_scored(dev_ids, vocab, block, chunk, k, P.PA_SCORE_MAX_IDF,
                                                    want_scores=True)
-    ref, _, mdf, _ = P.pulsar_select_summaries(dev_ids, vocab, block, chunk, k, want_mindf=True)
-    assert torch.equal(sel3, ref)
-    assert torch.equal(sc3, mdf.to(torch.int64))
+    df = oracle.document_frequency(ids, block, vocab)
+    assert np.array_equal(sel3.cpu().numpy(), oracle.select_summaries(ids, block, chunk, k, vocab))
+    assert np.array_equal(sc3.cpu().numpy(), oracle.chunk_min_df(ids, block, chunk, df))
+
+
+def test_mean_idf_hand_worked_tie(P):
+    """N = 16, chunks with df {3, 3, 16, 16} and {1, 9, 16, 16}: equal real
+    means, so the lower index wins whichever of the two it holds."""
+    for swap in (False, True):
+        F = 0
+        a, b = [3, 4, F, F], [1, 2, F, F]
+        if swap:
+            a, b = b, a
+        blocks = [[F] * 4 + a + b + [F] * 4]
+        for j in range(1, 16):
+            blocks.append([2 if j <= 8 else F, 3 if j <= 2 else F, 4 if j <= 2 else F, F] + [F] * 12)
+        ids = torch.tensor(sum(blocks, []), dtype=torch.int32, device=DEV)
+        sel, rank, _ = P.pulsar_select_summaries_scored(ids, 5, 16, 4, 1, P.PA_SCORE_MEAN_IDF, want_scores=True)
+        assert sel[0].tolist() == [1]
+        assert rank[:4].tolist() == [2, 0, 1, 3]
