@@ -123,6 +123,7 @@ def test_decode_sampled_groups(P, wname, groups):
         assert_close(f64(o[b:b + 1, :, hs].cpu()), ro, O_TOL[torch.bfloat16], "O")
         assert_close(lse[b:b + 1, :, hs].cpu().double().numpy(), rl, LSE_TOL, "lse")
         assert_close(pl[b:b + 1, :, :, hs].cpu().double().numpy(), rs, LSE_TOL, "s_h")
+        assert_close(f64(po[b:b + 1, :, :, hs].cpu()), ra, O_TOL[torch.bfloat16], "A_h")
 
 
 def test_query_128k_sampled_groups(P):
@@ -140,20 +141,33 @@ def test_query_128k_sampled_groups(P):
         assert_close(lse[:, :, hs].cpu().double().numpy(), rl, LSE_TOL, "lse")
 
 
-def test_lse_merge_entry_point(P):
-    # partials from star_phase2_attend, merged again by pa_lse_merge, give the
-    # same O / lse; an all-empty row merges to O = 0, lse = -inf
-    B, Tq, hq, hkv, d, T, S = 2, 3, 8, 2, 128, 1000, 5
-    q = workloads.normal((B, Tq, hq, d), 70, torch.bfloat16).to(DEV)
-    kc = workloads.normal((B, T, hkv, d), 71, torch.bfloat16).to(DEV)
-    vc = workloads.normal((B, T, hkv, d), 72, torch.bfloat16).to(DEV)
-    o, lse, po, pl, _ = P.star_phase2_attend(q, kc, vc, S, q_pos0=T, rope_theta=1e4, want_partials=True)
-    o2, lse2 = P.pa_lse_merge(po, pl, dtype=torch.bfloat16)
-    assert (o2.float() - o.float()).abs().max().item() <= 1e-2
-    assert (lse2 - lse).abs().max().item() <= 1e-5
-    pl_empty = torch.full_like(pl, float("-inf"))
-    o3, lse3 = P.pa_lse_merge(torch.zeros_like(po), pl_empty, dtype=torch.float32)
-    assert (o3 == 0).all() and torch.isneginf(lse3).all()
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_lse_merge_entry_point(P, dtype):
+    # pa_lse_merge fed partials the oracle computed (fp64 -> fp32), with whole
+    # shards empty (s_h = -inf, A_h garbage that must be ignored) next to
+    # finite ones, and rows whose shards are all empty, against the oracle's
+    # merge of the same partials
+    B, S, Tq, hq, hkv, d, T = 2, 6, 3, 8, 2, 128, 900
+    q = workloads.normal((B, Tq, hq, d), 70, torch.float32)
+    kc = workloads.normal((B, T, hkv, d), 71, torch.float32)
+    vc = workloads.normal((B, T, hkv, d), 72, torch.float32)
+    A, s = oracle.phase2_partials(f64(q), f64(kc), f64(vc), S)
+    s[0, 2] = -np.inf                    # shard 2 of batch 0 empty for every row
+    s[1, :, 1, 3] = -np.inf              # batch 1, token 1, head 3: every shard empty
+    s[1, 4, 2, :] = -np.inf              # batch 1, shard 4, token 2: empty for every head
+    s[0, 1] += 3.0                       # shards of very different weight
+    s[1, 0, 0] -= 40.0
+    A_in = A.copy()
+    A_in[np.isneginf(s)] = 1.0e30        # values of empty shards are ignored
+    po = torch.from_numpy(A_in).float().to(DEV)
+    pl = torch.from_numpy(s).float().to(DEV)
+    o, lse = P.pa_lse_merge(po, pl, dtype=dtype)
+    ro, rl = oracle.lse_merge(A, s)
+    assert_close(f64(o.cpu()), ro, O_TOL[dtype], "O")
+    fin = np.isfinite(rl)
+    assert (~fin).sum() == 1 and torch.isneginf(lse.cpu()[torch.from_numpy(~fin)]).all()
+    assert (o.cpu().float()[torch.from_numpy(~fin)] == 0).all()
+    assert np.abs(lse.cpu().double().numpy()[fin] - rl[fin]).max() <= LSE_TOL
 
 
 @pytest.mark.parametrize("where", ["key", "query"])
