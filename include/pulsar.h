@@ -197,9 +197,19 @@ int pulsar_select_summaries_noalloc(const int32_t* ids, int64_t L, int32_t vocab
 int pa_phase1_layout(int64_t L, int32_t block, int32_t sink, int32_t summary_tokens, int star,
                      int64_t* row_off);
 
-/* Bytes of scratch the Phase-1 calls need (star selects the variant). */
+/* Bytes of scratch the Phase-1 calls need (star selects the variant); enough
+ * for the call over every host and for any host range. */
 size_t pa_phase1_workspace_size(int64_t L, int32_t hq, int32_t hkv, int32_t d, int dtype,
                                 int32_t block, int32_t sink, int32_t summary_tokens, int star);
+
+/* Bytes of scratch a call over hosts [host_begin, host_end) needs (the
+ * *_phase1_encode_hosts calls).  A range that reads few of the sequence's
+ * positions rotates only those: the sink, the summaries of blocks
+ * 0 .. host_end - 2 and its own blocks (Star: B_0 and its own blocks), so
+ * its scratch scales with them, not with L.  0 for invalid arguments. */
+size_t pa_phase1_hosts_workspace_size(int64_t L, int32_t hq, int32_t hkv, int32_t d, int dtype,
+                                      int32_t block, int32_t sink, int32_t summary_tokens, int star,
+                                      int32_t host_begin, int32_t host_end);
 
 /*
  * Pulsar Phase-1 encoding of every host of one attention layer, all hosts
@@ -251,9 +261,12 @@ int star_phase1_encode(const void* q, const void* k, const void* v, int dtype, i
  * sequence's N = L / block hosts: the unit of work of one GPU when the hosts
  * of one sequence are spread over GPUs ([P] §2.1, §2.2: each host encodes
  * its own input and keeps its own block's KV; no communication in Phase 1).
- * Inputs, arguments and workspace size as pulsar_phase1_encode /
- * star_phase1_encode (q, k, v hold the whole sequence; only positions below
- * host_end * block are read).  Outputs cover the range only:
+ * Inputs and arguments as pulsar_phase1_encode / star_phase1_encode (q, k,
+ * v hold the whole sequence; only the positions the range's hosts read are
+ * read and rotated: the sink, the summary chunks of blocks before host_end - 1
+ * and the range's blocks, or B_0 and the range's blocks for Star).
+ * Workspace: pa_phase1_hosts_workspace_size (pa_phase1_workspace_size is
+ * always enough).  Outputs cover the range only:
  *  o, lse_opt     rows row_off[host_begin] .. row_off[host_end] of the full
  *                 layout (pa_phase1_layout), packed from row 0.
  *  k_ret, v_ret   [host_end - host_begin][block][hkv][d]: the range's blocks.

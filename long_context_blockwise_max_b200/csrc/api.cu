@@ -50,6 +50,36 @@ int layout(int64_t L, int32_t block, int32_t sink, int32_t summary_tokens, int s
   return PA_OK;
 }
 
+// Rows of one Phase-1 call over hosts [h0, h1) and the rows of its rotated
+// Q / K: by position (identity, rows 0 .. h1 * block) or, when that reads
+// fewer rows, compact: [sink || Sigma_0 .. Sigma_{h1-2} || blocks h0 .. h1-1]
+// (Star: [B_0 || blocks h0 .. h1-1]).
+struct RangePlan {
+  int64_t rows;      // packed output rows of the range
+  int64_t qk_rows;   // rows of Qr / Kr
+  int compact;
+  int64_t ci_blk;    // Qr / Kr row of the range's first block row
+};
+
+RangePlan plan_range(const int64_t* off_all, int32_t block, int32_t sink, int64_t summ, int star, int h0,
+                     int h1) {
+  RangePlan r;
+  r.rows = off_all[h1] - off_all[h0];
+  r.qk_rows = (int64_t)h1 * block;
+  r.compact = 0;
+  r.ci_blk = (int64_t)h0 * block;
+  if (h1 >= 2 && h1 > h0) {
+    const int64_t pre = star ? (int64_t)block : (int64_t)sink + (int64_t)(h1 - 1) * summ;
+    const int64_t c = pre + (int64_t)(h1 - h0) * block;
+    if (c < r.qk_rows) {
+      r.qk_rows = c;
+      r.compact = 1;
+      r.ci_blk = pre;
+    }
+  }
+  return r;
+}
+
 int check_heads(int32_t hq, int32_t hkv, int32_t d, int dtype) {
   if (hq <= 0 || hkv <= 0 || hq % hkv != 0) return PA_ERR_INVALID;
   if (d != 64 && d != 128) return PA_ERR_UNSUPPORTED;
@@ -104,7 +134,12 @@ int phase1_common(const void* q, const void* k, const void* v, int dtype, int64_
     ht.tile_off[i + 1] = ht.tile_off[i] + (int32_t)((ni + 127) / 128);
   }
   const int64_t R = ht.row_off[n];
-  const size_t need = phase1_workspace_bytes(L, hq, hkv, d, dtype, off_all[n_all]);
+  const RangePlan plan = plan_range(off_all, block, ht.sink, (int64_t)ht.k_chunks * ht.chunk, star,
+                                    host_begin, host_end);
+  ht.compact = plan.compact;
+  ht.ci_blk = plan.ci_blk;
+  const size_t need =
+      phase1_workspace_bytes(plan.qk_rows, hq, hkv, d, dtype, R, plan.compact ? plan.qk_rows : 0);
   rc = check_ws(ws, ws_bytes, need);
   if (rc) return rc;
   rc = clear_status(ws, s);
@@ -116,7 +151,8 @@ int phase1_common(const void* q, const void* k, const void* v, int dtype, int64_
   a.rope_theta = rope_theta;
   a.sel = sel;
   a.ht = ht;
-  a.rope_L = (int64_t)host_end * block;
+  a.qk_rows = plan.qk_rows;
+  a.kret_lo = plan.ci_blk;
   a.ret_lo = (int64_t)host_begin * block;
   a.ret_hi = (int64_t)host_end * block;
   a.o = o; a.lse = lse_opt; a.k_ret = k_ret; a.v_ret = v_ret;
@@ -125,9 +161,13 @@ int phase1_common(const void* q, const void* k, const void* v, int dtype, int64_
   size_t off = kStatusBytes;
   a.rowpos = reinterpret_cast<int32_t*>(w + off);
   off += align_up(sizeof(int32_t) * (size_t)R);
+  a.rowci = plan.compact ? reinterpret_cast<int32_t*>(w + off) : a.rowpos;
+  off += align_up(sizeof(int32_t) * (size_t)R);
+  a.posmap = plan.compact ? reinterpret_cast<int32_t*>(w + off) : nullptr;
+  off += align_up(sizeof(int32_t) * (size_t)(plan.compact ? plan.qk_rows : 0));
   const size_t qk_elem = dtype == PA_BF16 ? 2 : 4;
   a.qr = w + off;
-  off += align_up(qk_elem * (size_t)L * hq * d);
+  off += align_up(qk_elem * (size_t)plan.qk_rows * hq * d);
   a.kr = w + off;
   if (n == 0) return PA_OK;
   a.wait_limit_ns = wait_limit_ns;
@@ -279,7 +319,22 @@ size_t pa_phase1_workspace_size(int64_t L, int32_t hq, int32_t hkv, int32_t d, i
   int64_t off[kMaxBlocks + 1];
   int n = 0;
   if (layout(L, block, star ? 0 : sink, star ? 0 : summary_tokens, star, off, &n)) return 0;
-  return phase1_workspace_bytes(L, hq, hkv, d, dtype, off[n]);
+  // enough for the call over every host and for any host range (a compact
+  // range has fewer than L rotated rows)
+  return phase1_workspace_bytes(L, hq, hkv, d, dtype, off[n], L);
+}
+
+size_t pa_phase1_hosts_workspace_size(int64_t L, int32_t hq, int32_t hkv, int32_t d, int dtype,
+                                      int32_t block, int32_t sink, int32_t summary_tokens, int star,
+                                      int32_t host_begin, int32_t host_end) {
+  if (check_heads(hq, hkv, d, dtype)) return 0;
+  int64_t off[kMaxBlocks + 1];
+  int n = 0;
+  if (star) sink = summary_tokens = 0;
+  if (layout(L, block, sink, summary_tokens, star, off, &n)) return 0;
+  if (host_begin < 0 || host_begin > host_end || host_end > n) return 0;
+  const RangePlan plan = plan_range(off, block, sink, summary_tokens, star, host_begin, host_end);
+  return phase1_workspace_bytes(plan.qk_rows, hq, hkv, d, dtype, plan.rows, plan.compact ? plan.qk_rows : 0);
 }
 
 int pulsar_phase1_encode(const void* q, const void* k, const void* v, int dtype, int64_t L,

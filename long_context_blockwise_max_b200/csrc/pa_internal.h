@@ -56,6 +56,12 @@ struct HostTable {
   int32_t block, sink, chunk, k_chunks;
   int64_t row_off[kMaxBlocks + 1];   // packed output row offsets
   int32_t tile_off[kMaxBlocks + 1];  // cumulative 128-row tiles per host
+  // Rotated Q / K rows: by position (compact == 0), or, for a host range
+  // that reads few positions, in the compact order [sink || Sigma_0 ..
+  // Sigma_{host_end-2} || the range's blocks] (Star: [B_0 || the range's
+  // blocks]), the blocks starting at compact row ci_blk.
+  int32_t compact;
+  int64_t ci_blk;
 };
 
 struct Phase1Args {
@@ -70,12 +76,15 @@ struct Phase1Args {
   float* lse;                   // [R][hq] or null
   void *k_ret, *v_ret;          // [L][hkv][d]
   // workspace carve
-  int32_t* rowpos;              // [R] original position of every packed row
-  void* qr;                     // [L][hq][d] rotated, scaled Q (fp16 or fp32)
-  void* kr;                     // [L][hkv][d] rotated K in the QK type (fp16 or fp32)
-  // positions [0, rope_L) are rotated; k_ret / v_ret hold positions
+  int32_t* rowpos;              // [R] original position of every packed row (V rows)
+  int32_t* rowci;               // [R] row of Qr / Kr of every packed row (== rowpos unless compact)
+  int32_t* posmap;              // [qk_rows] original position of each Qr / Kr row, or null (identity)
+  void* qr;                     // [qk_rows][hq][d] rotated, scaled Q (fp16 or fp32)
+  void* kr;                     // [qk_rows][hkv][d] rotated K in the QK type (fp16 or fp32)
+  // Qr / Kr rows [0, qk_rows) are rotated; k_ret receives Qr/Kr rows
+  // [kret_lo, kret_lo + ret_hi - ret_lo); k_ret / v_ret hold positions
   // [ret_lo, ret_hi) (the blocks of the table's hosts)
-  int64_t rope_L = 0, ret_lo = 0, ret_hi = 0;
+  int64_t qk_rows = 0, kret_lo = 0, ret_lo = 0, ret_hi = 0;
   DeviceStatus* status;
   // bounded-wait limit of the tensor-core kernel and a test-only stall
   uint64_t wait_limit_ns = 1000000000ull;
@@ -83,8 +92,10 @@ struct Phase1Args {
 };
 bool phase1_tc_supported(const Phase1Args& a);
 int launch_phase1_tc(const Phase1Args& a, cudaStream_t s);
-size_t phase1_workspace_bytes(int64_t L, int32_t hq, int32_t hkv, int32_t d, int dtype,
-                              int64_t total_rows);
+// Scratch of one Phase-1 call: status, rowpos and rowci [rows], posmap
+// [posmap_rows], Qr / Kr [qk_rows].
+size_t phase1_workspace_bytes(int64_t qk_rows, int32_t hq, int32_t hkv, int32_t d, int dtype,
+                              int64_t rows, int64_t posmap_rows);
 int launch_phase1(const Phase1Args& a, cudaStream_t s);
 
 struct Phase2Args {

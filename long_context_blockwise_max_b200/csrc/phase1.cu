@@ -9,7 +9,17 @@
 // nothing is copied per host, and the retained cache (B_i's rotated K and V
 // for every host) is simply the whole sequence's rotated K and V.
 //
-//  rowpos_kernel     : packed row -> original position for every host.
+// A call over a range of hosts that reads few of the sequence's positions
+// (the later hosts of a sequence spread over GPUs) rotates only those: its
+// Qr / Kr rows are [sink || Sigma_0 .. Sigma_{host_end-2} || the range's
+// blocks] (Star: [B_0 || the range's blocks]), so its RoPE work and
+// workspace scale with the positions it reads, not with L.  Every host's
+// prefix rows are the first rows of that order, so a prefix row's Qr / Kr
+// row is its row index within the host.
+//
+//  rowpos_kernel     : packed row -> original position (V rows) and -> Qr /
+//                      Kr row (the same unless compact).
+//  posmap_kernel     : compact Qr / Kr row -> original position.
 //  rope_qk_kernel    : Q -> Qr (scaled by log2(e)/sqrt(d)), K -> Kr (QK
 //                      operand type) and k_ret (input dtype).
 //  phase1_simt_kernel: causal attention over a host's rows, fp32 SIMT with an
@@ -20,7 +30,8 @@
 namespace pa {
 
 __global__ void rowpos_kernel(HostTable ht, const int32_t* __restrict__ sel,
-                              int32_t* __restrict__ rowpos, DeviceStatus* st) {
+                              int32_t* __restrict__ rowpos, int32_t* __restrict__ rowci,
+                              DeviceStatus* st) {
   const int64_t R = ht.row_off[ht.n_hosts];
   const int64_t summ = (int64_t)ht.k_chunks * ht.chunk;
   const int C = ht.chunk > 0 ? ht.block / ht.chunk : 0;
@@ -31,6 +42,8 @@ __global__ void rowpos_kernel(HostTable ht, const int32_t* __restrict__ sel,
     const int64_t u = r - ht.row_off[li];
     const int i = ht.host0 + li;                     // the host's index in the sequence
     int64_t p;
+    // own-block rows start at row `pre` of the host
+    const int64_t pre = i == 0 ? 0 : (ht.star ? ht.block : ht.sink + (int64_t)i * summ);
     if (i == 0) {
       p = u;                                         // host 0: B_0 alone
     } else if (ht.star) {
@@ -51,6 +64,38 @@ __global__ void rowpos_kernel(HostTable ht, const int32_t* __restrict__ sel,
       p = (int64_t)i * ht.block + (u - ht.sink - (int64_t)i * summ);   // B_i
     }
     rowpos[r] = (int32_t)p;
+    if (rowci != rowpos) {
+      const int64_t ci = u < pre ? u : ht.ci_blk + (int64_t)(i - ht.host0) * ht.block + (u - pre);
+      rowci[r] = (int32_t)ci;
+    }
+  }
+}
+
+// Compact Qr / Kr row -> original position (the inverse of rowci over one
+// copy of every position the range reads).
+__global__ void posmap_kernel(HostTable ht, int64_t n, const int32_t* __restrict__ sel,
+                              int32_t* __restrict__ posmap, DeviceStatus* st) {
+  const int64_t summ = (int64_t)ht.k_chunks * ht.chunk;
+  const int C = ht.chunk > 0 ? ht.block / ht.chunk : 0;
+  for (int64_t ci = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; ci < n;
+       ci += (int64_t)gridDim.x * blockDim.x) {
+    int64_t p;
+    if (ci >= ht.ci_blk) {
+      p = (int64_t)ht.host0 * ht.block + (ci - ht.ci_blk);           // the range's blocks
+    } else if (ht.star || ci < ht.sink) {
+      p = ci;                                                        // B_0 anchor / sink
+    } else {
+      const int64_t w = ci - ht.sink;                                // Sigma_j, chunk m, token t
+      const int64_t j = w / summ, x = w % summ;
+      const int m = (int)(x / ht.chunk), t = (int)(x % ht.chunk);
+      int c = sel[j * ht.k_chunks + m];
+      if (c < 0 || c >= C) {
+        set_status(st, PA_ERR_INVALID, (int)(j * ht.k_chunks + m), c);
+        c = 0;
+      }
+      p = j * ht.block + (int64_t)c * ht.chunk + t;
+    }
+    posmap[ci] = (int32_t)p;
   }
 }
 
@@ -64,19 +109,27 @@ struct alignas(16) Vec {
   T v[N];
 };
 
+// Row ci of Qr / Kr holds position posmap[ci] (ci itself when posmap is
+// null); Kr rows [kret_lo, kret_lo + kret_n) are also written to k_ret.
 template <typename IT, typename QT, int POS>
 __global__ void __launch_bounds__(256) rope_qk_kernel(
-    const IT* __restrict__ q, const IT* __restrict__ k, int64_t L, int hq, int hkv, int d,
-    RopeFreqs f, float qscale, QT* __restrict__ qr, QT* __restrict__ kr, IT* __restrict__ k_ret,
-    int64_t ret_lo, int64_t ret_hi, DeviceStatus* st) {
+    const IT* __restrict__ q, const IT* __restrict__ k, int64_t n_rows, const int32_t* __restrict__ posmap,
+    int hq, int hkv, int d, RopeFreqs f, float qscale, QT* __restrict__ qr, QT* __restrict__ kr,
+    IT* __restrict__ k_ret, int64_t kret_lo, int64_t kret_n, DeviceStatus* st) {
   constexpr int VEC = 16 / sizeof(IT);          // input elements per 16-byte vector
   __shared__ float2 cs[POS][kMaxHalfDim];
+  __shared__ int64_t spos[POS];
   const int half = d / 2;
-  const int64_t p0 = (int64_t)blockIdx.x * POS;
+  const int64_t ci0 = (int64_t)blockIdx.x * POS;
+  if (threadIdx.x < POS) {
+    const int64_t ci = ci0 + threadIdx.x;
+    spos[threadIdx.x] = ci < n_rows ? (posmap != nullptr ? (int64_t)posmap[ci] : ci) : 0;
+  }
+  __syncthreads();
   for (int e = threadIdx.x; e < POS * half; e += blockDim.x) {
     const int pp = e / half, m = e % half;
     double sn, cn;
-    sincos((double)(p0 + pp) * f.omega[m], &sn, &cn);
+    sincos((double)spos[pp] * f.omega[m], &sn, &cn);
     cs[pp][m] = make_float2((float)cn, (float)sn);
   }
   __syncthreads();
@@ -85,13 +138,16 @@ __global__ void __launch_bounds__(256) rope_qk_kernel(
   bool bad = false;
   for (int e = threadIdx.x; e < POS * per_pos; e += blockDim.x) {
     const int pp = e / per_pos;
-    const int64_t p = p0 + pp;
-    if (p >= L) continue;
+    const int64_t ci = ci0 + pp;
+    if (ci >= n_rows) continue;
+    const int64_t p = spos[pp];
     const int w = e % per_pos;
     const int row = w / vpr, m0 = (w % vpr) * VEC;
     const bool is_q = row < hq;
     const int h = is_q ? row : row - hq;
-    const int64_t base = (p * (is_q ? hq : hkv) + h) * (int64_t)d;
+    const int nh = is_q ? hq : hkv;
+    const int64_t base = (p * nh + h) * (int64_t)d;        // input row (position p)
+    const int64_t obase = (ci * nh + h) * (int64_t)d;      // output row ci
     const IT* src = is_q ? q : k;
     const Vec<IT, VEC> a = *reinterpret_cast<const Vec<IT, VEC>*>(src + base + m0);
     const Vec<IT, VEC> b = *reinterpret_cast<const Vec<IT, VEC>*>(src + base + m0 + half);
@@ -112,17 +168,17 @@ __global__ void __launch_bounds__(256) rope_qk_kernel(
         o1.v[i] = from_f32<QT>(u1);
         o2.v[i] = from_f32<QT>(u2);
       }
-      *reinterpret_cast<Vec<QT, VEC>*>(qr + base + m0) = o1;
-      *reinterpret_cast<Vec<QT, VEC>*>(qr + base + m0 + half) = o2;
+      *reinterpret_cast<Vec<QT, VEC>*>(qr + obase + m0) = o1;
+      *reinterpret_cast<Vec<QT, VEC>*>(qr + obase + m0 + half) = o2;
     } else {
-      if (p >= ret_lo && p < ret_hi) {   // retained: the blocks of the encoded hosts
+      if (ci >= kret_lo && ci < kret_lo + kret_n) {   // retained: the blocks of the encoded hosts
         Vec<IT, VEC> r1, r2;
 #pragma unroll
         for (int i = 0; i < VEC; ++i) {
           r1.v[i] = from_f32<IT>(y1[i]);
           r2.v[i] = from_f32<IT>(y2[i]);
         }
-        const int64_t rb = base - ret_lo * hkv * (int64_t)d;
+        const int64_t rb = obase - kret_lo * hkv * (int64_t)d;
         *reinterpret_cast<Vec<IT, VEC>*>(k_ret + rb + m0) = r1;
         *reinterpret_cast<Vec<IT, VEC>*>(k_ret + rb + m0 + half) = r2;
       }
@@ -134,8 +190,8 @@ __global__ void __launch_bounds__(256) rope_qk_kernel(
           o1.v[i] = from_f32<QT>(y1[i]);
           o2.v[i] = from_f32<QT>(y2[i]);
         }
-        *reinterpret_cast<Vec<QT, VEC>*>(kr + base + m0) = o1;
-        *reinterpret_cast<Vec<QT, VEC>*>(kr + base + m0 + half) = o2;
+        *reinterpret_cast<Vec<QT, VEC>*>(kr + obase + m0) = o1;
+        *reinterpret_cast<Vec<QT, VEC>*>(kr + obase + m0 + half) = o2;
       }
     }
   }
@@ -150,8 +206,8 @@ __global__ void __launch_bounds__(256) rope_qk_kernel(
 template <int D, typename QT, typename VT, typename OT>
 __global__ void __launch_bounds__(256) phase1_simt_kernel(
     const QT* __restrict__ qr, const QT* __restrict__ kr, const VT* __restrict__ v,
-    const int32_t* __restrict__ rowpos, HostTable ht, int hq, int hkv, OT* __restrict__ o,
-    float* __restrict__ lse) {
+    const int32_t* __restrict__ rowpos, const int32_t* __restrict__ rowci, HostTable ht, int hq, int hkv,
+    OT* __restrict__ o, float* __restrict__ lse) {
   constexpr int BK = 32, HALF = D / 2, G4 = HALF / 4;
   __shared__ __align__(16) float ks[BK][D];
   __shared__ __align__(16) float vs[BK][D];
@@ -167,7 +223,7 @@ __global__ void __launch_bounds__(256) phase1_simt_kernel(
   // element index of group g, lane-half hf: 8*g + 4*hf + {0..3}
   float qv[HALF], acc[HALF];
   if (active) {
-    const int64_t pq = rowpos[row0 + r];
+    const int64_t pq = rowci[row0 + r];
     const QT* src = qr + (pq * hq + h) * (int64_t)D;
 #pragma unroll
     for (int g = 0; g < G4; ++g)
@@ -187,10 +243,9 @@ __global__ void __launch_bounds__(256) phase1_simt_kernel(
       const int kk = idx / D, mm = idx % D, c = c0 + kk;
       float kx = 0.f, vx = 0.f;
       if (c < n) {
-        const int64_t pk = rowpos[row0 + c];
-        const int64_t off = (pk * hkv + kvh) * (int64_t)D + mm;
-        kx = to_f32(kr[off]);
-        vx = to_f32(v[off]);
+        const int64_t ck = rowci[row0 + c], pv = rowpos[row0 + c];
+        kx = to_f32(kr[(ck * hkv + kvh) * (int64_t)D + mm]);
+        vx = to_f32(v[(pv * hkv + kvh) * (int64_t)D + mm]);
       }
       ks[kk][mm] = kx;
       vs[kk][mm] = vx;
@@ -243,13 +298,14 @@ __global__ void __launch_bounds__(256) phase1_simt_kernel(
   if (lse != nullptr && hf == 0) lse[(row0 + r) * hq + h] = (m_run + __log2f(l_run)) * kLn2f;
 }
 
-size_t phase1_workspace_bytes(int64_t L, int32_t hq, int32_t hkv, int32_t d, int dtype,
-                              int64_t total_rows) {
+size_t phase1_workspace_bytes(int64_t qk_rows, int32_t hq, int32_t hkv, int32_t d, int dtype,
+                              int64_t rows, int64_t posmap_rows) {
   const size_t qk_elem = dtype == PA_BF16 ? 2 : 4;
   size_t b = kStatusBytes;
-  b += align_up(sizeof(int32_t) * (size_t)total_rows);
-  b += align_up(qk_elem * (size_t)L * hq * d);
-  b += align_up(qk_elem * (size_t)L * hkv * d);
+  b += 2 * align_up(sizeof(int32_t) * (size_t)rows);
+  b += align_up(sizeof(int32_t) * (size_t)posmap_rows);
+  b += align_up(qk_elem * (size_t)qk_rows * hq * d);
+  b += align_up(qk_elem * (size_t)qk_rows * hkv * d);
   return b;
 }
 
@@ -259,19 +315,24 @@ static int launch_phase1_t(const Phase1Args& a, cudaStream_t s) {
   {
     const int threads = 256;
     const int64_t want = (R + threads - 1) / threads;
-    rowpos_kernel<<<(int)(want < 148 * 8 ? want : 148 * 8), threads, 0, s>>>(a.ht, a.sel,
-                                                                             a.rowpos, a.status);
+    rowpos_kernel<<<(int)(want < 148 * 8 ? want : 148 * 8), threads, 0, s>>>(a.ht, a.sel, a.rowpos, a.rowci,
+                                                                             a.status);
+    if (a.posmap != nullptr && a.qk_rows > 0) {
+      const int64_t wp = (a.qk_rows + threads - 1) / threads;
+      posmap_kernel<<<(int)(wp < 148 * 8 ? wp : 148 * 8), threads, 0, s>>>(a.ht, a.qk_rows, a.sel, a.posmap,
+                                                                          a.status);
+    }
   }
   RopeFreqs f;
   for (int m = 0; m < kMaxHalfDim; ++m)
     f.omega[m] = (m < a.d / 2) ? pow(a.rope_theta, -2.0 * m / a.d) : 0.0;
   const float qscale = (float)(kLog2e / sqrt((double)a.d));
   constexpr int POS = 8;
-  if (a.rope_L > 0) {
-    rope_qk_kernel<IT, QT, POS><<<(unsigned)((a.rope_L + POS - 1) / POS), 256, 0, s>>>(
-        static_cast<const IT*>(a.q), static_cast<const IT*>(a.k), a.rope_L, a.hq, a.hkv, a.d, f,
-        qscale, static_cast<QT*>(a.qr), static_cast<QT*>(a.kr), static_cast<IT*>(a.k_ret), a.ret_lo,
-        a.ret_hi, a.status);
+  if (a.qk_rows > 0) {
+    rope_qk_kernel<IT, QT, POS><<<(unsigned)((a.qk_rows + POS - 1) / POS), 256, 0, s>>>(
+        static_cast<const IT*>(a.q), static_cast<const IT*>(a.k), a.qk_rows, a.posmap, a.hq, a.hkv, a.d, f,
+        qscale, static_cast<QT*>(a.qr), static_cast<QT*>(a.kr), static_cast<IT*>(a.k_ret), a.kret_lo,
+        a.ret_hi - a.ret_lo, a.status);
   }
   const size_t vrow = sizeof(IT) * (size_t)a.hkv * a.d;
   if (a.ret_hi > a.ret_lo) {
@@ -290,12 +351,12 @@ static int launch_phase1_t(const Phase1Args& a, cudaStream_t s) {
   } else if (grid.x > 0) {
     if (a.d == 128)
       phase1_simt_kernel<128, QT, VT, OT><<<grid, 256, 0, s>>>(
-          static_cast<const QT*>(a.qr), kq, static_cast<const VT*>(a.v), a.rowpos, a.ht, a.hq,
-          a.hkv, static_cast<OT*>(a.o), a.lse);
+          static_cast<const QT*>(a.qr), kq, static_cast<const VT*>(a.v), a.rowpos, a.rowci, a.ht,
+          a.hq, a.hkv, static_cast<OT*>(a.o), a.lse);
     else
       phase1_simt_kernel<64, QT, VT, OT><<<grid, 256, 0, s>>>(
-          static_cast<const QT*>(a.qr), kq, static_cast<const VT*>(a.v), a.rowpos, a.ht, a.hq,
-          a.hkv, static_cast<OT*>(a.o), a.lse);
+          static_cast<const QT*>(a.qr), kq, static_cast<const VT*>(a.v), a.rowpos, a.rowci, a.ht,
+          a.hq, a.hkv, static_cast<OT*>(a.o), a.lse);
   }
   profile_end(s);
   if (rc != PA_OK) return rc;

@@ -65,7 +65,8 @@ struct TcBars {
 
 struct TcParams {
   HostTable ht;
-  const int32_t* rowpos;
+  const int32_t* rowpos;   // packed row -> position (V)
+  const int32_t* rowci;    // packed row -> row of Qr / Kr
   __nv_bfloat16* o;
   float* lse;
   int hq, hkv, pairs;   // pairs = (hq / hkv) / 2 head pairs per kv head
@@ -169,9 +170,10 @@ __global__ void __launch_bounds__(384, 1) phase1_tc_kernel(const __grid_constant
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       auto pos_of = [&](int r) -> int { return p.rowpos[row0 + (r < n ? r : 0)]; };
+      auto ci_of = [&](int r) -> int { return p.rowci[row0 + (r < n ? r : 0)]; };
       mbar_arrive_expect_tx(&bars->q_full, 2 * C::TILE_BYTES + (p.stall ? 16 : 0));
       for (int grp = 0; grp < 8; ++grp) {
-        const int pq = pos_of(r0 + 16 * grp);
+        const int pq = ci_of(r0 + 16 * grp);
         for (int t = 0; t < 2; ++t)
           for (int kb = 0; kb < C::NKB; ++kb)
             tma_load_3d(sQ + t * C::TILE_BYTES + kb * C::KB_BYTES + grp * 2048, &tmQ, &bars->q_full,
@@ -181,14 +183,17 @@ __global__ void __launch_bounds__(384, 1) phase1_tc_kernel(const __grid_constant
       for (int j = 0; j < nkv; ++j) {
         const int st = j & 1;
         const uint32_t ph = (j >> 1) & 1;
-        int pk[8];
-        for (int grp = 0; grp < 8; ++grp) pk[grp] = pos_of(j * 128 + 16 * grp);
+        int pk[8], ck[8];
+        for (int grp = 0; grp < 8; ++grp) {
+          pk[grp] = pos_of(j * 128 + 16 * grp);
+          ck[grp] = ci_of(j * 128 + 16 * grp);
+        }
         if (!mbar_wait(&bars->k_empty[st], ph ^ 1, abort, p.wait_ns, gabort)) { fail(1); break; }
         mbar_arrive_expect_tx(&bars->k_full[st], C::TILE_BYTES);
         for (int grp = 0; grp < 8; ++grp)
           for (int kb = 0; kb < C::NKB; ++kb)
             tma_load_3d(sK + st * C::TILE_BYTES + kb * C::KB_BYTES + grp * 2048, &tmK, &bars->k_full[st],
-                        kb * 64, kvh, pk[grp]);
+                        kb * 64, kvh, ck[grp]);
         ++armed_k[st];
         if (!mbar_wait(&bars->v_empty[st], ph ^ 1, abort, p.wait_ns, gabort)) { fail(2); break; }
         mbar_arrive_expect_tx(&bars->v_full[st], C::TILE_BYTES);
@@ -399,13 +404,14 @@ template <int D>
 int launch_tc(const Phase1Args& a, cudaStream_t s) {
   using C = TcCfg<D>;
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, a.qr, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.L, a.hq, D) ||
-      !make_map(&mk, a.kr, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.L, a.hkv, D) ||
+  if (!make_map(&mq, a.qr, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.qk_rows, a.hq, D) ||
+      !make_map(&mk, a.kr, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.qk_rows, a.hkv, D) ||
       !make_map(&mv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.L, a.hkv, D))
     return PA_ERR_CUDA;
   TcParams p;
   p.ht = a.ht;
   p.rowpos = a.rowpos;
+  p.rowci = a.rowci;
   p.o = static_cast<__nv_bfloat16*>(a.o);
   p.lse = a.lse;
   p.hq = a.hq;

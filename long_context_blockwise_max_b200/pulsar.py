@@ -26,7 +26,8 @@ ABI_SYMBOLS = (
     "pa_abi_version", "pa_status_string", "pa_workspace_status", "pa_set_profile_events",
     "pa_select_workspace_size", "pulsar_select_summaries", "pulsar_select_summaries_noalloc",
     "pulsar_select_summaries_scored",
-    "pa_phase1_layout", "pa_phase1_workspace_size", "pulsar_phase1_encode", "star_phase1_encode",
+    "pa_phase1_layout", "pa_phase1_workspace_size", "pa_phase1_hosts_workspace_size",
+    "pulsar_phase1_encode", "star_phase1_encode",
     "pulsar_phase1_encode_hosts", "star_phase1_encode_hosts",
     "pa_phase2_workspace_size", "star_phase2_attend", "star_phase2_query_step", "pa_lse_merge",
     "star_phase2_attend_art",
@@ -58,6 +59,8 @@ def _load() -> ctypes.CDLL:
                                                           P]),
         "pa_phase1_layout": (ctypes.c_int, [I64, I32, I32, I32, ctypes.c_int, P]),
         "pa_phase1_workspace_size": (SZ, [I64, I32, I32, I32, ctypes.c_int, I32, I32, I32, ctypes.c_int]),
+        "pa_phase1_hosts_workspace_size": (SZ, [I64, I32, I32, I32, ctypes.c_int, I32, I32, I32, ctypes.c_int,
+                                                I32, I32]),
         "pulsar_phase1_encode": (ctypes.c_int, [P, P, P, ctypes.c_int, I64, I32, I32, I32, D, I32, I32, I32,
                                                 I32, P, P, P, P, P, P, SZ, P]),
         "star_phase1_encode": (ctypes.c_int, [P, P, P, ctypes.c_int, I64, I32, I32, I32, D, I32, P, P, P, P,
@@ -245,6 +248,12 @@ def pa_phase1_workspace_size(L, hq, hkv, d, dtype, block, sink, summary_tokens, 
     return _lib.pa_phase1_workspace_size(L, hq, hkv, d, dtype, block, sink, summary_tokens, int(star))
 
 
+def pa_phase1_hosts_workspace_size(L, hq, hkv, d, dtype, block, sink, summary_tokens, star, host_begin,
+                                   host_end) -> int:
+    return _lib.pa_phase1_hosts_workspace_size(L, hq, hkv, d, dtype, block, sink, summary_tokens, int(star),
+                                               host_begin, host_end)
+
+
 def _phase1_check(q, k, v, rows, ret_rows, o, lse, k_ret, v_ret, sel=None, n_sel=0):
     """Inputs [L][h][d] of one dtype (K and V alike); caller-supplied outputs
     large enough for ``rows`` output rows and ``ret_rows`` retained rows."""
@@ -345,7 +354,8 @@ def pulsar_phase1_encode_hosts(q, k, v, rope_theta, block, sink, chunk, k_chunks
                   (L // block if block > 0 else 0) * k_chunks)
     o, lse, k_ret, v_ret = _phase1_range_outputs(q, k, block, row_off[-1] if row_off else 0, nh, o, lse, k_ret,
                                                  v_ret, want_lse)
-    need = pa_phase1_workspace_size(L, hq, hkv, d, dt, block, sink, k_chunks * chunk, False)
+    need = pa_phase1_hosts_workspace_size(L, hq, hkv, d, dt, block, sink, k_chunks * chunk, False, host_begin,
+                                          host_end)
     ws = _workspace(need, q.device, ws)
     rc = _lib.pulsar_phase1_encode_hosts(_ptr(q), _ptr(k), _ptr(v), dt, L, hq, hkv, d, float(rope_theta), block,
                                          sink, chunk, k_chunks, _ptr(sel), host_begin, host_end, _ptr(o), _ptr(lse),
@@ -368,7 +378,7 @@ def star_phase1_encode_hosts(q, k, v, rope_theta, block, host_begin, host_end, o
     _phase1_check(q, k, v, row_off[-1] if row_off else 0, nh * block, o, lse, k_ret, v_ret)
     o, lse, k_ret, v_ret = _phase1_range_outputs(q, k, block, row_off[-1] if row_off else 0, nh, o, lse, k_ret,
                                                  v_ret, want_lse)
-    need = pa_phase1_workspace_size(L, hq, hkv, d, dt, block, 0, 0, True)
+    need = pa_phase1_hosts_workspace_size(L, hq, hkv, d, dt, block, 0, 0, True, host_begin, host_end)
     ws = _workspace(need, q.device, ws)
     rc = _lib.star_phase1_encode_hosts(_ptr(q), _ptr(k), _ptr(v), dt, L, hq, hkv, d, float(rope_theta), block,
                                        host_begin, host_end, _ptr(o), _ptr(lse), _ptr(k_ret), _ptr(v_ret), _ptr(ws),

@@ -30,7 +30,7 @@ def _header_functions():
 
 def test_library_exports_every_declared_symbol(lib):
     names = _header_functions()
-    assert len(names) == 19
+    assert len(names) == 20
     assert sorted(lib.ABI_SYMBOLS) == names
     so = ctypes.CDLL(lib.LIB_PATH)
     for n in names:
@@ -55,6 +55,38 @@ def test_workspace_sizes(lib):
     assert lib.pa_phase1_workspace_size(2048, 4, 2, 96, 0, 512, 64, 64, False) == 0
     assert lib.pa_phase2_workspace_size(16, 1, 131072, 8, 32, 8, 128) > 0
     assert lib.pa_phase2_workspace_size(16, 1, 131072, 0, 32, 8, 128) == 0
+
+
+def _align(x):
+    return -(-x // 256) * 256
+
+
+def test_host_range_workspace_scales_with_the_positions_it_reads(lib):
+    # 128K Llama-3.1-8B shape, bf16: one GPU per host.  A range rotates the
+    # positions its hosts read -- the sink, the summaries of the blocks before
+    # its last host, its own blocks (Star: B_0 and its own blocks) -- not the
+    # whole prefix of the sequence.
+    L, b, sink, summ, hq, hkv, d = 131072, 16384, 64, 2048, 32, 8, 128
+    row = 2 * (hq + hkv) * d                      # fp16 Qr + Kr bytes per rotated row
+    full = lib.pa_phase1_workspace_size(L, hq, hkv, d, 1, b, sink, summ, False)
+    for h in range(8):
+        rows = b if h == 0 else sink + h * summ + b
+        want_rows = b if h == 0 else sink + h * summ + b     # host 0 reads B_0 only
+        got = lib.pa_phase1_hosts_workspace_size(L, hq, hkv, d, 1, b, sink, summ, False, h, h + 1)
+        posmap = 0 if h == 0 else _align(4 * want_rows)
+        want = 256 + 2 * _align(4 * rows) + posmap + _align(2 * want_rows * hq * d) + _align(2 * want_rows * hkv * d)
+        assert got == want, (h, got, want)
+        assert got <= full
+    last = lib.pa_phase1_hosts_workspace_size(L, hq, hkv, d, 1, b, sink, summ, False, 7, 8)
+    assert last * 4 < full and 30784 * row < last
+    # all hosts: every position once, by position
+    assert lib.pa_phase1_hosts_workspace_size(L, hq, hkv, d, 1, b, sink, summ, False, 0, 8) <= full
+    # Star, the last host: [B_0 || B_7]
+    star_last = lib.pa_phase1_hosts_workspace_size(L, hq, hkv, d, 1, b, 0, 0, True, 7, 8)
+    assert star_last == 256 + 2 * _align(4 * 2 * b) + _align(4 * 2 * b) + _align(2 * 2 * b * hq * d) + \
+        _align(2 * 2 * b * hkv * d)
+    assert lib.pa_phase1_hosts_workspace_size(L, hq, hkv, d, 1, b, sink, summ, False, 5, 9) == 0
+    assert lib.pa_phase1_hosts_workspace_size(L, hq, hkv, d, 1, b, sink, summ, False, 3, 2) == 0
 
 
 def test_host_validation_rejects_before_launch(lib):

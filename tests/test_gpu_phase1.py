@@ -179,13 +179,15 @@ def test_bad_summary_index_sets_status(P):
 
 @pytest.mark.parametrize("star,dtype,splits", [
     (False, torch.bfloat16, [(0, 2), (2, 5), (5, 6), (3, 3)]),   # tensor-core kernel; an empty range
-    (True, torch.bfloat16, [(0, 1), (1, 6)]),
+    (True, torch.bfloat16, [(0, 1), (1, 6), (4, 6)]),            # (4, 6) rotates B_0 and its blocks only
     (False, torch.float32, [(0, 4), (4, 6)]),                    # SIMT kernel
 ])
 def test_host_ranges_equal_full_encode(P, star, dtype, splits):
     # one GPU's share of a sequence's hosts (the multi-GPU layout of the
     # Pulsar page §2.1 / §2.2): the rows and retained blocks of every range
-    # are bit-identical to the same rows of the all-host call
+    # are bit-identical to the same rows of the all-host call.  Ranges that
+    # read few positions ((2, 5), (5, 6), (4, 6)) rotate only those, in the
+    # compact row order, with a smaller workspace.
     L, block, sink, chunk, kc = 6 * 256, 256, 64, 32, 2
     hq, hkv, d = (8, 2, 128) if dtype == torch.bfloat16 else (4, 2, 64)
     q, k, v = _inputs(L, hq, hkv, d, dtype, seed=30)
