@@ -16,8 +16,12 @@ shards (GB/s against HBM).
 
 With N > 1 (torchrun, one process per GPU) every rank encodes its own
 independent sequence (weak scaling, no data-path collective); the time is the
-max over ranks.  `--impl reference` times the fp64 CPU oracle on a bounded
-sample of the same step (rank 0 only).
+max over ranks.  `--layout hosts` runs the method's own multi-GPU layout
+instead: the 8 hosts of ONE sequence spread over the ranks (Phase 1 without
+communication), then the Phase-2 exchange -- every rank's shard partials
+all-gathered over NCCL and merged exactly (strong scaling; on one GPU the
+exchange runs in a process group of one rank).  `--impl reference` times
+the fp64 CPU oracle on a fixed sample of the same step (rank 0 only).
 """
 from __future__ import annotations
 
@@ -154,11 +158,17 @@ class ClockSampler:
 # our implementation
 # --------------------------------------------------------------------------
 class Step:
-    """Preallocated buffers and the calls of one hot-path step."""
+    """Preallocated buffers and the calls of one hot-path step.
 
-    def __init__(self, w, dev, seed_offset=0):
+    ``hosts = (h0, h1, group)`` runs the multi-GPU layout of the method on
+    this rank: Phase 1 of hosts [h0, h1) of the sequence, then the Phase-2
+    exchange (the rank's shard partials, an NCCL all-gather over ``group``,
+    the exact merge)."""
+
+    def __init__(self, w, dev, seed_offset=0, hosts=None):
         from long_context_blockwise_max_b200 import pulsar as P
         self.P, self.w, self.dev = P, w, dev
+        self.hosts = hosts
         ids = w.token_ids()
         if seed_offset:
             ids = np.roll(ids, seed_offset * 4099)
@@ -170,20 +180,27 @@ class Step:
         n = w.n_blocks
         summ = w.k_chunks * w.chunk
         self.row_off = P.pa_phase1_layout(w.L, w.block, w.sink, summ, False)
-        R = self.row_off[-1]
+        h0, h1 = (hosts[0], hosts[1]) if hosts else (0, n)
+        self.h0, self.h1 = h0, h1
+        R = self.row_off[h1] - self.row_off[h0]
         self.sel = torch.empty((n, w.k_chunks), dtype=torch.int32, device=dev)
         self.ws_sel = torch.empty(P.pa_select_workspace_size(w.L, w.vocab, w.block, w.chunk), dtype=torch.uint8,
                                   device=dev)
-        self.o1 = torch.empty((R, w.hq, w.d), dtype=w.dtype, device=dev)
-        self.lse1 = torch.empty((R, w.hq), dtype=torch.float32, device=dev)
-        self.k_ret = torch.empty_like(k)
-        self.v_ret = torch.empty_like(v)
-        self.ws1 = torch.empty(P.pa_phase1_workspace_size(w.L, w.hq, w.hkv, w.d, 1, w.block, w.sink, summ, False),
+        self.o1 = torch.empty((max(R, 1), w.hq, w.d), dtype=w.dtype, device=dev)
+        self.lse1 = torch.empty((max(R, 1), w.hq), dtype=torch.float32, device=dev)
+        nret = (h1 - h0) * w.block
+        self.k_ret = torch.empty((max(nret, 1), w.hkv, w.d), dtype=w.dtype, device=dev)
+        self.v_ret = torch.empty_like(self.k_ret)
+        self.ws1 = torch.empty(max(P.pa_phase1_hosts_workspace_size(w.L, w.hq, w.hkv, w.d, 1, w.block, w.sink, summ,
+                                                                    False, h0, h1), 256),
                                dtype=torch.uint8, device=dev)
         self.o2 = torch.empty_like(self.query)
         self.lse2 = torch.empty((1, w.q_tokens, w.hq), dtype=torch.float32, device=dev)
-        self.ws2 = torch.empty(P.pa_phase2_workspace_size(1, w.q_tokens, w.L, n, w.hq, w.hkv, w.d),
-                               dtype=torch.uint8, device=dev)
+        self.ws2 = torch.empty(P.pa_phase2_workspace_size(1, w.q_tokens, max(nret, 1), max(h1 - h0, 1), w.hq, w.hkv,
+                                                          w.d), dtype=torch.uint8, device=dev)
+        if hosts:
+            self.part_o = torch.empty((1, max(h1 - h0, 1), w.q_tokens, w.hq, w.d), dtype=torch.float32, device=dev)
+            self.part_lse = torch.empty((1, max(h1 - h0, 1), w.q_tokens, w.hq), dtype=torch.float32, device=dev)
         self.attn_events = None
         self.p2_events = None
         self.stage_events = None   # 4 events: before selection, after it, after Phase 1, after Phase 2
@@ -197,20 +214,71 @@ class Step:
         if ev:
             ev[1].record()
         P.pa_set_profile_events(*(self.attn_events or (None, None)))
-        P.pulsar_phase1_encode(self.q, self.k, self.v, w.rope_theta, w.block, w.sink, w.chunk, w.k_chunks,
-                               self.sel, o=self.o1, lse=self.lse1, k_ret=self.k_ret, v_ret=self.v_ret,
-                               ws=self.ws1)
+        if self.hosts:
+            P.pulsar_phase1_encode_hosts(self.q, self.k, self.v, w.rope_theta, w.block, w.sink, w.chunk,
+                                         w.k_chunks, self.sel, self.h0, self.h1, o=self.o1, lse=self.lse1,
+                                         k_ret=self.k_ret, v_ret=self.v_ret, ws=self.ws1)
+        else:
+            P.pulsar_phase1_encode(self.q, self.k, self.v, w.rope_theta, w.block, w.sink, w.chunk, w.k_chunks,
+                                   self.sel, o=self.o1, lse=self.lse1, k_ret=self.k_ret, v_ret=self.v_ret,
+                                   ws=self.ws1)
         if ev:
             ev[2].record()
         P.pa_set_profile_events(*(self.p2_events or (None, None)))
-        P.star_phase2_attend(self.query, self.k_ret[None], self.v_ret[None], w.n_blocks, q_pos0=w.L,
-                             rope_theta=w.rope_theta, o=self.o2, lse=self.lse2, ws=self.ws2)
+        if self.hosts:
+            self._exchange()
+        else:
+            P.star_phase2_attend(self.query, self.k_ret[None], self.v_ret[None], w.n_blocks, q_pos0=w.L,
+                                 rope_theta=w.rope_theta, o=self.o2, lse=self.lse2, ws=self.ws2)
         P.pa_set_profile_events(None, None)
         if ev:
             ev[3].record()
 
-    # kernels of ours launched by one step (selection 3, Phase 1 3, Phase 2 3)
-    LAUNCHES = 9
+    def _exchange(self):
+        """Phase 2 of the multi-GPU layout: this rank's shards' partials, the
+        NCCL all-gather of every rank's partials, the exact merge."""
+        from long_context_blockwise_max_b200 import distributed as D
+        P, w = self.P, self.w
+        n_local = self.h1 - self.h0
+
+        def partials(q, kl, vl, n, q_pos0, theta):
+            P.star_phase2_attend(q, kl, vl, n, q_pos0=q_pos0, rope_theta=theta, o=self.o2, lse=self.lse2,
+                                 want_partials=True, part_o=self.part_o, part_lse=self.part_lse, ws=self.ws2)
+            return self.part_o, self.part_lse
+
+        def merge(all_o, all_lse, dtype):
+            return P.pa_lse_merge(all_o, all_lse, dtype=dtype, o=self.o2, lse=self.lse2)
+        nret = n_local * w.block
+        D.phase2_attend_distributed(self.query, self.k_ret[None, :nret], self.v_ret[None, :nret], n_local,
+                                    w.n_blocks, w.L, w.rope_theta, group=self.hosts[2], partials_fn=partials,
+                                    merge_fn=merge)
+
+    def launches(self):
+        """Kernels of ours one step launches: selection 3 (presence, min df,
+        top-k); Phase 1 3 (row map, RoPE, attention) plus the position map
+        of a compact host range; Phase 2 3 (query RoPE, partials, merge)
+        plus the exchange's merge of the gathered partials."""
+        n = 9
+        if self.hosts:
+            w, h0, h1 = self.w, self.h0, self.h1
+            pre = w.sink + (h1 - 1) * w.k_chunks * w.chunk
+            n += 1 + (1 if h1 >= 2 and pre + (h1 - h0) * w.block < h1 * w.block else 0)
+        return n
+
+    def check_status(self, where):
+        """Device status of the step's three workspaces (selection, Phase 1,
+        Phase 2); a run whose kernels reported an error yields no number."""
+        for name, ws in (("selection", self.ws_sel), ("Phase 1", self.ws1), ("Phase 2", self.ws2)):
+            st = self.P.pa_workspace_status(ws)
+            if st != 0:
+                raise RuntimeError(f"{name} device status {st} ({self.P.status_string(st)}) {where}")
+
+
+def require_ok(P, ws, what):
+    """Raise if a side measurement's kernels reported a device error."""
+    st = P.pa_workspace_status(ws)
+    if st != 0:
+        raise RuntimeError(f"{what}: device status {st} ({P.status_string(st)})")
 
 
 def host_lengths(w, star):
@@ -219,10 +287,14 @@ def host_lengths(w, star):
     return [w.block] + [(2 * w.block if star else w.sink + i * summ + w.block) for i in range(1, n)]
 
 
-def attn_flops(w, star=False):
+def attn_flops(w, star=False, hosts=None):
     """Algorithmic Phase-1 FLOPs: 4 * d * Hq * n(n+1)/2 per host (QK^T and PV
-    over the causal pairs, diagonal included; softmax not counted)."""
-    return float(sum(4.0 * w.d * w.hq * n * (n + 1) / 2.0 for n in host_lengths(w, star)))
+    over the causal pairs, diagonal included; softmax not counted), over all
+    hosts or hosts [h0, h1)."""
+    ns = host_lengths(w, star)
+    if hosts is not None:
+        ns = ns[hosts[0]:hosts[1]]
+    return float(sum(4.0 * w.d * w.hq * n * (n + 1) / 2.0 for n in ns))
 
 
 def sync_all(dist_on, device="cuda"):
@@ -254,12 +326,19 @@ def run_ours(args, rank, world, local_rank, dist_on):
     torch.cuda.set_device(dev)
     w = WORKLOAD
     peaks, peak_kind = load_peaks()
-    step = Step(w, dev, seed_offset=rank)
+    hosts_layout = args.layout == "hosts"
+    if hosts_layout:
+        # one sequence, its hosts spread over the ranks (Phase 1 without
+        # communication, then the Phase-2 all-gather over NCCL)
+        from long_context_blockwise_max_b200.distributed import shard_ranges
+        h0, h1 = shard_ranges(w.n_blocks, world)[rank]
+        step = Step(w, dev, hosts=(h0, h1, torch.distributed.group.WORLD))
+    else:
+        h0, h1 = 0, w.n_blocks
+        step = Step(w, dev, seed_offset=rank)
     for _ in range(args.warmup):
         step.run()
-    st = step.P.pa_workspace_status(step.ws1)
-    if st != 0:
-        raise RuntimeError(f"Phase-1 device status {st}")
+    step.check_status("after warm-up")
 
     # ---- timed region: K steps -----------------------------------------
     K = args.steps
@@ -287,15 +366,18 @@ def run_ours(args, rank, world, local_rank, dist_on):
     step.p2_events = None
     step.stage_events = None
     sync_all(dist_on)
+    step.check_status("after the timed steps")
     ms = max_over_ranks(t0.elapsed_time(t1), dist_on) / K
-    attn_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_attn)
+    # a rank with no host (more ranks than hosts) launches no attention kernel
+    attn_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_attn) if h1 > h0 else float("nan")
     p2_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_p2)
     sel_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev_stage)
     enc_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev_stage)
     p2_call_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in ev_stage)
 
-    flops = attn_flops(w)
-    tokens_per_s = whole_job_rate(w.L, world, ms)
+    flops = attn_flops(w, hosts=(h0, h1))
+    # whole job: one sequence per rank, or one sequence spread over the ranks
+    tokens_per_s = w.L / (ms * 1e-3) if hosts_layout else whole_job_rate(w.L, world, ms)
     peak_tf = peaks["bf16_tflops_sustained"]
     attn_tf = flops / (attn_ms * 1e-3) / 1e12
 
@@ -349,11 +431,13 @@ def run_ours(args, rank, world, local_rank, dist_on):
     sync_all(dist_on)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist_on) / K
     step.ids, step.q, step.k, step.v, step.query = bufs[0]
+    step.check_status("after the end-to-end steps")
+    e2e_rate = w.L / (e2e_ms * 1e-3) if hosts_layout else whole_job_rate(w.L, world, e2e_ms)
 
     # ---- side measurements: Star Phase 1, Phase-2 decode ----------------
     P = step.P
     extra = {}
-    if not args.headline_only:
+    if not args.headline_only and not hosts_layout:
         row_star = P.pa_phase1_layout(w.L, w.block, 0, 0, True)[-1]
         o_star = torch.empty((row_star, w.hq, w.d), dtype=w.dtype, device=dev)
         ws_star = torch.empty(P.pa_phase1_workspace_size(w.L, w.hq, w.hkv, w.d, 1, w.block, 0, 0, True),
@@ -374,6 +458,7 @@ def run_ours(args, rank, world, local_rank, dist_on):
         s1.record()
         torch.cuda.synchronize()
         star_ms = s0.elapsed_time(s1) / reps
+        require_ok(P, ws_star, "Star Phase 1")
         sf = attn_flops(w, star=True)
         extra["star_phase1"] = {"ms": round(star_ms, 3), "tflop": round(sf / 1e12, 3),
                                 "tflop_s": round(sf / (star_ms * 1e-3) / 1e12, 1),
@@ -406,6 +491,7 @@ def run_ours(args, rank, world, local_rank, dist_on):
         d1.record()
         torch.cuda.synchronize()
         dec_ms = d0.elapsed_time(d1) / K
+        require_ok(P, dws, "128K decode")
         dec_kernel_ms = statistics.mean(a.elapsed_time(b) for a, b in pev)
         kv_bytes = 2.0 * B * T * DECODE.hkv * DECODE.d * 2
         extra["phase2_decode"] = {
@@ -433,6 +519,7 @@ def run_ours(args, rank, world, local_rank, dist_on):
         r1.record()
         torch.cuda.synchronize()
         art_ms = r0.elapsed_time(r1) / K
+        require_ok(P, aws, "ART decode")
         frac = float(vis.float().mean().item()) * 128 / T
         extra["phase2_decode_art"] = {"ms": round(art_ms, 4), "visited_fraction": round(frac, 4),
                                       "gb_s_of_visited": round(kv_bytes * frac / (art_ms * 1e-3) / 1e9, 1),
@@ -474,6 +561,8 @@ def run_ours(args, rank, world, local_rank, dist_on):
         art2_ms, (_, _, vis2, _) = timed(art2)
         ex2_ms, _ = timed(exact2)
         frac2 = float(vis2.float().mean().item()) * 128 / T
+        require_ok(P, aws, "ART decode, recency cache")
+        require_ok(P, ews, "exact decode, recency cache")
         extra["phase2_decode_art_recency"] = {
             "ms": round(art2_ms, 4), "exact_ms": round(ex2_ms, 4), "speedup": round(ex2_ms / art2_ms, 2),
             "visited_fraction": round(frac2, 4),
@@ -496,6 +585,7 @@ def run_ours(args, rank, world, local_rank, dist_on):
         def dec1m():
             P.star_phase2_attend(sq, sk, sv, S1, q_pos0=T1, rope_theta=SC.rope_theta, o=so_, lse=sl_, ws=sws)
         dec1m_ms, _ = timed(dec1m)
+        require_ok(P, sws, "1M decode")
         kv1m = 2.0 * B1 * T1 * SC.hkv * SC.d * 2
         extra["phase2_decode_1m"] = {
             "workload": SC.name, "ms": round(dec1m_ms, 4), "gb_s": round(kv1m / (dec1m_ms * 1e-3) / 1e9, 1),
@@ -532,6 +622,7 @@ def run_ours(args, rank, world, local_rank, dist_on):
         g1.record()
         torch.cuda.synchronize()
         gen_ms = g0.elapsed_time(g1) / gen
+        require_ok(P, gws, "generation steps")
         # the same 128 steps captured once in a CUDA graph and replayed (each
         # replay rewrites the same own-cache rows): GPU time per token without
         # the Python / ctypes cost of the per-token call
@@ -578,6 +669,7 @@ def run_ours(args, rank, world, local_rank, dist_on):
                 a1.record()
                 torch.cuda.synchronize()
                 sc[f"{wl.name}:{name}_us"] = round(a0.elapsed_time(a1) / 10 * 1e3, 1)
+                require_ok(P, sws, f"selection {wl.name} {name}")
                 # the same call captured once in a CUDA graph and replayed: the
                 # GPU time without the Python / ctypes enqueue cost per call
                 graph = torch.cuda.CUDAGraph()
@@ -604,16 +696,20 @@ def run_ours(args, rank, world, local_rank, dist_on):
     line = {
         "metric": METRIC, "value": round(tokens_per_s, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "scaling": "strong" if hosts_layout else "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
         "config": {"workload": w.name, "L": w.L, "block": w.block, "n_blocks": w.n_blocks, "hq": w.hq,
                    "hkv": w.hkv, "d": w.d, "sink": w.sink, "chunk": w.chunk,
                    "summary_tokens": w.k_chunks * w.chunk, "q_tokens": w.q_tokens,
-                   "rope_theta": w.rope_theta, "per_rank": "one independent 128K sequence",
+                   "rope_theta": w.rope_theta,
+                   "layout": args.layout,
+                   "per_rank": (f"hosts [{h0}, {h1}) of one shared 128K sequence, then the Phase-2 NCCL all-gather"
+                                if hosts_layout else "one independent 128K sequence"),
                    "l2": "inputs larger than L2 (Q alone is 1 GiB)"},
         "clocks": clocks,
-        "e2e": {"value": round(whole_job_rate(w.L, world, e2e_ms), 1), "unit": "tokens/s",
+        "e2e": {"value": round(e2e_rate, 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3)},
-        "gpu_launches": Step.LAUNCHES * K,
+        "gpu_launches": step.launches() * K,
         "roofline": {"bound": "tensor", "kernel": "phase-1 attention", "achieved": round(attn_tf, 1),
                      "peak": peak_tf, "unit": "TFLOP/s", "frac": round(attn_tf / peak_tf, 4),
                      "peak_kind": f"{peak_kind} bf16 sustained",
@@ -642,70 +738,119 @@ def run_ours(args, rank, world, local_rank, dist_on):
 # --------------------------------------------------------------------------
 # the oracle on the host cores (cpu_baseline leg and --impl reference)
 # --------------------------------------------------------------------------
-def oracle_sample(w, target_s=12.0, seed=0):
-    """Time the fp64 oracle on a bounded sample of one step and extrapolate.
-    Returns (estimated step seconds, sample description, threads)."""
-    import oracle
-    from threadpoolctl import threadpool_info
+ORACLE_SAMPLE_ROWS = 384   # Phase-1 rows of the last host timed on the host cores (about 9 s on 16 cores)
 
-    threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    ids = w.token_ids()
-    t = time.perf_counter()
-    sel = oracle.select_summaries(ids, w.block, w.chunk, w.k_chunks, w.vocab)
-    t_sel = time.perf_counter() - t
-    pos = oracle.host_positions(w.L, w.block, w.sink, w.chunk, sel)
-    last = len(pos) - 1
-    n = len(pos[last])
-    q, k, v = w.qkv()
-    qf = q.to(torch.float64).numpy()
-    kf = k.to(torch.float64).numpy()
-    vf = v.to(torch.float64).numpy()
-    rng = np.random.default_rng(seed)
-    nrows = 4
-    t_p1 = 0.0
-    sample_flops = 0.0
-    while True:
-        rows = np.sort(rng.choice(n, size=nrows, replace=False))
+
+def _oracle_threads():
+    """Threads the oracle's numpy BLAS uses, and the host's logical cores."""
+    from threadpoolctl import threadpool_info
+    blas = max([i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"] + [1])
+    return blas, os.cpu_count() or 1
+
+
+class OracleSample:
+    """The fp64 oracle timed on one fixed sample of a step, extrapolated.
+
+    The sample is the same in every run (and in both the cpu_baseline leg
+    and --impl reference): the whole Max-IDF selection; Phase 1 of the last
+    (longest) host for ``n_rows`` rows evenly spaced over it, which the
+    oracle evaluates against every column up to the last sampled row (after
+    rotating those rows), extrapolated to the step's algorithmic Phase-1
+    FLOPs by the FLOPs it executed; Phase 2 of one kv group of the 64-token
+    query, times the number of kv groups.  The fp64 inputs are prepared once,
+    untimed, and paged in by an untimed call on the last sampled row."""
+
+    def __init__(self, w, n_rows=ORACLE_SAMPLE_ROWS):
+        import oracle
+        self.oracle, self.w = oracle, w
+        self.ids = w.token_ids()
+        q, k, v = w.qkv()
+        self.qf = q.to(torch.float64).numpy()
+        self.kf = k.to(torch.float64).numpy()
+        self.vf = v.to(torch.float64).numpy()
+        del q, k, v
+        sel = oracle.select_summaries(self.ids, w.block, w.chunk, w.k_chunks, w.vocab)
+        self.pos_last = oracle.host_positions(w.L, w.block, w.sink, w.chunk, sel)[-1]
+        n = len(self.pos_last)
+        self.rows = np.unique(np.linspace(0, n - 1, n_rows).round().astype(np.int64))
+        self.kc, self.vc = oracle.retained_kv(self.kf[:, :1], self.vf[:, :1], w.rope_theta)   # one kv head
+        self.qq = w.query().to(torch.float64).numpy()[:, :, :w.hq // w.hkv]
+        oracle.phase1_encode(self.qf, self.kf, self.vf, [self.pos_last], w.rope_theta, [self.rows[-1:]])
+
+    def run(self):
+        """Returns (estimated step seconds, sample description)."""
+        o, w = self.oracle, self.w
         t = time.perf_counter()
-        oracle.phase1_encode(qf, kf, vf, [pos[last]], w.rope_theta, [rows])
-        dt = time.perf_counter() - t
-        t_p1 += dt
-        sample_flops += float(sum(4.0 * w.d * w.hq * (r + 1) for r in rows))
-        if t_p1 >= target_s * 0.7 or nrows >= 256:
-            break
-        nrows *= 2
-    total_flops = attn_flops(w)
-    t_p1_est = t_p1 * total_flops / sample_flops
-    kc, vc = oracle.retained_kv(kf[:, :1], vf[:, :1], w.rope_theta)   # one kv head
-    g = w.hq // w.hkv
-    qq = w.query().to(torch.float64).numpy()[:, :, :g]
+        sel = o.select_summaries(self.ids, w.block, w.chunk, w.k_chunks, w.vocab)
+        t_sel = time.perf_counter() - t
+        pos = o.host_positions(w.L, w.block, w.sink, w.chunk, sel)
+        assert np.array_equal(pos[-1], self.pos_last)
+        t = time.perf_counter()
+        o.phase1_encode(self.qf, self.kf, self.vf, [pos[-1]], w.rope_theta, [self.rows])
+        t_p1 = time.perf_counter() - t
+        cols = int(self.rows.max()) + 1
+        executed = 4.0 * w.d * w.hq * self.rows.size * cols    # QK^T and PV of every sampled row over `cols`
+        total_flops = attn_flops(w)
+        t_p1_est = t_p1 * total_flops / executed
+        t = time.perf_counter()
+        o.phase2_attend(self.qq, self.kc[None], self.vc[None], w.n_blocks, w.L, w.rope_theta)
+        t_p2 = time.perf_counter() - t
+        est = t_sel + t_p1_est + t_p2 * w.hkv
+        desc = (f"full selection ({t_sel:.2f} s); Phase 1 of the last host for {self.rows.size} evenly spaced "
+                f"rows against {cols} columns ({executed / 1e9:.0f} GFLOP executed of {total_flops / 1e12:.1f} "
+                f"TFLOP, {t_p1:.1f} s, extrapolated by FLOPs); Phase 2 one kv group of {w.hkv} ({t_p2:.2f} s, "
+                f"x{w.hkv})")
+        return est, desc
+
+
+def oracle_tiny_full():
+    """The complete oracle run of the tiny workload (selection, Phase 1 of
+    every row of every host, the 32-token query over its 4 shards): seconds,
+    nothing extrapolated."""
+    import oracle
+    w = workloads.TINY
     t = time.perf_counter()
-    oracle.phase2_attend(qq, kc[None], vc[None], w.n_blocks, w.L, w.rope_theta)
-    t_p2 = time.perf_counter() - t
-    t_p2_est = t_p2 * w.hkv
-    est = t_sel + t_p1_est + t_p2_est
-    desc = (f"full selection ({t_sel:.2f} s); Phase-1 rows of the last host ({int(sample_flops / 1e9)} GFLOP "
-            f"of {total_flops / 1e12:.1f} TFLOP, {t_p1:.1f} s, extrapolated by FLOPs); Phase-2 one kv group "
-            f"of {w.hkv} ({t_p2:.1f} s, x{w.hkv})")
-    return est, desc, threads
+    ids = w.token_ids()
+    sel = oracle.select_summaries(ids, w.block, w.chunk, w.k_chunks, w.vocab)
+    pos = oracle.host_positions(w.L, w.block, w.sink, w.chunk, sel)
+    q, k, v = (x.to(torch.float64).numpy() for x in w.qkv())
+    oracle.phase1_encode(q, k, v, pos, w.rope_theta)
+    kc, vc = oracle.retained_kv(k, v, w.rope_theta)
+    oracle.phase2_attend(w.query().to(torch.float64).numpy(), kc[None], vc[None], w.n_blocks, w.L, w.rope_theta)
+    return time.perf_counter() - t
+
+
+def cpu_baseline_record(est, desc, tiny_s):
+    blas, nproc = _oracle_threads()
+    w = WORKLOAD
+    return {"value": round(w.L / est, 3), "unit": "tokens/s", "cores": blas, "nproc": nproc, "kind": "oracle",
+            "sample": desc,
+            "tiny_full": {"workload": workloads.TINY.name, "seconds": round(tiny_s, 3),
+                          "tokens_per_s": round(workloads.TINY.L / tiny_s, 1), "extrapolated": False}}
 
 
 def run_reference(args):
     w = WORKLOAD
-    ests, desc, threads = [], "", 1
-    for i in range(args.warmup):
-        oracle_sample(w, target_s=2.0, seed=100 + i)
-    for i in range(args.steps):
-        est, desc, threads = oracle_sample(w, target_s=8.0, seed=i)
+    sample = OracleSample(w)
+    ests, desc = [], ""
+    for _ in range(args.warmup):
+        sample.run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        est, desc = sample.run()
         ests.append(est)
+    sample_ms = (time.perf_counter() - t0) / max(args.steps, 1) * 1e3
     est = statistics.mean(ests)
     value = w.L / est
+    rec = cpu_baseline_record(est, desc + f"; mean of {args.steps} runs of the same sample", oracle_tiny_full())
     return {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(est * 1e3, 1),
+            "sample_ms_per_step": round(sample_ms, 1),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": w.name, "L": w.L, "block": w.block},
-            "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                             "sample": desc},
+            "data": "synthetic", "config": {"workload": w.name, "L": w.L, "block": w.block,
+                       "note": "ms_per_step is the step's extrapolated oracle time; each timed step runs the "
+                               "fixed sample (sample_ms_per_step)"},
+            "cpu_baseline": rec,
             "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
@@ -780,6 +925,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--headline-only", action="store_true", help="skip the side measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layout", default="sequences", choices=["sequences", "hosts"],
+                    help="sequences: one independent sequence per rank (weak scaling); hosts: the hosts of one "
+                         "sequence spread over the ranks, with the Phase-2 all-gather over NCCL (strong scaling)")
     ap.add_argument("--profile-case", default=None,
                     help="run one kernel family on a small workload (phase1-32k, decode-16k, decode-128k, query-128k, select-1m)")
     args = ap.parse_args()
@@ -795,21 +943,29 @@ def main():
             print(json.dumps(run_reference(args)), flush=True)
         return
     dist_on = world > 1
-    if dist_on:
+    group_on = dist_on or args.layout == "hosts"
+    if group_on:
         import datetime
         torch.cuda.set_device(local_rank)
+        if not dist_on:   # the hosts layout on one GPU: a process group of one rank
+            import socket
+            with socket.socket() as sk:
+                sk.bind(("127.0.0.1", 0))
+                os.environ.setdefault("MASTER_PORT", str(sk.getsockname()[1]))
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            os.environ.setdefault("RANK", "0")
+            os.environ.setdefault("WORLD_SIZE", "1")
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                              device_id=torch.device("cuda", local_rank))
     try:
         line = run_ours(args, rank, world, local_rank, dist_on)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
-            est, desc, threads = oracle_sample(WORKLOAD)
-            line["cpu_baseline"] = {"value": round(WORKLOAD.L / est, 3), "unit": "tokens/s", "cores": threads,
-                                    "kind": "oracle", "sample": desc}
+            est, desc = OracleSample(WORKLOAD).run()
+            line["cpu_baseline"] = cpu_baseline_record(est, desc, oracle_tiny_full())
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:
-        if dist_on:
+        if group_on:
             torch.distributed.destroy_process_group()
 
 

@@ -90,3 +90,16 @@ def test_clock_summary_reads_median_max_and_active_reasons():
 def test_whole_job_rate_counts_every_rank():
     assert bench.whole_job_rate(131072, 1, 37.0) == pytest.approx(131072 / 0.037)
     assert bench.whole_job_rate(131072, 8, 40.0) == pytest.approx(8 * 131072 / 0.040)
+
+
+def test_attn_flops_of_host_ranges_add_up():
+    # --layout hosts: each rank's roofline counts the FLOPs of its own hosts;
+    # the ranks' ranges tile the sequence, so their FLOPs add up to the whole
+    from long_context_blockwise_max_b200.distributed import shard_ranges
+    w = workloads.LLAMA_128K
+    for world in (1, 2, 3, 8):
+        parts = [bench.attn_flops(w, hosts=r) for r in shard_ranges(w.n_blocks, world)]
+        assert sum(parts) == pytest.approx(bench.attn_flops(w), rel=1e-12)
+    # the last host alone: n = 64 + 7 * 2048 + 16384 rows
+    n = 64 + 7 * 2048 + 16384
+    assert bench.attn_flops(w, hosts=(7, 8)) == 4.0 * w.d * w.hq * n * (n + 1) / 2.0
