@@ -214,25 +214,27 @@ __global__ void __launch_bounds__(384, 1) phase1_tc_kernel(const __grid_constant
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0) {
-      const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
+      // base descriptors, computed once; each MMA adds a constant offset
+      const uint64_t q_desc = sdesc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t k_desc = sdesc_sw128(smem_u32(sK), 16, 1024);
+      const uint64_t v_desc = sdesc_sw128(smem_u32(sV), C::KB_BYTES, 1024);
       auto qk = [&](int t, int st) {
         const uint32_t d_tmem = tmem + t * 256;
+        const uint64_t qd = sdesc_add(q_desc, t * C::TILE_BYTES);
+        const uint64_t kd = sdesc_add(k_desc, st * C::TILE_BYTES);
 #pragma unroll
         for (int kb = 0; kb < C::NKB; ++kb)
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t a = sdesc_sw128(q_addr + t * C::TILE_BYTES + kb * C::KB_BYTES + ks * 32, 16, 1024);
-            const uint64_t b = sdesc_sw128(k_addr + st * C::TILE_BYTES + kb * C::KB_BYTES + ks * 32, 16, 1024);
-            mma_ss(d_tmem, a, b, C::IDESC_QK, (kb | ks) != 0);
-          }
+          for (int ks = 0; ks < 4; ++ks)
+            mma_ss(d_tmem, sdesc_add(qd, kb * C::KB_BYTES + ks * 32), sdesc_add(kd, kb * C::KB_BYTES + ks * 32),
+                   C::IDESC_QK, (kb | ks) != 0);
       };
       auto pv = [&](int t, int st, int acc) {
         const uint32_t d_tmem = tmem + t * 256 + 128;
+        const uint64_t vd = sdesc_add(v_desc, st * C::TILE_BYTES);
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint64_t b = sdesc_sw128(v_addr + st * C::TILE_BYTES + ks * 2048, C::KB_BYTES, 1024);
-          mma_ts(d_tmem, tmem + t * 256 + ks * 8, b, C::IDESC_PV, (acc | ks) != 0);
-        }
+        for (int ks = 0; ks < 8; ++ks)
+          mma_ts(d_tmem, tmem + t * 256 + ks * 8, sdesc_add(vd, ks * 2048), C::IDESC_PV, (acc | ks) != 0);
       };
       bool ok = mbar_wait(&bars->q_full, 0, abort, p.wait_ns, gabort);
       if (!ok) fail(3);

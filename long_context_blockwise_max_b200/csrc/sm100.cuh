@@ -210,6 +210,14 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
   return d;
 }
 
+// The descriptor of base + off: the start-address field holds bits 4..17 of
+// a shared-memory address, and every shared address and offset used here is
+// below 256 KB and 16-byte aligned, so the field never carries into the next
+// one and adding off / 16 to the whole descriptor is exact.
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t desc, uint32_t off_bytes) {
+  return desc + static_cast<uint64_t>(off_bytes >> 4);
+}
+
 // Instruction descriptor of tcgen05.mma kind::f16 with an fp32 accumulator.
 // a_fmt / b_fmt: 0 = f16, 1 = bf16.  a_mn / b_mn: 1 = MN-major operand.
 __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int a_fmt, int b_fmt, int a_mn, int b_mn) {
