@@ -70,8 +70,8 @@ const char* pa_status_string(int status);
  * Waits for `stream`, then returns the device status recorded in `ws` by the
  * last call that used this workspace: PA_OK, PA_ERR_INVALID (an id out of
  * [0, vocab) or a chunk index out of range met on the device), PA_ERR_RANGE
- * (a rotated Q/K value outside the fp16 range used internally for bf16
- * inputs) or PA_ERR_TIMEOUT.  Returns PA_ERR_CUDA if the copy fails.  This
+ * (a Phase-1 rotated Q/K value outside the fp16 range used internally for
+ * bf16 inputs) or PA_ERR_TIMEOUT.  Returns PA_ERR_CUDA if the copy fails.  This
  * is the only synchronising call of the library.
  */
 int pa_workspace_status(const void* ws, void* stream);
@@ -235,9 +235,11 @@ size_t pa_phase1_hosts_workspace_size(int64_t L, int32_t hq, int32_t hkv, int32_
  *                 may equal v (then it is not written).
  *
  * d must be 64 or 128, hq % hkv == 0.  For PA_BF16, rotated Q and K are
- * carried in fp16 for the QK^T product (status PA_ERR_RANGE if a rotated
- * value exceeds 65504); P is rounded to bf16 for the PV product; all sums
- * are fp32.  For PA_F32 the whole path is fp32.
+ * carried in fp16 for the QK^T product; P is rounded to bf16 for the PV
+ * product; all sums are fp32.  For PA_F32 the whole path is fp32.
+ * Limit (bf16): a rotated Q value times log2(e)/sqrt(d), or a rotated K
+ * value, beyond 65504 is refused through the device status PA_ERR_RANGE
+ * (pa_workspace_status); the outputs are then unspecified.
  */
 int pulsar_phase1_encode(const void* q, const void* k, const void* v, int dtype, int64_t L,
                          int32_t hq, int32_t hkv, int32_t d, double rope_theta, int32_t block,
@@ -315,10 +317,13 @@ size_t pa_phase2_workspace_size(int32_t B, int32_t Tq, int64_t T, int32_t n_shar
  * Precision (bf16): on the tensor-core path (at least 64 query rows per kv
  * head, Tq * hq / hkv; hq / hkv dividing 128; 16-byte aligned caches) the
  * scores are computed from the rotated query rounded to fp16 against the
- * keys converted exactly to fp16 (device status PA_ERR_RANGE if a rotated,
- * scaled query value or a key is outside fp16 range); otherwise from a bf16
- * high part plus a bf16 residual of the query, exact against the stored
- * keys to fp32 rounding.  P is rounded to bf16 for P V.
+ * keys converted exactly to fp16; a work unit that meets a key beyond fp16
+ * range (every unit, if a rotated query value times log2(e)/sqrt(d) is) is
+ * recomputed in fp32 (bf16 keys widened exactly, fp32 sums), so every bf16
+ * input is computed.  Otherwise
+ * the scores come from a bf16 high part plus a bf16 residual of the query
+ * (about 16 significant bits of the rotated query) against the stored keys,
+ * summed in fp32.  P is rounded to bf16 for P V.
  */
 int star_phase2_attend(const void* q, int dtype, int32_t B, int32_t Tq, int64_t q_pos0,
                        double rope_theta, const void* k_ret, const void* v_ret, int64_t T,

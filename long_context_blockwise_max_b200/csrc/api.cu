@@ -186,6 +186,10 @@ void carve_phase2(Phase2Args& a, void* ws) {
   a.unit_o = reinterpret_cast<float*>(w + off);
   off += align_up(sizeof(float) * rows * units * a.d);
   a.unit_lse = reinterpret_cast<float*>(w + off);
+  off += align_up(sizeof(float) * rows * units);
+  a.q16 = reinterpret_cast<__half*>(w + off);
+  off += align_up(sizeof(__half) * rows * a.d);
+  a.redo = reinterpret_cast<int32_t*>(w + off);
 }
 
 }  // namespace

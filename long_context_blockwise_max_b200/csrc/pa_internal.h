@@ -125,6 +125,11 @@ struct Phase2Args {
   // bounded-wait limit of the tensor-core query kernel and a test-only stall
   uint64_t wait_limit_ns = 1000000000ull;
   int stall = 0;
+  // tensor-core query path: the fp16 query, and per (batch, unit, kv head)
+  // flags of units to recompute exactly (+ one flag: the query left fp16
+  // range), both in the workspace
+  __half* q16 = nullptr;
+  int32_t* redo = nullptr;   // [B * units * hkv + 1]
 };
 
 // One Phase-2 work unit: a split of a context shard, or (the last unit, when

@@ -19,13 +19,13 @@ namespace pa {
 
 // q [B][Tq][hq][d] -> qr fp32, rotated at q_pos0 + t (theta > 0) and scaled
 // by log2(e)/sqrt(d) so that scores come out in log2 units.  With `q16` set,
-// writes that value in fp16 instead (same layout; the operand of the
-// tensor-core query kernel) and sets PA_ERR_RANGE when it is not finite in
-// fp16.
+// also writes that value in fp16 (same layout; the operand of the
+// tensor-core query kernel) and, when it is not finite in fp16, sets
+// *redo_all so that every unit is recomputed from the fp32 query.
 template <typename IT>
 __global__ void rope_query_kernel(const IT* __restrict__ q, int B, int Tq, int hq, int d,
                                   int64_t q_pos0, int use_rope, RopeFreqs f, float qscale,
-                                  float* __restrict__ qr, __half* __restrict__ q16, DeviceStatus* st) {
+                                  float* __restrict__ qr, __half* __restrict__ q16, int32_t* redo_all) {
   bool bad = false;
   const int half = d / 2;
   const int64_t n = (int64_t)B * Tq * hq * half;
@@ -45,26 +45,33 @@ __global__ void rope_query_kernel(const IT* __restrict__ q, int B, int Tq, int h
       y2 = x2 * c + x1 * s;
     }
     const float z1 = y1 * qscale, z2 = y2 * qscale;
+    qr[base + m] = z1;
+    qr[base + m + half] = z2;
     if (q16 != nullptr) {
       q16[base + m] = __float2half_rn(z1);
       q16[base + m + half] = __float2half_rn(z2);
       bad |= !(fabsf(z1) <= 65504.f) || !(fabsf(z2) <= 65504.f);
-    } else {
-      qr[base + m] = z1;
-      qr[base + m + half] = z2;
     }
   }
-  if (bad) set_status(st, PA_ERR_RANGE, 0, 2);
+  if (bad) atomicExch(redo_all, 1);
 }
 
+// fp32 partial attention of one (batch, unit, kv head, 128 query rows): the
+// kernel of fp32 inputs, and the exact recomputation of bf16 units flagged
+// by the tensor-core query kernel (`redo` non-null: only CTAs whose unit is
+// flagged, or all when the query itself was flagged, do any work; bf16 keys
+// widen exactly to fp32 and the query is the fp32 rotated one).
 template <int D, typename VT>
-__global__ void __launch_bounds__(256) phase2_simt_kernel(Phase2Args a) {
+__global__ void __launch_bounds__(256) phase2_simt_kernel(Phase2Args a, const int32_t* __restrict__ redo) {
   constexpr int BK = 32, HALF = D / 2, G4 = HALF / 4;
   __shared__ __align__(16) float ks[BK][D];
   __shared__ __align__(16) float vs[BK][D];
   const int units = phase2_units(a);
   const int b = blockIdx.x / units, u = blockIdx.x % units;
   const int kvh = blockIdx.y, g = a.hq / a.hkv;
+  if (redo != nullptr && redo[(int64_t)blockIdx.x * a.hkv + kvh] == 0 &&
+      redo[(int64_t)a.B * units * a.hkv] == 0)
+    return;
   const int idx = blockIdx.z * 128 + (threadIdx.x >> 1);
   const int hf = threadIdx.x & 1;
   const bool active = idx < a.Tq * g;
@@ -318,6 +325,8 @@ size_t phase2_workspace_bytes(int32_t B, int32_t Tq, int64_t T, int32_t n_shards
   b += align_up(sizeof(float) * rows * d);          // rotated query
   b += align_up(sizeof(float) * rows * units * d);  // unit partial outputs
   b += align_up(sizeof(float) * rows * units);      // unit partial lse
+  b += align_up(sizeof(__half) * rows * d);         // fp16 query (tensor-core path)
+  b += align_up(sizeof(int32_t) * ((size_t)B * units * hkv + 1));   // redo flags
   return b;
 }
 
@@ -328,31 +337,37 @@ static int launch_phase2_t(const Phase2Args& a, cudaStream_t s) {
     f.omega[m] = (m < a.d / 2 && a.rope_theta > 0) ? pow(a.rope_theta, -2.0 * m / a.d) : 0.0;
   const float qscale = (float)(kLog2e / sqrt((double)a.d));
   const int64_t nq = (int64_t)a.B * a.Tq * a.hq * (a.d / 2);
-  // the tensor-core query kernel reads the query in fp16, which takes the
-  // place of the fp32 rotated query in the workspace
+  // the tensor-core query kernel reads the query in fp16; units it cannot
+  // carry in fp16 (a key, or the query, outside fp16 range) are flagged and
+  // recomputed in fp32 by phase2_simt_kernel afterwards
   const bool tc = phase2_tc_supported(a);
-  __half* q16 = tc ? reinterpret_cast<__half*>(a.qr) : nullptr;
+  const int units = phase2_units(a);
+  const size_t n_flags = (size_t)a.B * units * a.hkv + 1;
+  if (tc && cudaMemsetAsync(a.redo, 0, sizeof(int32_t) * n_flags, s) != cudaSuccess) return PA_ERR_CUDA;
   if (nq > 0) {
     const int64_t want = (nq + 255) / 256;
     rope_query_kernel<IT><<<(int)(want < 148 * 8 ? want : 148 * 8), 256, 0, s>>>(
         static_cast<const IT*>(a.q), a.B, a.Tq, a.hq, a.d, a.q_pos0, a.rope_theta > 0, f, qscale,
-        a.qr, q16, a.status);
+        a.qr, tc ? a.q16 : nullptr, a.redo + (n_flags - 1));
   }
-  const int units = phase2_units(a);
   const int g = a.hq / a.hkv;
   const dim3 grid((unsigned)(a.B * units), a.hkv, (unsigned)((a.Tq * g + 127) / 128));
   int rc = PA_OK;
   profile_begin(s);
   if (tc) {
-    rc = launch_phase2_tc(a, q16, s);
+    rc = launch_phase2_tc(a, a.q16, s);
   } else if (a.dtype == PA_BF16) {
     rc = launch_phase2_mma(a, s);
   } else if (grid.x > 0 && grid.z > 0) {
-    if (a.d == 128) phase2_simt_kernel<128, IT><<<grid, 256, 0, s>>>(a);
-    else phase2_simt_kernel<64, IT><<<grid, 256, 0, s>>>(a);
+    if (a.d == 128) phase2_simt_kernel<128, IT><<<grid, 256, 0, s>>>(a, nullptr);
+    else phase2_simt_kernel<64, IT><<<grid, 256, 0, s>>>(a, nullptr);
   }
   profile_end(s);
   if (rc != PA_OK) return rc;
+  if (tc && grid.x > 0 && grid.z > 0) {   // exact recomputation of the flagged units (usually none)
+    if (a.d == 128) phase2_simt_kernel<128, IT><<<grid, 256, 0, s>>>(a, a.redo);
+    else phase2_simt_kernel<64, IT><<<grid, 256, 0, s>>>(a, a.redo);
+  }
   launch_merge_kernel<IT>(a, s);
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
@@ -423,11 +438,11 @@ int launch_rope_query(const Phase2Args& a, cudaStream_t s) {
     if (a.dtype == PA_F32)
       rope_query_kernel<float><<<(int)(want < 148 * 8 ? want : 148 * 8), 256, 0, s>>>(
           static_cast<const float*>(a.q), a.B, a.Tq, a.hq, a.d, a.q_pos0, a.rope_theta > 0, f, qscale, a.qr,
-          nullptr, a.status);
+          nullptr, nullptr);
     else
       rope_query_kernel<__nv_bfloat16><<<(int)(want < 148 * 8 ? want : 148 * 8), 256, 0, s>>>(
           static_cast<const __nv_bfloat16*>(a.q), a.B, a.Tq, a.hq, a.d, a.q_pos0, a.rope_theta > 0, f, qscale,
-          a.qr, nullptr, a.status);
+          a.qr, nullptr, nullptr);
   }
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }

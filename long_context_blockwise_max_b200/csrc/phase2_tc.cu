@@ -302,7 +302,9 @@ __global__ void __launch_bounds__(384, 1) phase2_tc_kernel(const __grid_constant
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       mbar_arrive(&bars->k_conv[sk]);
     }
-    if (bad) set_status(a.status, PA_ERR_RANGE, static_cast<int>(blockIdx.x), 1);
+    // a key of this unit outside fp16 range: the unit is recomputed exactly
+    // (mma.sync row kernel, high / low bf16 query) after this kernel
+    if (bad) atomicExch(a.redo + (static_cast<int64_t>(b) * p.units + u) * a.hkv + kvh, 1);
   } else {
     // -------------------------------------------------------------- softmax
     const int t = warp >= 8 ? 1 : 0;

@@ -99,9 +99,33 @@ def _stream():
     return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
 
 
-def _check(rc: int, where: str):
+def _check(rc: int, where: str, ws=None):
+    """Raise PulsarError for a negative return code; with device-status
+    checks on (set_status_checks), also wait for the call and raise for a
+    non-zero status its kernels recorded in the workspace ``ws``."""
     if rc != 0:
         raise PulsarError(rc, where)
+    if _STATUS_CHECKS and ws is not None:
+        code = _lib.pa_workspace_status(_ptr(ws), _stream())
+        if code != 0:
+            raise PulsarError(code, where + " (device status)")
+
+
+# Device-status checks after every call (off by default: reading the status
+# waits for the stream).  Device-detected errors -- an id or summary index
+# out of range, a Phase-1 value beyond the fp16 range used for bf16 inputs,
+# an expired bounded wait -- otherwise only land in the workspace's status
+# block (pa_workspace_status).
+_STATUS_CHECKS = os.environ.get("PULSAR_CHECK_STATUS", "0") not in ("", "0")
+
+
+def set_status_checks(enabled: bool) -> bool:
+    """Turn the device-status check after every call on or off; returns the
+    previous setting."""
+    global _STATUS_CHECKS
+    prev = _STATUS_CHECKS
+    _STATUS_CHECKS = bool(enabled)
+    return prev
 
 
 def _dtype_code(t: torch.Tensor) -> int:
@@ -193,7 +217,7 @@ def pulsar_select_summaries(ids: torch.Tensor, vocab: int, block: int, chunk: in
     ws = _workspace(need, dev, ws)
     rc = _lib.pulsar_select_summaries(_ptr(ids), L, vocab, block, chunk, k_chunks, _ptr(sel),
                                       _ptr(df), _ptr(chunk_mindf), _ptr(ws), ws.numel() * ws.element_size(), _stream())
-    _check(rc, "pulsar_select_summaries")
+    _check(rc, "pulsar_select_summaries", ws)
     return sel, df, chunk_mindf, ws
 
 
@@ -232,7 +256,7 @@ def pulsar_select_summaries_scored(ids, vocab: int, block: int, chunk: int, k_ch
     ws = _workspace(pa_select_workspace_size(L, vocab, block, chunk), dev, ws)
     rc = _lib.pulsar_select_summaries_scored(_ptr(ids), L, vocab, block, chunk, k_chunks, int(method), _ptr(sel),
                                              _ptr(scores), _ptr(ws), ws.numel() * ws.element_size(), _stream())
-    _check(rc, "pulsar_select_summaries_scored")
+    _check(rc, "pulsar_select_summaries_scored", ws)
     return sel, scores, ws
 
 
@@ -300,7 +324,7 @@ def pulsar_phase1_encode(q, k, v, rope_theta, block, sink, chunk, k_chunks, sel,
     rc = _lib.pulsar_phase1_encode(_ptr(q), _ptr(k), _ptr(v), dt, L, hq, hkv, d, float(rope_theta), block,
                                    sink, chunk, k_chunks, _ptr(sel), _ptr(o), _ptr(lse), _ptr(k_ret),
                                    _ptr(v_ret), _ptr(ws), ws.numel() * ws.element_size(), _stream())
-    _check(rc, "pulsar_phase1_encode")
+    _check(rc, "pulsar_phase1_encode", ws)
     return o, lse, k_ret, v_ret, row_off, ws
 
 
@@ -319,7 +343,7 @@ def star_phase1_encode(q, k, v, rope_theta, block, o=None, lse=None, k_ret=None,
     rc = _lib.star_phase1_encode(_ptr(q), _ptr(k), _ptr(v), dt, L, hq, hkv, d, float(rope_theta), block,
                                  _ptr(o), _ptr(lse), _ptr(k_ret), _ptr(v_ret), _ptr(ws), ws.numel(),
                                  _stream())
-    _check(rc, "star_phase1_encode")
+    _check(rc, "star_phase1_encode", ws)
     return o, lse, k_ret, v_ret, row_off, ws
 
 
@@ -360,7 +384,7 @@ def pulsar_phase1_encode_hosts(q, k, v, rope_theta, block, sink, chunk, k_chunks
     rc = _lib.pulsar_phase1_encode_hosts(_ptr(q), _ptr(k), _ptr(v), dt, L, hq, hkv, d, float(rope_theta), block,
                                          sink, chunk, k_chunks, _ptr(sel), host_begin, host_end, _ptr(o), _ptr(lse),
                                          _ptr(k_ret), _ptr(v_ret), _ptr(ws), ws.numel(), _stream())
-    _check(rc, "pulsar_phase1_encode_hosts")
+    _check(rc, "pulsar_phase1_encode_hosts", ws)
     return o, lse, k_ret, v_ret, row_off, ws
 
 
@@ -383,7 +407,7 @@ def star_phase1_encode_hosts(q, k, v, rope_theta, block, host_begin, host_end, o
     rc = _lib.star_phase1_encode_hosts(_ptr(q), _ptr(k), _ptr(v), dt, L, hq, hkv, d, float(rope_theta), block,
                                        host_begin, host_end, _ptr(o), _ptr(lse), _ptr(k_ret), _ptr(v_ret), _ptr(ws),
                                        ws.numel(), _stream())
-    _check(rc, "star_phase1_encode_hosts")
+    _check(rc, "star_phase1_encode_hosts", ws)
     return o, lse, k_ret, v_ret, row_off, ws
 
 
@@ -429,7 +453,7 @@ def star_phase2_attend(q, k_ret, v_ret, n_shards, q_pos0=0, rope_theta=0.0, o=No
     rc = _lib.star_phase2_attend(_ptr(q), dt, B, Tq, int(q_pos0), float(rope_theta), _ptr(k_ret), _ptr(v_ret),
                                  T, n_shards, hq, hkv, d, _ptr(o), _ptr(lse), _ptr(part_o), _ptr(part_lse),
                                  _ptr(ws), ws.numel() * ws.element_size(), _stream())
-    _check(rc, "star_phase2_attend")
+    _check(rc, "star_phase2_attend", ws)
     return o, lse, part_o, part_lse, ws
 
 
@@ -451,7 +475,7 @@ def star_phase2_attend_art(q, k_ret, v_ret, q_pos0=0, rope_theta=0.0, block_keys
                                      _ptr(v_ret), T, hq, hkv, d, int(block_keys), float(tau), float(phi),
                                      int(patience), _ptr(o), _ptr(lse), _ptr(visited), _ptr(ws),
                                      ws.numel() * ws.element_size(), _stream())
-    _check(rc, "star_phase2_attend_art")
+    _check(rc, "star_phase2_attend_art", ws)
     return o, lse, visited, ws
 
 
@@ -500,7 +524,7 @@ def star_phase2_query_step(q, k_new, v_new, k_ret, v_ret, n_shards, k_self, v_se
                                      float(rope_theta), _ptr(k_ret), _ptr(v_ret), T, n_shards, _ptr(k_self),
                                      _ptr(v_self), k_self.shape[1], int(self_len), hq, hkv, d, _ptr(o), _ptr(lse),
                                      _ptr(ws), ws.numel() * ws.element_size(), _stream())
-    _check(rc, "star_phase2_query_step")
+    _check(rc, "star_phase2_query_step", ws)
     return o, lse, ws
 
 

@@ -167,6 +167,20 @@ def test_range_status_for_values_beyond_fp16(P):
     *_, ws = P.pulsar_phase1_encode(qd, kd, vd, 1e4, block, 0, 16, 1, torch.zeros((2, 1), dtype=torch.int32,
                                                                                    device=DEV))
     assert P.pa_workspace_status(ws) == -6   # PA_ERR_RANGE
+    # Phase 1 carries rotated Q and K in fp16 for bf16 inputs and refuses
+    # values beyond its range through the device status; with the binding's
+    # status checks on, the call itself raises
+    prev = P.set_status_checks(True)
+    try:
+        with pytest.raises(P.PulsarError) as e:
+            P.pulsar_phase1_encode(qd, kd, vd, 1e4, block, 0, 16, 1, torch.zeros((2, 1), dtype=torch.int32,
+                                                                              device=DEV))
+        assert e.value.code == -6
+        k[5, 1, 3] = 1.0
+        P.pulsar_phase1_encode(qd, k.to(DEV), vd, 1e4, block, 0, 16, 1,
+                               torch.zeros((2, 1), dtype=torch.int32, device=DEV))   # in range: no error
+    finally:
+        P.set_status_checks(prev)
 
 
 def test_bad_summary_index_sets_status(P):

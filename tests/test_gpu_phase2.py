@@ -170,27 +170,63 @@ def test_lse_merge_entry_point(P, dtype):
     assert np.abs(lse.cpu().double().numpy()[fin] - rl[fin]).max() <= LSE_TOL
 
 
-@pytest.mark.parametrize("where", ["key", "query"])
-def test_query_kernel_range_status(P, where):
-    # the tensor-core query kernel carries the query and the keys in fp16: a
-    # value beyond fp16 range is reported as PA_ERR_RANGE (device status)
-    B, Tq, hq, hkv, d, T, S = 1, 64, 8, 2, 128, 700, 3   # 256 rows per kv head
+@pytest.mark.parametrize("where,d", [("key", 128), ("query", 128), ("key", 64), ("both", 128)])
+def test_query_kernel_values_beyond_fp16(P, where, d):
+    # the tensor-core query kernel carries the query and the keys in fp16; a
+    # unit that meets a key beyond fp16 range (any unit, when the scaled
+    # rotated query is) is recomputed in fp32, so bf16 inputs of any size give
+    # the right result (status PA_OK).  Scores here reach ~10^5 nat, and fp32
+    # sums of d products of that size carry a rounding of about
+    # |s| * 2^-24 * sqrt(d): the lse tolerance grows as 2^-20 |lse| beyond the
+    # stated 1e-3 (below 1e-3 for every score of normal-range inputs).
+    B, Tq, hq, hkv, T, S = 1, 64, 8, 2, 700, 3    # 256 rows per kv head: the tensor-core kernel
     q = workloads.normal((B, Tq, hq, d), 90, torch.bfloat16)
     kc = workloads.normal((B, T, hkv, d), 91, torch.bfloat16)
     vc = workloads.normal((B, T, hkv, d), 92, torch.bfloat16)
-    if where == "key":
-        kc[0, 321, 1, 7] = 1.0e5
-    else:
-        q[0, 5, 3, 9] = 1.0e7
-    *_, ws = P.star_phase2_attend(q.to(DEV), kc.to(DEV), vc.to(DEV), S, q_pos0=T, rope_theta=0.0)
-    assert P.pa_workspace_status(ws) == -6   # PA_ERR_RANGE
-    # the same inputs within range give PA_OK on the next call
-    if where == "key":
-        kc[0, 321, 1, 7] = 1.0
-    else:
-        q[0, 5, 3, 9] = 1.0
-    *_, ws = P.star_phase2_attend(q.to(DEV), kc.to(DEV), vc.to(DEV), S, q_pos0=T, rope_theta=0.0)
+    if where in ("key", "both"):
+        kc[0, 321, 1, 7] = 7.0e4      # beyond 65504: its unit is recomputed
+        kc[0, 650, 0, 3] = -9.0e4
+    if where in ("query", "both"):
+        q[0, 5, 3, 9] = 6.0e5         # x log2(e)/sqrt(d) is beyond 65504: every unit is recomputed
+    o, lse, po, pl, ws = P.star_phase2_attend(q.to(DEV), kc.to(DEV), vc.to(DEV), S, q_pos0=T, rope_theta=0.0,
+                                              want_partials=True)
     assert P.pa_workspace_status(ws) == 0
+    ro, rl, ra, rs = oracle.phase2_attend(f64(q), f64(kc), f64(vc), S, T, 0.0)
+    assert_close(f64(o.cpu()), ro, O_TOL[torch.bfloat16], "O")
+    assert_close(f64(po.cpu()), ra, O_TOL[torch.bfloat16], "A_h")
+    for got, want, what in ((lse.cpu().double().numpy(), rl, "lse"), (pl.cpu().double().numpy(), rs, "s_h")):
+        fin = np.isfinite(want)
+        err = np.abs(got[fin] - want[fin])
+        assert (err <= LSE_TOL + 2.0 ** -20 * np.abs(want[fin])).all(), (what, float(err.max()))
+    # the same inputs within range still run the tensor-core path alone
+    kc[0, 321, 1, 7], kc[0, 650, 0, 3], q[0, 5, 3, 9] = 1.0, -1.0, 1.0
+    o2, lse2, _, _, ws = P.star_phase2_attend(q.to(DEV), kc.to(DEV), vc.to(DEV), S, q_pos0=T, rope_theta=0.0)
+    assert P.pa_workspace_status(ws) == 0
+    ro2, rl2, _, _ = oracle.phase2_attend(f64(q), f64(kc), f64(vc), S, T, 0.0)
+    assert_close(f64(o2.cpu()), ro2, O_TOL[torch.bfloat16], "O in range")
+    assert_close(lse2.cpu().double().numpy(), rl2, LSE_TOL, "lse in range")
+
+
+def test_query_step_own_key_beyond_fp16(P):
+    # a generated token's key beyond fp16 range lands in the query host's own
+    # cache; the own-cache unit is recomputed exactly like a shard's
+    B, Tq, hq, hkv, d, T, S, cap = 1, 64, 8, 2, 128, 500, 2, 80
+    dt = torch.bfloat16
+    q = workloads.normal((B, Tq, hq, d), 93, dt)
+    kn = workloads.normal((B, Tq, hkv, d), 94, dt)
+    vn = workloads.normal((B, Tq, hkv, d), 95, dt)
+    kc = workloads.normal((B, T, hkv, d), 96, dt)
+    vc = workloads.normal((B, T, hkv, d), 97, dt)
+    kn[0, 10, 1, 4] = 8.0e4
+    ks = torch.zeros((B, cap, hkv, d), dtype=dt, device=DEV)
+    vs = torch.zeros_like(ks)
+    o, lse, ws = P.star_phase2_query_step(q.to(DEV), kn.to(DEV), vn.to(DEV), kc.to(DEV), vc.to(DEV), S, ks, vs, 0,
+                                          T, 0.0)
+    assert P.pa_workspace_status(ws) == 0
+    ro, rl = oracle.phase2_attend_with_self(f64(q), f64(kc), f64(vc), S, f64(kn), f64(vn), 0, T, 0.0)
+    assert_close(f64(o.cpu()), ro, O_TOL[dt], "O")
+    err = np.abs(lse.cpu().double().numpy() - rl)
+    assert (err <= LSE_TOL + 2.0 ** -20 * np.abs(rl)).all(), float(err.max())
 
 
 def test_query_32k_sampled_groups(P):
