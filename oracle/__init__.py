@@ -29,6 +29,11 @@ from .pulsar_oracle import (  # noqa: F401
     chunk_df_product,
     select_evenly_spaced,
     select_summaries_mean_idf,
+    chunk_entropy,
+    chunk_tf_power_product,
+    select_summaries_entropy,
+    chunk_bm25,
+    select_summaries_bm25,
     phase2_attend_with_self,
     phase2_attend_art,
 )

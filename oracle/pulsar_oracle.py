@@ -44,7 +44,11 @@ form lse = ln(r+1), and complex-multiplication RoPE (Phase 1); the shard merge
 equals library dense attention over the concatenated cache (Phase 2).  Added
 rows: mean-IDF against hand-worked Figure-2 means, a hand-worked tie at
 N = 16 and brute force over a high-precision evaluation of the real mean
-IDF; evenly spaced chunks against their closed form; the query-host step against masked
+IDF; evenly spaced chunks against their closed form; entropy against its
+closed forms (all distinct, all equal), a hand-worked tie between tf
+multisets {4, 1, 1, 1, 1} and {2, 2, 2, 2}, and brute force over a
+high-precision evaluation; BM25 against hand-worked values (the formulas of
+entropy and BM25 are not on the pages: parity unpinned beyond these); the query-host step against masked
 library attention; ART with zero thresholds against library attention and
 its stop block against a closed form where the weights underflow.
 """
@@ -207,6 +211,121 @@ def select_summaries_mean_idf(ids: np.ndarray, block: int, chunk: int, k: int, v
             rank[j * C + c] = r
         sel[j] = sorted(order[:k])
     return (sel, rank) if return_rank else sel
+
+
+def chunk_entropy(ids: np.ndarray, block: int, chunk: int) -> np.ndarray:
+    """Shannon entropy (natural log) of each chunk's token distribution,
+    H(c) = -sum_t p_t ln p_t with p_t = tf(t, c) / |c|, float64 [N][C].
+    Reading: the pages list entropy among the statistical scorers of §3.1 /
+    Table 1 without a formula; this is the textbook Shannon entropy of the
+    chunk's empirical token frequencies, and chunks of higher entropy are
+    kept.  Parity unpinned beyond the closed forms and hand-worked values in
+    the tests."""
+    blocks = _blocks(ids, block)
+    C = block // chunk
+    out = np.empty((len(blocks), C), dtype=np.float64)
+    for j, blk in enumerate(blocks):
+        for c in range(C):
+            toks = blk[c * chunk:(c + 1) * chunk].tolist()
+            tf = {}
+            for t in toks:
+                tf[t] = tf.get(t, 0) + 1
+            out[j, c] = -math.fsum((n / chunk) * math.log(n / chunk) for n in tf.values())
+    return out
+
+
+def chunk_tf_power_product(ids: np.ndarray, block: int, chunk: int) -> list:
+    """prod_t tf(t, c)^tf(t, c) over the distinct tokens of each chunk, as
+    exact Python integers [N * C].  With a fixed chunk length,
+    H(c) = ln |c| - (1/|c|) ln prod_t tf^tf, so a higher entropy is exactly a
+    smaller product and equal entropies are exactly equal products."""
+    blocks = _blocks(ids, block)
+    C = block // chunk
+    out = []
+    for blk in blocks:
+        for c in range(C):
+            tf = {}
+            for t in blk[c * chunk:(c + 1) * chunk].tolist():
+                tf[t] = tf.get(t, 0) + 1
+            prod = 1
+            for n in tf.values():
+                prod *= n ** n
+            out.append(prod)
+    return out
+
+
+def select_summaries_entropy(ids: np.ndarray, block: int, chunk: int, k: int, return_rank: bool = False):
+    """Top-k chunks per block by entropy (chunk_entropy), exact order
+    (ascending chunk_tf_power_product), equal entropies to the lower index,
+    kept in original order.  Returns int64 [N][k] (and the int64 [N * C]
+    ranks, best first, when ``return_rank``)."""
+    n_blocks = len(ids) // block
+    C = block // chunk
+    if not 0 <= k <= C:
+        raise ValueError("k must be in [0, block/chunk]")
+    prod = chunk_tf_power_product(ids, block, chunk)
+    sel = np.empty((n_blocks, k), dtype=np.int64)
+    rank = np.empty(n_blocks * C, dtype=np.int64)
+    for j in range(n_blocks):
+        order = sorted(range(C), key=lambda c: (prod[j * C + c], c))
+        for r, c in enumerate(order):
+            rank[j * C + c] = r
+        sel[j] = sorted(order[:k])
+    return (sel, rank) if return_rank else sel
+
+
+BM25_K1 = 1.2
+BM25_B = 0.75
+
+
+def chunk_bm25(ids: np.ndarray, block: int, chunk: int, vocab: int) -> np.ndarray:
+    """BM25 weight of each chunk over its own tokens, float64 [N * C] in
+    sequence order: sum over the distinct tokens t of the chunk, in order of
+    their first occurrence, of
+        idf(t) * tf (k1 + 1) / (tf + k1 (1 - b + b |c| / avgdl)),
+        idf(t) = ln(1 + (N - df(t) + 0.5) / (df(t) + 0.5)),
+    with blocks as the documents for df (as for Max-IDF), k1 = 1.2, b = 0.75,
+    and |c| = avgdl = chunk (every chunk has the chunk length).
+    Reading: the pages list BM25 among the statistical scorers of §3.1 /
+    Table 1 without a formula; this is the standard Okapi BM25 term weight
+    (Robertson-Sparck Jones idf with +1 inside the log) summed over the
+    chunk's own terms.  Parity unpinned beyond the hand-worked values in the
+    tests."""
+    n = len(ids) // block
+    df = document_frequency(ids, block, vocab)
+    blocks = _blocks(ids, block)
+    C = block // chunk
+    norm = BM25_K1 * (1.0 - BM25_B + BM25_B * chunk / chunk)
+    out = np.empty(n * C, dtype=np.float64)
+    for j, blk in enumerate(blocks):
+        for c in range(C):
+            tf, order = {}, []
+            for t in blk[c * chunk:(c + 1) * chunk].tolist():
+                if t not in tf:
+                    order.append(t)
+                tf[t] = tf.get(t, 0) + 1
+            total = 0.0
+            for t in order:
+                d = float(df[t])
+                idf = math.log(1.0 + (n - d + 0.5) / (d + 0.5))
+                total += idf * (tf[t] * (BM25_K1 + 1.0)) / (tf[t] + norm)
+            out[j * C + c] = total
+    return out
+
+
+def select_summaries_bm25(ids: np.ndarray, block: int, chunk: int, k: int, vocab: int):
+    """Top-k chunks per block by chunk_bm25 (descending, ties to the lower
+    index), kept in original order.  Returns int64 [N][k]."""
+    n_blocks = len(ids) // block
+    C = block // chunk
+    if not 0 <= k <= C:
+        raise ValueError("k must be in [0, block/chunk]")
+    sc = chunk_bm25(ids, block, chunk, vocab).reshape(n_blocks, C)
+    sel = np.empty((n_blocks, k), dtype=np.int64)
+    for j in range(n_blocks):
+        order = sorted(range(C), key=lambda c: (-sc[j, c], c))
+        sel[j] = sorted(order[:k])
+    return sel
 
 
 # ----------------------------------------------------------------------------

@@ -300,3 +300,81 @@ def test_evenly_spaced_closed_form():
     assert sel.shape == (3, 16) and sel[1].tolist() == list(range(0, 128, 8))
     assert oracle.select_evenly_spaced(1, 96, 32, 3).tolist() == [[0, 1, 2]]
     assert oracle.select_evenly_spaced(2, 320, 32, 3).tolist() == [[0, 3, 6]] * 2
+
+
+# --------------------------------------------------------------------------
+# entropy and BM25 scorers (named on the Pulsar page, §3.1 / Table 1, without
+# formulas: the textbook definitions, pinned by closed forms and hand-worked
+# values)
+# --------------------------------------------------------------------------
+def test_entropy_closed_forms():
+    ids = np.array(list(range(8)) + [5] * 8 + [1, 1, 2, 2, 3, 3, 4, 4] + [9, 9, 9, 9, 1, 2, 3, 4], dtype=np.int64)
+    h = oracle.chunk_entropy(ids, 32, 8)[0]
+    assert abs(h[0] - math.log(8)) < 1e-15           # all distinct: ln |c|
+    assert h[1] == 0.0                               # one token repeated
+    # tf multisets {2, 2, 2, 2} and {4, 1, 1, 1, 1}: ln 8 - (1/8) 4 (2 ln 2)
+    # = ln 8 - (1/8) 4 ln 4 = ln 4, the same real number
+    assert abs(h[2] - math.log(4)) < 1e-15 and abs(h[3] - math.log(4)) < 1e-15
+    prod = oracle.chunk_tf_power_product(ids, 32, 8)
+    assert prod == [1, 8 ** 8, 256, 256]
+
+
+@pytest.mark.parametrize("swap", [False, True])
+def test_entropy_hand_worked_tie_goes_to_the_lower_index(swap):
+    a = [1, 1, 2, 2, 3, 3, 4, 4]
+    b = [9, 9, 9, 9, 1, 2, 3, 4]
+    if swap:
+        a, b = b, a
+    ids = np.array([5] * 8 + a + b + [6, 6, 7, 7, 7, 7, 7, 7], dtype=np.int64)
+    sel, rank = oracle.select_summaries_entropy(ids, 32, 8, 1, return_rank=True)
+    assert sel.tolist() == [[1]]
+    assert rank.tolist() == [3, 0, 1, 2]
+
+
+def _real_entropy_resolved(ids, block, chunk):
+    """-sum p ln p of every chunk to 60 digits; entropies of different tf
+    multisets with c <= 8 tokens differ by more than 1e-16, so values closer
+    than 1e-40 are the same real number (each replaced by the smallest of its
+    group)."""
+    from decimal import Decimal, getcontext
+    getcontext().prec = 60
+    n, C = len(ids) // block, block // chunk
+    rows = []
+    for j in range(n):
+        vals = []
+        for c in range(C):
+            toks = ids[j * block + c * chunk:j * block + (c + 1) * chunk].tolist()
+            tot = Decimal(0)
+            for t in set(toks):
+                p = Decimal(toks.count(t)) / Decimal(chunk)
+                tot -= p * p.ln()
+            vals.append(tot)
+        srt = sorted(vals)
+        rows.append([next(w for w in srt if abs(w - v) < Decimal("1e-40")) for v in vals])
+    return rows
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_entropy_brute_force_real_order(seed):
+    rng = np.random.default_rng(70 + seed)
+    block, chunk = 64, 8
+    ids = rng.integers(0, 6, size=block * 3)        # few distinct ids: many equal entropies
+    real = _real_entropy_resolved(ids, block, chunk)
+    C = block // chunk
+    for k in (1, 3, 6):
+        sel = oracle.select_summaries_entropy(ids, block, chunk, k)
+        for j in range(3):
+            assert sel[j].tolist() == _brute_force_topk(real[j], k)
+
+
+def test_bm25_hand_worked():
+    # N = 2 blocks of 4 ids, 2-token chunks: df(1) = df(3) = df(4) = 1,
+    # df(2) = 2; idf = ln(1 + (N - df + 0.5)/(df + 0.5)): ln 2 for df 1,
+    # ln 1.2 for df 2; tf weight tf (k1 + 1)/(tf + k1) with k1 = 1.2: 1 for
+    # tf 1, 4.4 / 3.2 = 1.375 for tf 2.
+    ids = np.array([1, 1, 2, 3, 2, 4, 4, 4], dtype=np.int64)
+    got = oracle.chunk_bm25(ids, 4, 2, 5)
+    l2, l12 = math.log(2.0), math.log(1.2)
+    want = [1.375 * l2, l12 + l2, l12 + l2, 1.375 * l2]
+    assert np.allclose(got, want, rtol=0, atol=1e-15)
+    assert oracle.select_summaries_bm25(ids, 4, 2, 1, 5).tolist() == [[0], [1]]
