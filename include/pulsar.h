@@ -126,7 +126,9 @@ int pulsar_select_summaries(const int32_t* ids, int64_t L, int32_t vocab, int32_
 typedef enum {
   PA_SCORE_MAX_IDF = 0,       /* the method: max IDF over the chunk (= pulsar_select_summaries) */
   PA_SCORE_MEAN_IDF = 1,      /* mean IDF over the chunk's tokens */
-  PA_SCORE_EVENLY_SPACED = 2  /* no score: chunks floor(m * C / k), m = 0..k-1, in every block */
+  PA_SCORE_EVENLY_SPACED = 2, /* no score: chunks floor(m * C / k), m = 0..k-1, in every block */
+  PA_SCORE_ENTROPY = 3,       /* Shannon entropy of the chunk's token frequencies */
+  PA_SCORE_BM25 = 4           /* Okapi BM25 weight of the chunk over its own tokens */
 } pa_score_method;
 
 /*
@@ -140,12 +142,22 @@ typedef enum {
  *    integer product of df over the chunk (ascending), compared as exact
  *    256-bit integers; equal means go to the lower chunk index.  Requires
  *    chunk <= 32 and block / chunk <= 4096 (PA_ERR_UNSUPPORTED otherwise).
+ *  - PA_SCORE_ENTROPY ranks chunks by -sum_t p_t ln p_t, p_t = tf(t) /
+ *    chunk, exactly: the order is that of the integer prod_t tf^tf
+ *    (ascending), compared as 256-bit integers.  Same limits as mean IDF.
+ *  - PA_SCORE_BM25 ranks chunks by sum over their distinct tokens (in order
+ *    of first occurrence) of ln(1 + (N - df + 0.5)/(df + 0.5)) *
+ *    tf (k1 + 1)/(tf + k1), k1 = 1.2 (length normalisation 1: every chunk
+ *    has the average length), in fp64; equal scores go to the lower index.
+ *    Same limits as mean IDF.  (The pages name entropy and BM25 without
+ *    formulas; these are the textbook definitions.)
  *  - PA_SCORE_EVENLY_SPACED does not read ids (may be NULL).
- *  chunk_score_opt  out [L / chunk] int64, or NULL: for PA_SCORE_MEAN_IDF
- *                   each chunk's rank in its block's order (0 = highest
- *                   mean IDF; the ranks of a block are a permutation of
- *                   0 .. block/chunk - 1); for PA_SCORE_MAX_IDF the min df;
- *                   not written for PA_SCORE_EVENLY_SPACED.
+ *  chunk_score_opt  out [L / chunk] int64, or NULL: for PA_SCORE_MEAN_IDF,
+ *                   PA_SCORE_ENTROPY and PA_SCORE_BM25 each chunk's rank in
+ *                   its block's order (0 = best; the ranks of a block are a
+ *                   permutation of 0 .. block/chunk - 1); for
+ *                   PA_SCORE_MAX_IDF the min df; not written for
+ *                   PA_SCORE_EVENLY_SPACED.
  * Workspace: pa_select_workspace_size.
  */
 int pulsar_select_summaries_scored(const int32_t* ids, int64_t L, int32_t vocab, int32_t block,
@@ -314,6 +326,10 @@ size_t pa_phase2_workspace_size(int32_t B, int32_t Tq, int64_t T, int32_t n_shar
  *
  * An empty shard has s_h = -inf and A_h = 0; with T == 0, O = 0 and
  * lse = -inf.  d must be 64 or 128, hq % hkv == 0, 1 <= n_shards <= 4096.
+ * When neither partial output is asked for and a kv head has more than 8
+ * query rows, the work is cut into equal key ranges regardless of shard
+ * boundaries (the merge is exact either way; results differ only in fp32
+ * rounding order).
  * Precision (bf16): on the tensor-core path (at least 64 query rows per kv
  * head, Tq * hq / hkv; hq / hkv dividing 128; 16-byte aligned caches) the
  * scores are computed from the rotated query rounded to fp16 against the

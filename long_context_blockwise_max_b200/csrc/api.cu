@@ -242,16 +242,17 @@ int pulsar_select_summaries_scored(const int32_t* ids, int64_t L, int32_t vocab,
                                    int64_t* chunk_score_opt, void* ws, size_t ws_bytes,
                                    void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (method != PA_SCORE_MAX_IDF && method != PA_SCORE_MEAN_IDF && method != PA_SCORE_EVENLY_SPACED)
+  if (method != PA_SCORE_MAX_IDF && method != PA_SCORE_MEAN_IDF && method != PA_SCORE_EVENLY_SPACED &&
+      method != PA_SCORE_ENTROPY && method != PA_SCORE_BM25)
     return PA_ERR_INVALID;
+  const bool ranked = method == PA_SCORE_MEAN_IDF || method == PA_SCORE_ENTROPY || method == PA_SCORE_BM25;
   if (L <= 0 || vocab <= 0 || block <= 0 || chunk <= 0) return PA_ERR_INVALID;
   if (L % block != 0 || block % chunk != 0) return PA_ERR_INVALID;
   if (k_chunks < 0 || k_chunks > block / chunk) return PA_ERR_INVALID;
   if ((ids == nullptr && method != PA_SCORE_EVENLY_SPACED) || (sel == nullptr && k_chunks > 0))
     return PA_ERR_INVALID;
   if (L / block > kMaxBlocks) return PA_ERR_UNSUPPORTED;
-  if (method == PA_SCORE_MEAN_IDF && (block / chunk > kMaxScoredChunks || chunk > kMaxScoredChunk))
-    return PA_ERR_UNSUPPORTED;
+  if (ranked && (block / chunk > kMaxScoredChunks || chunk > kMaxScoredChunk)) return PA_ERR_UNSUPPORTED;
   const size_t need = pa_select_workspace_size(L, vocab, block, chunk);
   int rc = check_ws(ws, ws_bytes, need);
   if (rc) return rc;
@@ -413,8 +414,9 @@ int star_phase2_attend(const void* q, int dtype, int32_t B, int32_t Tq, int64_t 
   a.dtype = dtype;
   a.q = q; a.B = B; a.Tq = Tq; a.q_pos0 = q_pos0; a.rope_theta = rope_theta;
   a.k_ret = k_ret; a.v_ret = v_ret; a.T = T;
-  a.n_shards = n_shards;
-  a.n_split = phase2_split(B, Tq, T, n_shards, hq, hkv);
+  // without per-shard partials the units need not follow shard boundaries
+  a.n_shards = phase2_flat_units(Tq, hq, hkv, part_o_opt || part_lse_opt) ? 1 : n_shards;
+  a.n_split = phase2_split(B, Tq, T, a.n_shards, hq, hkv);
   a.hq = hq; a.hkv = hkv; a.d = d;
   a.o = o; a.lse = lse; a.part_o_opt = part_o_opt; a.part_lse_opt = part_lse_opt;
   carve_phase2(a, ws);
@@ -510,8 +512,9 @@ int star_phase2_query_step(const void* q, const void* k_new, const void* v_new, 
   a.dtype = dtype;
   a.q = q; a.B = B; a.Tq = Tq; a.q_pos0 = q_pos0; a.rope_theta = rope_theta;
   a.k_ret = k_ret; a.v_ret = v_ret; a.T = T;
-  a.n_shards = n_shards;
-  a.n_split = phase2_split(B, Tq, T, n_shards, hq, hkv);
+  // no per-shard partials: the context's units need not follow shard boundaries
+  a.n_shards = phase2_flat_units(Tq, hq, hkv, false) ? 1 : n_shards;
+  a.n_split = phase2_split(B, Tq, T, a.n_shards, hq, hkv);
   a.hq = hq; a.hkv = hkv; a.d = d;
   a.o = o; a.lse = lse; a.part_o_opt = nullptr; a.part_lse_opt = nullptr;
   a.k_self = k_self; a.v_self = v_self; a.self_cap = self_cap; a.self_len = self_len;

@@ -201,6 +201,14 @@ __global__ void __launch_bounds__(THREADS) topk_kernel(const int32_t* __restrict
 //    0..C-1); a chunk is kept when its rank is below k.  Without a rank
 //    output the count stops at k.
 //  select_by_rank_kernel: ordered compaction of the chunks with rank < k.
+//  Entropy.  With a fixed chunk length c, H = ln c - (1/c) sum_t tf ln tf, so
+//    a higher entropy is exactly a smaller prod_t tf^tf, and that product is
+//    the product over the chunk's positions of their token's frequency in
+//    the chunk (a 256-bit key as above, __match_any_sync counting).
+//  BM25.  fp64 sum over the chunk's distinct tokens, in order of first
+//    occurrence, of idf(df) * tf (k1 + 1) / (tf + k1), k1 = 1.2 (the length
+//    normalisation is 1: every chunk has the average length); ranked by
+//    that score, descending.
 //  evenly_spaced_kernel: chunk floor(m * C / k) in every block.
 // ---------------------------------------------------------------------------
 struct Key256 {
@@ -260,23 +268,88 @@ __global__ void chunk_df_product_kernel(const int32_t* __restrict__ ids, int64_t
   }
 }
 
+// chunk entropy key: prod over the chunk's positions of tf(token) (= prod_t tf^tf)
+__global__ void chunk_tf_product_kernel(const int32_t* __restrict__ ids, int64_t n_chunks, int32_t chunk,
+                                        Key256* __restrict__ key) {
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t c = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; c < n_chunks;
+       c += nwarps) {
+    // lanes past the chunk get keys no token has, and contribute 1
+    const int t = lane < chunk ? ids[c * chunk + lane] : 0;
+    const unsigned long long tk = lane < chunk ? (unsigned long long)(unsigned)t
+                                               : (0x100000000ull | (unsigned)lane);
+    const unsigned peers = __match_any_sync(0xffffffffu, tk);
+    unsigned long long f = lane < chunk ? (unsigned long long)__popc(peers) : 1ull;
+#pragma unroll
+    for (int off = 1; off < 8; off <<= 1) f *= __shfl_xor_sync(0xffffffffu, f, off);
+    const unsigned long long p8 = __shfl_sync(0xffffffffu, f, 8);
+    const unsigned long long p16 = __shfl_sync(0xffffffffu, f, 16);
+    const unsigned long long p24 = __shfl_sync(0xffffffffu, f, 24);
+    if (lane == 0) {
+      Key256 k;
+      k.w[0] = f;
+      k.w[1] = k.w[2] = k.w[3] = 0;
+      key_mul_small(k, p8);
+      key_mul_small(k, p16);
+      key_mul_small(k, p24);
+      key[c] = k;
+    }
+  }
+}
+
+// chunk BM25 score (fp64), summed in lane order over first occurrences
+__global__ void chunk_bm25_kernel(const int32_t* __restrict__ ids, int64_t n_chunks, int32_t chunk, int32_t vocab,
+                                  int32_t n_blocks, const unsigned long long* __restrict__ mask,
+                                  double* __restrict__ score) {
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  constexpr double k1 = 1.2;
+  for (int64_t c = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; c < n_chunks;
+       c += nwarps) {
+    const int t = lane < chunk ? ids[c * chunk + lane] : 0;
+    const unsigned long long tk = lane < chunk ? (unsigned long long)(unsigned)t
+                                               : (0x100000000ull | (unsigned)lane);
+    const unsigned peers = __match_any_sync(0xffffffffu, tk);
+    double term = 0.0;
+    if (lane < chunk && lane == __ffs(peers) - 1 && t >= 0 && t < vocab) {
+      const double d = (double)__popcll(mask[t]);
+      const double tf = (double)__popc(peers);
+      const double idf = log(1.0 + ((double)n_blocks - d + 0.5) / (d + 0.5));
+      term = idf * (tf * (k1 + 1.0)) / (tf + k1);
+    }
+    double total = 0.0;
+    for (int l = 0; l < 32; ++l) total += __shfl_sync(0xffffffffu, term, l);   // lane order
+    if (lane == 0) score[c] = total;
+  }
+}
+
+// a better than b: a smaller 256-bit key (mean IDF, entropy) ...
+__device__ __forceinline__ bool key_better(const Key256& a, const Key256& b) { return key_less(a, b); }
+__device__ __forceinline__ bool key_same(const Key256& a, const Key256& b) { return key_equal(a, b); }
+// ... or a larger score (BM25)
+__device__ __forceinline__ bool key_better(double a, double b) { return a > b; }
+__device__ __forceinline__ bool key_same(double a, double b) { return a == b; }
+
 // grid (ceil(C / 256), n_blocks); the block's keys are staged in shared memory.
-__global__ void __launch_bounds__(256) rank_kernel(const Key256* __restrict__ key, int32_t C, int32_t k,
+template <typename K>
+__global__ void __launch_bounds__(256) rank_kernel(const K* __restrict__ key, int32_t C, int32_t k,
                                                    int32_t* __restrict__ rank,
                                                    long long* __restrict__ rank_out) {
-  extern __shared__ Key256 sk[];
+  extern __shared__ __align__(16) uint8_t sk_raw[];
+  K* sk = reinterpret_cast<K*>(sk_raw);
   const int j = blockIdx.y;
-  const Key256* kb = key + (int64_t)j * C;
+  const K* kb = key + (int64_t)j * C;
   for (int o = threadIdx.x; o < C; o += blockDim.x) sk[o] = kb[o];
   __syncthreads();
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
   if (c >= C) return;
-  const Key256 v = sk[c];
+  const K v = sk[c];
   const int stop = rank_out != nullptr ? C : k;   // the count only decides rank < k
   int better = 0;
   for (int o = 0; o < C && better < stop; ++o) {
-    const Key256 w = sk[o];
-    better += key_less(w, v) || (o < c && key_equal(w, v));
+    const K w = sk[o];
+    better += key_better(w, v) || (o < c && key_same(w, v));
   }
   rank[(int64_t)j * C + c] = better;
   if (rank_out != nullptr) rank_out[(int64_t)j * C + c] = better;
@@ -345,19 +418,34 @@ int launch_select_scored(const SelectArgs& a, int method, void* key_ws, long lon
     }
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
   }
-  int rc = launch_presence(a, s);
+  int rc = method == PA_SCORE_ENTROPY ? PA_OK : launch_presence(a, s);
   if (rc) return rc;
-  Key256* key = static_cast<Key256*>(key_ws);
   const int threads = 256;
   const int64_t wgrid = (n_chunks * 32 + threads - 1) / threads;
-  chunk_df_product_kernel<<<(int)(wgrid < 148 * 32 ? wgrid : 148 * 32), threads, 0, s>>>(
-      a.ids, n_chunks, a.chunk, a.vocab, a.mask, key);
+  const int wblocks = (int)(wgrid < 148 * 32 ? wgrid : 148 * 32);
+  if (method == PA_SCORE_MEAN_IDF)
+    chunk_df_product_kernel<<<wblocks, threads, 0, s>>>(a.ids, n_chunks, a.chunk, a.vocab, a.mask,
+                                                        static_cast<Key256*>(key_ws));
+  else if (method == PA_SCORE_ENTROPY)
+    chunk_tf_product_kernel<<<wblocks, threads, 0, s>>>(a.ids, n_chunks, a.chunk, static_cast<Key256*>(key_ws));
+  else
+    chunk_bm25_kernel<<<wblocks, threads, 0, s>>>(a.ids, n_chunks, a.chunk, a.vocab, n_blocks, a.mask,
+                                                  static_cast<double*>(key_ws));
   if (a.k > 0 || rank_out != nullptr) {
-    const size_t sm = sizeof(Key256) * (size_t)C;
-    if (cudaFuncSetAttribute(rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) != cudaSuccess)
-      return PA_ERR_CUDA;
     const dim3 grid((unsigned)((C + 255) / 256), (unsigned)n_blocks);
-    rank_kernel<<<grid, 256, sm, s>>>(key, C, a.k, a.mindf, rank_out);
+    if (method == PA_SCORE_BM25) {
+      const size_t sm = sizeof(double) * (size_t)C;
+      if (cudaFuncSetAttribute(rank_kernel<double>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) !=
+          cudaSuccess)
+        return PA_ERR_CUDA;
+      rank_kernel<double><<<grid, 256, sm, s>>>(static_cast<double*>(key_ws), C, a.k, a.mindf, rank_out);
+    } else {
+      const size_t sm = sizeof(Key256) * (size_t)C;
+      if (cudaFuncSetAttribute(rank_kernel<Key256>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) !=
+          cudaSuccess)
+        return PA_ERR_CUDA;
+      rank_kernel<Key256><<<grid, 256, sm, s>>>(static_cast<Key256*>(key_ws), C, a.k, a.mindf, rank_out);
+    }
   }
   if (a.k > 0) select_by_rank_kernel<1024><<<n_blocks, 1024, 0, s>>>(a.mindf, C, a.k, a.sel);
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;

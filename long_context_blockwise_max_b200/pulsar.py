@@ -17,7 +17,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libpulsar_b200.so")
 
 PA_F32, PA_BF16 = 0, 1
-PA_SCORE_MAX_IDF, PA_SCORE_MEAN_IDF, PA_SCORE_EVENLY_SPACED = 0, 1, 2
+PA_SCORE_MAX_IDF, PA_SCORE_MEAN_IDF, PA_SCORE_EVENLY_SPACED, PA_SCORE_ENTROPY, PA_SCORE_BM25 = 0, 1, 2, 3, 4
 _STATUS = {0: "PA_OK", -1: "PA_ERR_INVALID", -2: "PA_ERR_UNSUPPORTED", -3: "PA_ERR_WORKSPACE",
            -4: "PA_ERR_CUDA", -5: "PA_ERR_TIMEOUT", -6: "PA_ERR_RANGE"}
 
@@ -243,7 +243,7 @@ def pulsar_select_summaries_scored(ids, vocab: int, block: int, chunk: int, k_ch
     """Selection with another chunk scorer (PA_SCORE_*).  ``ids`` may be None
     for PA_SCORE_EVENLY_SPACED (then pass ``L``).  Returns (sel, scores or
     None, ws); with ``want_scores`` the int64 scores are each chunk's rank in
-    its block (mean IDF) or its min df (max IDF)."""
+    its block (mean IDF, entropy, BM25) or its min df (max IDF)."""
     _dev(ids, sel)
     L = ids.numel() if ids is not None else int(L)
     dev = ids.device if ids is not None else torch.device("cuda", torch.cuda.current_device())

@@ -144,7 +144,7 @@ def test_host_validation_of_the_other_entry_points(lib):
     assert so.pa_set_profile_events(None, None) == 0
     # scorer: unknown method; missing ids for a scorer that reads them; mean-IDF beyond 4096 chunks per
     # block or beyond 32 tokens per chunk (the exact 256-bit product)
-    assert so.pulsar_select_summaries_scored(dummy, 1024, 100, 512, 32, 2, 3, dummy, None, ws, 1 << 20,
+    assert so.pulsar_select_summaries_scored(dummy, 1024, 100, 512, 32, 2, 5, dummy, None, ws, 1 << 20,
                                              None) == -1
     assert so.pulsar_select_summaries_scored(None, 1024, 100, 512, 32, 2, 1, dummy, None, ws, 1 << 20,
                                              None) == -1
@@ -152,6 +152,9 @@ def test_host_validation_of_the_other_entry_points(lib):
                                              None) == -2
     assert so.pulsar_select_summaries_scored(dummy, 4096, 100, 1024, 64, 1, 1, dummy, None, ws, 1 << 30,
                                              None) == -2
+    for method in (3, 4):   # entropy and BM25: the same limits as mean IDF
+        assert so.pulsar_select_summaries_scored(dummy, 4096, 100, 1024, 64, 1, method, dummy, None, ws, 1 << 30,
+                                                 None) == -2
 
     def art(dtype=1, Tq=1, hq=32, hkv=8, block_keys=128, tau=1e-5, phi=1e-3, patience=5, theta=5e5):
         return so.star_phase2_attend_art(dummy, dtype, 2, Tq, 1000, theta, dummy, dummy, 1000, hq, hkv, 128,

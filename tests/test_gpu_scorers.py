@@ -1,8 +1,9 @@
 """GPU parity of the alternative summary scorers (Pulsar Attention page
-§3.1, Table 1): mean-IDF (exact order, ties to the lower index) and evenly
-spaced sampling, bit-exact against the oracle -- the selection and every
-chunk's rank; Max-IDF through the scored entry point against the oracle's
-selection and min df."""
+§3.1, Table 1): mean-IDF and entropy (exact orders, ties to the lower index)
+and evenly spaced sampling, bit-exact against the oracle -- the selection and
+every chunk's rank; BM25 (fp64) against the oracle's order except among
+scores equal to fp64 rounding; Max-IDF through the scored entry point
+against the oracle's selection and min df."""
 import json
 import os
 
@@ -43,6 +44,32 @@ def _cases():
 N_CASES = 9
 
 
+def _check_bm25(P, dev_ids, ids, vocab, block, chunk, k):
+    """BM25 is an fp64 score (the kernel's and the oracle's logarithms may
+    differ in the last bit): every chunk's rank must equal the oracle's
+    unless its score is within 1e-12 (relative) of another chunk's of the
+    same block, where only the order among those near-equal chunks may
+    differ; the selection must be the oracle's unless the k-th and (k+1)-th
+    best scores are within 1e-12."""
+    sel, rank, ws = P.pulsar_select_summaries_scored(dev_ids, vocab, block, chunk, k, P.PA_SCORE_BM25,
+                                                    want_scores=True)
+    assert P.pa_workspace_status(ws) == 0
+    n, C = ids.size // block, block // chunk
+    sc = oracle.chunk_bm25(ids, block, chunk, vocab).reshape(n, C)
+    want_sel = oracle.select_summaries_bm25(ids, block, chunk, k, vocab)
+    got_rank = rank.cpu().numpy().reshape(n, C)
+    got_sel = sel.cpu().numpy()
+    for j in range(n):
+        order = sorted(range(C), key=lambda c: (-sc[j, c], c))
+        near = lambda a, b: abs(a - b) <= 1e-12 * max(abs(a), abs(b), 1.0)
+        for r, c in enumerate(order):
+            if got_rank[j, c] != r:   # allowed only inside a group of near-equal scores
+                assert near(sc[j, c], sc[j, order[got_rank[j, c]]]), (j, c, r, got_rank[j, c])
+        if 0 < k < C and near(sc[j, order[k - 1]], sc[j, order[k]]):
+            continue
+        assert got_sel[j].tolist() == want_sel[j].tolist(), j
+
+
 @pytest.mark.parametrize("idx", range(N_CASES))
 def test_mean_idf_and_evenly_spaced(P, idx):
     ids, vocab, block, chunk, k = list(_cases())[idx]
@@ -59,6 +86,14 @@ def test_mean_idf_and_evenly_spaced(P, idx):
     sel2, _, _ = P.pulsar_select_summaries_scored(None, vocab, block, chunk, k, P.PA_SCORE_EVENLY_SPACED,
                                                  L=ids.size)
     assert np.array_equal(sel2.cpu().numpy(), oracle.select_evenly_spaced(ids.size // block, block, chunk, k))
+    # entropy: exact order (integer prod tf^tf), bit-exact selection and ranks
+    sel_e, rank_e, ws = P.pulsar_select_summaries_scored(dev_ids, vocab, block, chunk, k, P.PA_SCORE_ENTROPY,
+                                                        want_scores=True)
+    assert P.pa_workspace_status(ws) == 0
+    want_e, want_re = oracle.select_summaries_entropy(ids, block, chunk, k, return_rank=True)
+    assert np.array_equal(rank_e.cpu().numpy(), want_re)
+    assert np.array_equal(sel_e.cpu().numpy(), want_e)
+    _check_bm25(P, dev_ids, ids, vocab, block, chunk, k)
     sel3, sc3, _ = P.pulsar_select_summaries_scored(dev_ids, vocab, block, chunk, k, P.PA_SCORE_MAX_IDF,
                                                    want_scores=True)
     df = oracle.document_frequency(ids, block, vocab)
