@@ -316,10 +316,22 @@ int32_t phase2_split(int32_t B, int32_t Tq, int64_t T, int32_t n_shards, int32_t
   return (int32_t)best;
 }
 
+// Work units of the context: by shard (a shard cut into phase2_split
+// splits), or -- many query rows and no per-shard partials asked for -- the
+// whole cache as one range cut into equal units, so that units need not
+// follow shard boundaries and fill the SMs more evenly (the exact merge does
+// not depend on where the units are cut).
+bool phase2_flat_units(int32_t Tq, int32_t hq, int32_t hkv, bool want_partials) {
+  return !want_partials && (int64_t)Tq * (hq / hkv) > 8;
+}
+
 size_t phase2_workspace_bytes(int32_t B, int32_t Tq, int64_t T, int32_t n_shards, int32_t hq,
                               int32_t hkv, int32_t d) {
   const int32_t ns = phase2_split(B, Tq, T, n_shards, hq, hkv);
-  const size_t units = (size_t)n_shards * ns + 1;   // + the query host's own cache
+  const int32_t ns_flat = phase2_split(B, Tq, T, 1, hq, hkv);
+  size_t units = (size_t)n_shards * ns;
+  if ((size_t)ns_flat > units) units = ns_flat;
+  units += 1;                                       // + the query host's own cache
   const size_t rows = (size_t)B * Tq * hq;
   size_t b = kStatusBytes;
   b += align_up(sizeof(float) * rows * d);          // rotated query
