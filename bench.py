@@ -655,6 +655,7 @@ def run_ours(args, rank, world, local_rank, dist_on):
             sws = torch.empty(P.pa_select_workspace_size(wl.L, wl.vocab, wl.block, wl.chunk), dtype=torch.uint8,
                               device=dev)
             for name, method in (("max_idf", P.PA_SCORE_MAX_IDF), ("mean_idf", P.PA_SCORE_MEAN_IDF),
+                                 ("entropy", P.PA_SCORE_ENTROPY), ("bm25", P.PA_SCORE_BM25),
                                  ("evenly_spaced", P.PA_SCORE_EVENLY_SPACED)):
                 def sel_call():
                     P.pulsar_select_summaries_scored(idd, wl.vocab, wl.block, wl.chunk, wl.k_chunks, method,
@@ -738,7 +739,7 @@ def run_ours(args, rank, world, local_rank, dist_on):
 # --------------------------------------------------------------------------
 # the oracle on the host cores (cpu_baseline leg and --impl reference)
 # --------------------------------------------------------------------------
-ORACLE_SAMPLE_ROWS = 384   # Phase-1 rows of the last host timed on the host cores (about 9 s on 16 cores)
+ORACLE_SAMPLE_ROWS = 512   # Phase-1 rows of the last host timed on the host cores (about 7 s on 16 cores)
 
 
 def _oracle_threads():
