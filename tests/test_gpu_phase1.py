@@ -124,8 +124,9 @@ def test_bf16_running_max_jumps_mid_sequence(P, star):
     # with p = 3 (mod 4), score the keys before that point about 7 nat lower
     # through sixteen of the slowest-turning RoPE dimensions.  Their running
     # max therefore jumps by more than 2^8 at key tile 1 or 2, which takes the
-    # lazy-rescale branch (half a tile recomputed, O rescaled) for some rows of
-    # every warp while the others keep their max.  The jump comes from pushing
+    # lazy-rescale branch (the running max moves and O in TMEM is rescaled
+    # before the next PV) for some rows of every warp while the others keep
+    # their max.  The jump comes from pushing
     # early keys down, so the dominant scores stay small and the fp16 operand
     # rounding stays well inside the lse tolerance.
     L, block, theta, a = 2 * 512, 512, 500000.0, 5.0
