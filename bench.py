@@ -378,7 +378,9 @@ def run_ours(args, rank, world, local_rank, dist_on):
     flops = attn_flops(w, hosts=(h0, h1))
     # whole job: one sequence per rank, or one sequence spread over the ranks
     tokens_per_s = w.L / (ms * 1e-3) if hosts_layout else whole_job_rate(w.L, world, ms)
-    peak_tf = peaks["bf16_tflops_sustained"]
+    # the burst peak: the timed region is a fraction of a second, not the
+    # seconds-long loop the sustained figure was measured over
+    peak_tf = peaks["bf16_tflops"]
     attn_tf = flops / (attn_ms * 1e-3) / 1e12
 
     # ---- end to end through the public API with host buffers ------------
@@ -690,9 +692,9 @@ def run_ours(args, rank, world, local_rank, dist_on):
 
     q2_bytes = 2.0 * w.L * w.hkv * w.d * 2
     # the query's roofline: the slower of streaming K/V at the measured copy
-    # bandwidth and its QK^T + PV work at the measured sustained bf16 peak
+    # bandwidth and its QK^T + PV work at the measured burst bf16 peak
     q2_roof_ms = max(q2_bytes / (peaks["hbm_gbs"] * 1e9),
-                     4.0 * w.d * w.hq * w.q_tokens * w.L / (peaks["bf16_tflops_sustained"] * 1e12)) * 1e3
+                     4.0 * w.d * w.hq * w.q_tokens * w.L / (peaks["bf16_tflops"] * 1e12)) * 1e3
     clocks = clk.summary()
     line = {
         "metric": METRIC, "value": round(tokens_per_s, 1), "unit": "tokens/s", "n_gpus": world,
@@ -713,11 +715,11 @@ def run_ours(args, rank, world, local_rank, dist_on):
         "gpu_launches": step.launches() * K,
         "roofline": {"bound": "tensor", "kernel": "phase-1 attention", "achieved": round(attn_tf, 1),
                      "peak": peak_tf, "unit": "TFLOP/s", "frac": round(attn_tf / peak_tf, 4),
-                     "peak_kind": f"{peak_kind} bf16 sustained",
+                     "peak_kind": f"{peak_kind} bf16 burst",
                      "traffic": recorded_traffic("phase1_tc_kernel", w.name),
                      "kernel_ms": round(attn_ms, 3), "flop_per_launch": flops,
                      "frac_of_nominal_dense_bf16": round(attn_tf / NOMINAL_BF16_TFLOPS, 4),
-                     "frac_of_burst": round(attn_tf / peaks["bf16_tflops"], 4)},
+                     "frac_of_sustained": round(attn_tf / peaks["bf16_tflops_sustained"], 4)},
         "phase1_encode": {"selection_ms": round(sel_ms, 4), "encode_ms": round(enc_ms, 3),
                           "tokens_per_s": round(w.L / (enc_ms * 1e-3), 1),
                           "with_selection_tokens_per_s": round(w.L / ((sel_ms + enc_ms) * 1e-3), 1),
