@@ -76,13 +76,15 @@ __global__ void __launch_bounds__(256) presence_tile_kernel(const int32_t* __res
     if (ok && lane == __ffs(peers) - 1) atomicOr(&bm[t >> 5], 1u << (t & 31));
   }
   __syncthreads();
+  // one atomic OR per distinct id of the tile; its result is unused, so it is
+  // issued without waiting for it and the tile's ORs overlap in flight
   const unsigned long long bit = 1ull << j;
   for (int w = threadIdx.x; w < words; w += blockDim.x) {
     uint32_t x = bm[w];
     while (x) {
       const int t = (w << 5) + __ffs(x) - 1;
       x &= x - 1u;
-      if (!(ld_cg_u64(mask + t) & bit)) atomicOr(mask + t, bit);
+      atomicOr(mask + t, bit);
     }
   }
 }
