@@ -326,10 +326,10 @@ size_t pa_phase2_workspace_size(int32_t B, int32_t Tq, int64_t T, int32_t n_shar
  *
  * An empty shard has s_h = -inf and A_h = 0; with T == 0, O = 0 and
  * lse = -inf.  d must be 64 or 128, hq % hkv == 0, 1 <= n_shards <= 4096.
- * When neither partial output is asked for and a kv head has more than 8
- * query rows, the work is cut into equal key ranges regardless of shard
- * boundaries (the merge is exact either way; results differ only in fp32
- * rounding order).
+ * When neither partial output is asked for and the query has more than 8
+ * rows per kv head, or B * n_shards * hkv < 148, the work is cut into equal
+ * key ranges regardless of shard boundaries (the merge is exact either way;
+ * results differ only in fp32 rounding order).
  * Precision (bf16): on the tensor-core path (at least 64 query rows per kv
  * head, Tq * hq / hkv; hq / hkv dividing 128; 16-byte aligned caches) the
  * scores are computed from the rotated query rounded to fp16 against the

@@ -415,7 +415,7 @@ int star_phase2_attend(const void* q, int dtype, int32_t B, int32_t Tq, int64_t 
   a.q = q; a.B = B; a.Tq = Tq; a.q_pos0 = q_pos0; a.rope_theta = rope_theta;
   a.k_ret = k_ret; a.v_ret = v_ret; a.T = T;
   // without per-shard partials the units need not follow shard boundaries
-  a.n_shards = phase2_flat_units(Tq, hq, hkv, part_o_opt || part_lse_opt) ? 1 : n_shards;
+  a.n_shards = phase2_flat_units(B, Tq, n_shards, hq, hkv, part_o_opt || part_lse_opt) ? 1 : n_shards;
   a.n_split = phase2_split(B, Tq, T, a.n_shards, hq, hkv);
   a.hq = hq; a.hkv = hkv; a.d = d;
   a.o = o; a.lse = lse; a.part_o_opt = part_o_opt; a.part_lse_opt = part_lse_opt;
@@ -513,7 +513,7 @@ int star_phase2_query_step(const void* q, const void* k_new, const void* v_new, 
   a.q = q; a.B = B; a.Tq = Tq; a.q_pos0 = q_pos0; a.rope_theta = rope_theta;
   a.k_ret = k_ret; a.v_ret = v_ret; a.T = T;
   // no per-shard partials: the context's units need not follow shard boundaries
-  a.n_shards = phase2_flat_units(Tq, hq, hkv, false) ? 1 : n_shards;
+  a.n_shards = phase2_flat_units(B, Tq, n_shards, hq, hkv, false) ? 1 : n_shards;
   a.n_split = phase2_split(B, Tq, T, a.n_shards, hq, hkv);
   a.hq = hq; a.hkv = hkv; a.d = d;
   a.o = o; a.lse = lse; a.part_o_opt = nullptr; a.part_lse_opt = nullptr;

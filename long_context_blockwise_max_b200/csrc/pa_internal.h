@@ -171,7 +171,7 @@ __device__ inline UnitView phase2_unit(const Phase2Args& a, int u) {
   return v;
 }
 int launch_phase2_mma(const Phase2Args& a, cudaStream_t s);
-bool phase2_flat_units(int32_t Tq, int32_t hq, int32_t hkv, bool want_partials);
+bool phase2_flat_units(int32_t B, int32_t Tq, int32_t n_shards, int32_t hq, int32_t hkv, bool want_partials);
 // Tensor-core (tcgen05) kernel for queries with at least kPhase2TcMinRows rows
 // per kv head; q16 is the rotated query scaled to log2 units, in fp16.
 constexpr int kPhase2TcMinRows = 64;
