@@ -14,14 +14,16 @@ shards (GB/s against HBM).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-With N > 1 (torchrun, one process per GPU) every rank encodes its own
-independent sequence (weak scaling, no data-path collective); the time is the
-max over ranks.  `--layout hosts` runs the method's own multi-GPU layout
-instead: the 8 hosts of ONE sequence spread over the ranks (Phase 1 without
+With N > 1 (torchrun, one process per GPU) the default is the method's own
+multi-GPU layout (`--layout hosts`): the 8 hosts of ONE sequence spread over
+the ranks in contiguous ranges balanced by attention work (Phase 1 without
 communication), then the Phase-2 exchange -- every rank's shard partials
-all-gathered over NCCL and merged exactly (strong scaling; on one GPU the
-exchange runs in a process group of one rank).  `--impl reference` times
-the fp64 CPU oracle on a fixed sample of the same step (rank 0 only).
+all-gathered over NCCL and merged exactly (strong scaling); the time is the
+max over ranks.  `--layout sequences` gives every rank its own independent
+sequence instead (weak scaling, no data-path collective); on one GPU the two
+are the same work and `sequences` is the default (`--layout hosts` then runs
+the exchange in a process group of one rank).  `--impl reference` times the
+fp64 CPU oracle on a fixed sample of the same step (rank 0 only).
 """
 from __future__ import annotations
 
@@ -160,10 +162,11 @@ class ClockSampler:
 class Step:
     """Preallocated buffers and the calls of one hot-path step.
 
-    ``hosts = (h0, h1, group)`` runs the multi-GPU layout of the method on
-    this rank: Phase 1 of hosts [h0, h1) of the sequence, then the Phase-2
-    exchange (the rank's shard partials, an NCCL all-gather over ``group``,
-    the exact merge)."""
+    ``hosts = (h0, h1, group, max_local)`` runs the multi-GPU layout of the
+    method on this rank: Phase 1 of hosts [h0, h1) of the sequence, then the
+    Phase-2 exchange (the rank's shard partials, an NCCL all-gather over
+    ``group`` with every rank padded to ``max_local`` shards, the exact
+    merge)."""
 
     def __init__(self, w, dev, seed_offset=0, hosts=None):
         from long_context_blockwise_max_b200 import pulsar as P
@@ -251,7 +254,7 @@ class Step:
         nret = n_local * w.block
         D.phase2_attend_distributed(self.query, self.k_ret[None, :nret], self.v_ret[None, :nret], n_local,
                                     w.n_blocks, w.L, w.rope_theta, group=self.hosts[2], partials_fn=partials,
-                                    merge_fn=merge)
+                                    merge_fn=merge, max_local=self.hosts[3])
 
     def launches(self):
         """Kernels of ours one step launches: selection 3 (presence, min df,
@@ -330,9 +333,10 @@ def run_ours(args, rank, world, local_rank, dist_on):
     if hosts_layout:
         # one sequence, its hosts spread over the ranks (Phase 1 without
         # communication, then the Phase-2 all-gather over NCCL)
-        from long_context_blockwise_max_b200.distributed import shard_ranges
-        h0, h1 = shard_ranges(w.n_blocks, world)[rank]
-        step = Step(w, dev, hosts=(h0, h1, torch.distributed.group.WORLD))
+        from long_context_blockwise_max_b200.distributed import phase1_host_ranges
+        ranges = phase1_host_ranges(w.L, w.block, w.sink, w.chunk, w.k_chunks, False, world)
+        h0, h1 = ranges[rank]
+        step = Step(w, dev, hosts=(h0, h1, torch.distributed.group.WORLD, max(b - a for a, b in ranges)))
     else:
         h0, h1 = 0, w.n_blocks
         step = Step(w, dev, seed_offset=rank)
@@ -929,9 +933,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--headline-only", action="store_true", help="skip the side measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--layout", default="sequences", choices=["sequences", "hosts"],
-                    help="sequences: one independent sequence per rank (weak scaling); hosts: the hosts of one "
-                         "sequence spread over the ranks, with the Phase-2 all-gather over NCCL (strong scaling)")
+    ap.add_argument("--layout", default=None, choices=["sequences", "hosts"],
+                    help="hosts (the default with several GPUs): the hosts of one sequence spread over the ranks, "
+                         "then the Phase-2 all-gather over NCCL (strong scaling); sequences (the default on one "
+                         "GPU, where both are the same work): one independent sequence per rank (weak scaling)")
     ap.add_argument("--profile-case", default=None,
                     help="run one kernel family on a small workload (phase1-32k, decode-16k, decode-128k, query-128k, select-1m)")
     args = ap.parse_args()
@@ -942,6 +947,8 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.layout is None:
+        args.layout = "hosts" if world > 1 else "sequences"
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)

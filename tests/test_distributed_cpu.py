@@ -83,6 +83,25 @@ def test_exchange_uneven_shards_pads_empty():
     _run(3)      # rank 0 holds 2 shards, rank 1 holds 1 and pads one empty shard
 
 
+def test_balanced_host_ranges_are_optimal():
+    # every contiguous split of the hosts into `world` ranges, by brute force:
+    # none has a smaller largest range work (sum of n (n + 1) / 2)
+    import itertools
+    from long_context_blockwise_max_b200.distributed import balanced_host_ranges, host_rows
+    cost = lambda rows, rg: max(sum(x * (x + 1) // 2 for x in rows[a:b]) for a, b in rg)
+    for rows in (host_rows(8, 16384, 64, 2048, False), host_rows(8, 16384, 0, 0, True),
+                 host_rows(7, 256, 16, 32, False), [5, 100, 3, 3, 90, 1]):
+        n = len(rows)
+        for world in range(1, n + 1):
+            got = balanced_host_ranges(rows, world)
+            assert len(got) == world and got[0][0] == 0 and got[-1][1] == n
+            assert all(a[1] == b[0] and a[0] < a[1] for a, b in zip(got, got[1:]))
+            best = min(cost(rows, [(0, c[0])] + list(zip(c, c[1:])) + [(c[-1], n)] if c else [(0, n)])
+                       for c in itertools.combinations(range(1, n), world - 1))
+            assert cost(rows, got) == best, (rows, world)
+    assert balanced_host_ranges([10, 20], 4) == [(0, 1), (1, 2), (2, 2), (2, 2)]
+
+
 def test_shard_ranges():
     from long_context_blockwise_max_b200.distributed import shard_ranges
     assert shard_ranges(8, 4) == [(0, 2), (2, 4), (4, 6), (6, 8)]
@@ -126,8 +145,10 @@ def _pipeline_worker(rank, world, port, star, out):
         q, k, v, sel, qq = _pipeline_inputs()
         o, lse, kr, vr, (h0, h1) = D.phase1_encode_distributed(q, k, v, TH1, BLK1, SINK1, CH1, K1, sel, star,
                                                                encode_fn=_oracle_encode_hosts)
+        ranges = D.phase1_host_ranges(L1, BLK1, SINK1, CH1, K1, star, world)
         og, lg = D.phase2_attend_distributed(qq, kr[None], vr[None], h1 - h0, L1 // BLK1, L1, TH1,
-                                             partials_fn=_oracle_partials, merge_fn=_oracle_merge)
+                                             partials_fn=_oracle_partials, merge_fn=_oracle_merge,
+                                             max_local=max(b - a for a, b in ranges))
         out[rank] = (h0, h1, o.numpy(), lse.numpy(), og.numpy(), lg.numpy())
     finally:
         dist.destroy_process_group()
@@ -143,8 +164,11 @@ def _pipeline(world, star):
     q, k, v, sel, qq = _pipeline_inputs()
     n = L1 // BLK1
     # the ranks' host ranges tile [0, n) in order
-    assert [(r[0], r[1]) for r in res] == __import__(
-        "long_context_blockwise_max_b200.distributed", fromlist=["x"]).shard_ranges(n, world)
+    from long_context_blockwise_max_b200 import distributed as D
+    ranges = D.phase1_host_ranges(L1, BLK1, SINK1, CH1, K1, star, world)
+    assert [(r[0], r[1]) for r in res] == ranges
+    assert ranges[0][0] == 0 and ranges[-1][1] == n
+    assert all(a[1] == b[0] for a, b in zip(ranges, ranges[1:]))
     # Phase 1: the ranks' rows, in rank order, are the one-process encoding
     pos = oracle.host_positions(L1, BLK1, SINK1, CH1, sel.numpy(), star=star)
     full = oracle.phase1_encode(q.numpy(), k.numpy(), v.numpy(), pos, TH1)
