@@ -116,3 +116,49 @@ def test_mean_idf_hand_worked_tie(P):
         sel, rank, _ = P.pulsar_select_summaries_scored(ids, 5, 16, 4, 1, P.PA_SCORE_MEAN_IDF, want_scores=True)
         assert sel[0].tolist() == [1]
         assert rank[:4].tolist() == [2, 0, 1, 3]
+
+
+def test_scorers_at_the_1m_scale_shape(P):
+    # 1M Zipf ids, 32 blocks of 32768, 1024 chunks per block, 128 kept: mean
+    # IDF and entropy bit-exact (selection and ranks), BM25 by order
+    w = workloads.SCALE_1M
+    ids = w.token_ids()
+    dev_ids = torch.from_numpy(ids).to(DEV)
+    for method, ref in ((P.PA_SCORE_MEAN_IDF,
+                         lambda: oracle.select_summaries_mean_idf(ids, w.block, w.chunk, w.k_chunks, w.vocab,
+                                                                  return_rank=True)),
+                        (P.PA_SCORE_ENTROPY,
+                         lambda: oracle.select_summaries_entropy(ids, w.block, w.chunk, w.k_chunks,
+                                                                 return_rank=True))):
+        sel, rank, ws = P.pulsar_select_summaries_scored(dev_ids, w.vocab, w.block, w.chunk, w.k_chunks, method,
+                                                        want_scores=True)
+        assert P.pa_workspace_status(ws) == 0
+        want_sel, want_rank = ref()
+        assert np.array_equal(sel.cpu().numpy(), want_sel), method
+        assert np.array_equal(rank.cpu().numpy(), want_rank), method
+    _check_bm25(P, dev_ids, ids, w.vocab, w.block, w.chunk, w.k_chunks)
+
+
+@pytest.mark.parametrize("case", [
+    # (L, vocab, block, chunk, k, what)
+    (512, 40, 512, 32, 3, "one block: every df is 1, all means equal"),
+    (2048, 40, 512, 32, 0, "k = 0"),
+    (2048, 40, 512, 32, 16, "k = C: every chunk kept"),
+    (1024, 30, 256, 1, 5, "one-token chunks"),
+    (2048, 1, 512, 32, 4, "a one-id vocabulary: every score equal"),
+    (64 * 64, 50, 64, 32, 1, "64 blocks, two chunks each"),
+])
+def test_scorer_edge_cases(P, case):
+    L, vocab, block, chunk, k, _ = case
+    ids = workloads.zipf_token_ids(L, vocab, 1.0, seed=L + vocab)
+    dev_ids = torch.from_numpy(ids).to(DEV)
+    for method in (P.PA_SCORE_MEAN_IDF, P.PA_SCORE_ENTROPY):
+        sel, rank, ws = P.pulsar_select_summaries_scored(dev_ids, vocab, block, chunk, k, method, want_scores=True)
+        assert P.pa_workspace_status(ws) == 0
+        if method == P.PA_SCORE_MEAN_IDF:
+            want_sel, want_rank = oracle.select_summaries_mean_idf(ids, block, chunk, k, vocab, return_rank=True)
+        else:
+            want_sel, want_rank = oracle.select_summaries_entropy(ids, block, chunk, k, return_rank=True)
+        assert np.array_equal(sel.cpu().numpy().reshape(want_sel.shape), want_sel), (case, method)
+        assert np.array_equal(rank.cpu().numpy(), want_rank), (case, method)
+    _check_bm25(P, dev_ids, ids, vocab, block, chunk, k)
