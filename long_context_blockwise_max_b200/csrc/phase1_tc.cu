@@ -252,15 +252,16 @@ __global__ void __launch_bounds__(384, 1) phase1_tc_kernel(const __grid_constant
           mma_commit(&bars->s_full[1]);
           mma_commit(&bars->k_empty[0]);
         }
-        // head 0: O0 += P0 V_j, then S0 = Q0 K_{j+1}
-        if (!mbar_wait(&bars->p_full[0], j & 1, abort, p.wait_ns, gabort)) { fail(5); break; }
+        // head 0: O0 += P0 V_j, then S0 = Q0 K_{j+1}.  V_j and K_{j+1} are
+        // waited for first, while the tensor pipe still runs head 1's MMAs,
+        // so that nothing stands between P0 and the MMAs that consume it.
         if (!mbar_wait(&bars->v_full[st], ph, abort, p.wait_ns, gabort)) { fail(6); break; }
+        if (j + 1 < nkv && !mbar_wait(&bars->k_full[st1], ph1, abort, p.wait_ns, gabort)) { fail(7); break; }
+        if (!mbar_wait(&bars->p_full[0], j & 1, abort, p.wait_ns, gabort)) { fail(5); break; }
         tc_fence_after();
         pv(0, st, j > 0);
         if (j == nkv - 1) mma_commit(&bars->o_final[0]);
         if (j + 1 < nkv) {
-          if (!mbar_wait(&bars->k_full[st1], ph1, abort, p.wait_ns, gabort)) { fail(7); break; }
-          tc_fence_after();
           qk(0, st1);
           mma_commit(&bars->s_full[0]);
         }
