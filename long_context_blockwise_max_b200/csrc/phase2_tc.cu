@@ -90,13 +90,16 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 // Two bf16 (one 32-bit word) -> two fp16.  bf16 -> fp32 is exact (the bf16
 // bits are the top half of the fp32 word); fp32 -> fp16 rounds to nearest,
-// which is exact for bf16 values in fp16's normal range.  `bad` collects
-// results that are not finite.
-__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w, bool& bad) {
+// which is exact for bf16 values in fp16's normal range.  `flags` collects
+// results that are not finite: each half's exponent field plus 0x0400
+// carries into that half's top bit only when the field is all ones (inf or
+// NaN), and a half's sum stays below 0x10000, so the halves never carry into
+// each other; flags & 0x80008000 is non-zero iff some result was not finite.
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w, uint32_t& flags) {
   const float lo = __uint_as_float(w << 16), hi = __uint_as_float(w & 0xFFFF0000u);
   const __half2 h = __floats2half2_rn(lo, hi);
   const uint32_t r = *reinterpret_cast<const uint32_t*>(&h);
-  bad |= ((r & 0x7C00u) == 0x7C00u) || ((r & 0x7C000000u) == 0x7C000000u);
+  flags |= (r & 0x7C007C00u) + 0x04000400u;
   return r;
 }
 
@@ -283,7 +286,7 @@ __global__ void __launch_bounds__(384, 1) phase2_tc_kernel(const __grid_constant
   } else if (warp < 4) {
     // ------------------------------------------------------- K converters
     const int ct = threadIdx.x - 64;   // 0 .. 63
-    bool bad = false;
+    uint32_t flags = 0;
     for (int j = 0; j < nkv; ++j) {
       const int sk = j % KST;
       if (!mbar_wait(&bars->k_full[sk], (j / KST) & 1, abort, wait_ns, gabort)) { fail(12); break; }
@@ -292,10 +295,10 @@ __global__ void __launch_bounds__(384, 1) phase2_tc_kernel(const __grid_constant
 #pragma unroll 4
       for (int c = ct; c < N16; c += kConvThreads) {
         uint4 v = tile[c];
-        v.x = bf16x2_to_f16x2(v.x, bad);
-        v.y = bf16x2_to_f16x2(v.y, bad);
-        v.z = bf16x2_to_f16x2(v.z, bad);
-        v.w = bf16x2_to_f16x2(v.w, bad);
+        v.x = bf16x2_to_f16x2(v.x, flags);
+        v.y = bf16x2_to_f16x2(v.y, flags);
+        v.z = bf16x2_to_f16x2(v.z, flags);
+        v.w = bf16x2_to_f16x2(v.w, flags);
         tile[c] = v;
       }
       // generic-proxy stores -> visible to the tensor core's async proxy
@@ -304,7 +307,7 @@ __global__ void __launch_bounds__(384, 1) phase2_tc_kernel(const __grid_constant
     }
     // a key of this unit outside fp16 range: the unit is recomputed exactly
     // (mma.sync row kernel, high / low bf16 query) after this kernel
-    if (bad) atomicExch(a.redo + (static_cast<int64_t>(b) * p.units + u) * a.hkv + kvh, 1);
+    if (flags & 0x80008000u) atomicExch(a.redo + (static_cast<int64_t>(b) * p.units + u) * a.hkv + kvh, 1);
   } else {
     // -------------------------------------------------------------- softmax
     const int t = warp >= 8 ? 1 : 0;
