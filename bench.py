@@ -106,23 +106,40 @@ def recorded_traffic(kernel: str, workload: str):
 # clocks during the timed region
 # --------------------------------------------------------------------------
 class ClockSampler:
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi sampling every 50 ms, started well before the timed region
+    (the tool takes a few hundred ms to produce its first line) and summarised
+    over the samples whose timestamps fall inside the window marked with
+    mark_start() / mark_end()."""
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, index: int):
         self.index = index
         self.proc = None
+        self.t_start = self.t_end = None
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+        import atexit
+        atexit.register(self._stop)   # no sampler outlives the run, even after an error
         return self
+
+    def _stop(self):
+        if self.proc is not None and self.proc.poll() is None:
+            self.proc.kill()
+
+    def mark_start(self):
+        self.t_start = time.time()
+
+    def mark_end(self):
+        self.t_end = time.time()
 
     def __exit__(self, *exc):
         self.out = ""
@@ -135,25 +152,37 @@ class ClockSampler:
                 self.out, _ = self.proc.communicate()
         return False
 
+    @staticmethod
+    def _epoch(stamp: str):
+        import datetime
+        try:
+            return datetime.datetime.strptime(stamp, "%Y/%m/%d %H:%M:%S.%f").timestamp()
+        except ValueError:
+            return None
+
     def summary(self):
-        sm, mx, reasons = [], 0.0, set()
+        """Median SM clock, maximum clock and the throttle reasons seen over
+        the samples inside the marked window (all samples if the window holds
+        none, with "in_window": false)."""
+        rows = []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in (self.out or "").strip().splitlines():
             f = [x.strip() for x in line.split(",")]
-            if len(f) < 8:
+            if len(f) < 9:
                 continue
             try:
-                sm.append(float(f[0]))
-                mx = max(mx, float(f[1]))
+                rows.append((self._epoch(f[0]), float(f[1]), float(f[2]),
+                             {n for n, val in zip(names, f[5:9]) if val.lower().startswith("active")}))
             except ValueError:
                 continue
-            for n, val in zip(names, f[4:8]):
-                if val.lower().startswith("active"):
-                    reasons.add(n)
-        if not sm:
+        inside = [r for r in rows if r[0] is not None and self.t_start is not None and self.t_end is not None
+                  and self.t_start <= r[0] <= self.t_end]
+        use = inside or rows
+        if not use:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        return {"sm_mhz": statistics.median(r[1] for r in use), "sm_max_mhz": max(r[2] for r in use),
+                "reasons": sorted(set().union(*(r[3] for r in use))), "samples": len(use),
+                "in_window": bool(inside)}
 
 
 # --------------------------------------------------------------------------
@@ -327,6 +356,7 @@ def whole_job_rate(units_per_rank: float, world: int, ms_per_step: float) -> flo
 def run_ours(args, rank, world, local_rank, dist_on):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
+    clk = ClockSampler(local_rank).__enter__()   # running before the timed region starts
     w = WORKLOAD
     peaks, peak_kind = load_peaks()
     hosts_layout = args.layout == "hosts"
@@ -357,15 +387,17 @@ def run_ours(args, rank, world, local_rank, dist_on):
             e.record()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sync_all(dist_on)
-    with ClockSampler(local_rank) as clk:
-        t0.record()
-        for i in range(K):
-            step.attn_events = ev_attn[i]
-            step.p2_events = ev_p2[i]
-            step.stage_events = ev_stage[i]
-            step.run()
-        t1.record()
-        torch.cuda.synchronize()
+    clk.mark_start()
+    t0.record()
+    for i in range(K):
+        step.attn_events = ev_attn[i]
+        step.p2_events = ev_p2[i]
+        step.stage_events = ev_stage[i]
+        step.run()
+    t1.record()
+    torch.cuda.synchronize()
+    clk.mark_end()
+    clk.__exit__(None, None, None)
     step.attn_events = None
     step.p2_events = None
     step.stage_events = None

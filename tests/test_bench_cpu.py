@@ -75,14 +75,25 @@ def test_committed_traffic_records_parse():
 def test_clock_summary_reads_median_max_and_active_reasons():
     c = bench.ClockSampler(0)
     c.out = "\n".join([
-        "1965, 1965, 700.1, 0x0, Not Active, Not Active, Not Active, Not Active",
-        "1800, 1965, 995.0, 0x4, Not Active, Not Active, Not Active, Active",
-        "1700, 1965, 1001.2, 0x4, Not Active, Not Active, Not Active, Active",
-        "[N/A], 1965, 0, 0x0, Not Active, Not Active, Not Active, Not Active",   # unreadable sample
+        "2026/12/03 05:41:00.000, 1965, 1965, 700.1, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "2026/12/03 05:41:00.050, 1800, 1965, 995.0, 0x4, Not Active, Not Active, Not Active, Active",
+        "2026/12/03 05:41:00.100, 1700, 1965, 1001.2, 0x4, Not Active, Not Active, Not Active, Active",
+        "2026/12/03 05:41:00.150, [N/A], 1965, 0, 0x0, Not Active, Not Active, Not Active, Not Active",  # unreadable
         "garbage",
     ])
+    # no window marked: every readable sample, flagged as such
     s = c.summary()
-    assert s == {"sm_mhz": 1800.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
+    assert s == {"sm_mhz": 1800.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3,
+                 "in_window": False}
+    # a window holding the last two samples only (timestamps are host-local time)
+    t1 = bench.ClockSampler._epoch("2026/12/03 05:41:00.040")
+    t2 = bench.ClockSampler._epoch("2026/12/03 05:41:00.120")
+    c.t_start, c.t_end = t1, t2
+    assert c.summary() == {"sm_mhz": 1750.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 2,
+                           "in_window": True}
+    # a window with no sample in it falls back to all of them
+    c.t_start, c.t_end = t2 + 10, t2 + 11
+    assert c.summary()["samples"] == 3 and c.summary()["in_window"] is False
     c.out = ""
     assert c.summary()["samples"] == 0
 
