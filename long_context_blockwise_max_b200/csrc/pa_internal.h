@@ -64,6 +64,10 @@ struct HostTable {
   int64_t ci_blk;
 };
 
+// Rows at the start of every host that Phase 1 recomputes in fp32 when Q / K
+// are carried in fp16 (they see too few keys to average the rounding out).
+constexpr int kHeadRows = 32;
+
 struct Phase1Args {
   int dtype;                    // PA_F32 / PA_BF16
   const void *q, *k, *v;        // inputs [L][h][d]

@@ -25,6 +25,8 @@
 //  phase1_simt_kernel: causal attention over a host's rows, fp32 SIMT with an
 //                      online softmax (used for fp32 inputs, and for bf16
 //                      inputs when the tensor-core kernel is not selected).
+//  phase1_head_rows_kernel: the first kHeadRows rows of every host again, in
+//                      fp32 from the unrounded inputs (bf16 inputs only).
 #include "pa_internal.h"
 
 namespace pa {
@@ -298,6 +300,102 @@ __global__ void __launch_bounds__(256) phase1_simt_kernel(
   if (lse != nullptr && hf == 0) lse[(row0 + r) * hq + h] = (m_run + __log2f(l_run)) * kLn2f;
 }
 
+// ---------------------------------------------------------------------------
+// Head rows in fp32.  For bf16 inputs the attention kernels read rotated Q / K
+// rounded to fp16, so every logit carries up to 2^-11 relative rounding per
+// operand.  A row that sees many keys averages those errors in its lse, but
+// the first rows of a host see only a few keys (row r sees r + 1), and their
+// lse keeps one logit's error: on unit-normal inputs up to ~1.2e-3.  This
+// kernel recomputes the first kHeadRows rows of every host from the bf16
+// inputs, rotating in fp32 (fp64 angles, as rope_qk_kernel) without the
+// fp16 rounding, and overwrites their O and lse.  CTA = one host x one kv
+// head: the keys of those rows are rotated once into shared memory; one warp
+// per (row, query head of the group), each lane owning D / 32 elements.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) phase1_head_rows_kernel(
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+    const int32_t* __restrict__ rowpos, HostTable ht, int hq, int hkv, RopeFreqs f, __nv_bfloat16* __restrict__ o,
+    float* __restrict__ lse) {
+  constexpr int HALF = D / 2, PER = D / 64;   // per lane: PER elements of each half
+  __shared__ float ks[kHeadRows][D];
+  __shared__ float vs[kHeadRows][D];
+  const int host = blockIdx.x, kvh = blockIdx.y;
+  const int64_t row0 = ht.row_off[host];
+  const int64_t n_host = ht.row_off[host + 1] - row0;
+  const int R = n_host < kHeadRows ? (int)n_host : kHeadRows;
+  for (int e = threadIdx.x; e < R * HALF; e += blockDim.x) {
+    const int j = e / HALF, m = e % HALF;
+    const int64_t pos = rowpos[row0 + j];
+    double sn, cn;
+    sincos((double)pos * f.omega[m], &sn, &cn);
+    const float c = (float)cn, sg = (float)sn;
+    const __nv_bfloat16* kr = k + (pos * hkv + kvh) * (int64_t)D;
+    const __nv_bfloat16* vr = v + (pos * hkv + kvh) * (int64_t)D;
+    const float x1 = __bfloat162float(kr[m]), x2 = __bfloat162float(kr[m + HALF]);
+    ks[j][m] = x1 * c - x2 * sg;
+    ks[j][m + HALF] = x2 * c + x1 * sg;
+    vs[j][m] = __bfloat162float(vr[m]);
+    vs[j][m + HALF] = __bfloat162float(vr[m + HALF]);
+  }
+  __syncthreads();
+  const int g = hq / hkv;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const float scale = (float)(1.0 / sqrt((double)D));
+  for (int w = warp; w < R * g; w += blockDim.x / 32) {
+    const int r = w / g, h = kvh * g + w % g;
+    const int64_t pos = rowpos[row0 + r];
+    const __nv_bfloat16* qr = q + (pos * hq + h) * (int64_t)D;
+    float qa[PER], qb[PER];   // elements lane + 32 i and lane + 32 i + D / 2
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int m = lane + 32 * i;
+      double sn, cn;
+      sincos((double)pos * f.omega[m], &sn, &cn);
+      const float c = (float)cn, sg = (float)sn;
+      const float x1 = __bfloat162float(qr[m]), x2 = __bfloat162float(qr[m + HALF]);
+      qa[i] = x1 * c - x2 * sg;
+      qb[i] = x2 * c + x1 * sg;
+    }
+    float sc[kHeadRows];
+    float mx = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < kHeadRows; ++j) {
+      float a = 0.f;
+      if (j <= r) {
+#pragma unroll
+        for (int i = 0; i < PER; ++i) a = fmaf(qa[i], ks[j][lane + 32 * i], fmaf(qb[i], ks[j][lane + 32 * i + HALF], a));
+#pragma unroll
+        for (int sh = 16; sh > 0; sh >>= 1) a += __shfl_xor_sync(0xffffffffu, a, sh);
+      }
+      sc[j] = j <= r ? a * scale : -INFINITY;
+      mx = fmaxf(mx, sc[j]);
+    }
+    float l = 0.f, oa[PER], ob[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) oa[i] = ob[i] = 0.f;
+#pragma unroll
+    for (int j = 0; j < kHeadRows; ++j) {
+      if (j > r) break;
+      const float pj = expf(sc[j] - mx);
+      l += pj;
+#pragma unroll
+      for (int i = 0; i < PER; ++i) {
+        oa[i] = fmaf(pj, vs[j][lane + 32 * i], oa[i]);
+        ob[i] = fmaf(pj, vs[j][lane + 32 * i + HALF], ob[i]);
+      }
+    }
+    const float inv = 1.f / l;
+    __nv_bfloat16* dst = o + ((row0 + r) * hq + h) * (int64_t)D;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      dst[lane + 32 * i] = __float2bfloat16(oa[i] * inv);
+      dst[lane + 32 * i + HALF] = __float2bfloat16(ob[i] * inv);
+    }
+    if (lse != nullptr && lane == 0) lse[(row0 + r) * hq + h] = mx + logf(l);
+  }
+}
+
 size_t phase1_workspace_bytes(int64_t qk_rows, int32_t hq, int32_t hkv, int32_t d, int dtype,
                               int64_t rows, int64_t posmap_rows) {
   const size_t qk_elem = dtype == PA_BF16 ? 2 : 4;
@@ -357,6 +455,20 @@ static int launch_phase1_t(const Phase1Args& a, cudaStream_t s) {
       phase1_simt_kernel<64, QT, VT, OT><<<grid, 256, 0, s>>>(
           static_cast<const QT*>(a.qr), kq, static_cast<const VT*>(a.v), a.rowpos, a.rowci, a.ht,
           a.hq, a.hkv, static_cast<OT*>(a.o), a.lse);
+  }
+  // fp16-carried Q / K: the first rows of every host again in fp32
+  if (rc == PA_OK && sizeof(QT) == 2 && a.ht.n_hosts > 0) {
+    const dim3 hg(a.ht.n_hosts, a.hkv);
+    if (a.d == 128)
+      phase1_head_rows_kernel<128><<<hg, 256, 0, s>>>(
+          static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),
+          static_cast<const __nv_bfloat16*>(a.v), a.rowpos, a.ht, a.hq, a.hkv, f, static_cast<__nv_bfloat16*>(a.o),
+          a.lse);
+    else
+      phase1_head_rows_kernel<64><<<hg, 256, 0, s>>>(
+          static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),
+          static_cast<const __nv_bfloat16*>(a.v), a.rowpos, a.ht, a.hq, a.hkv, f, static_cast<__nv_bfloat16*>(a.o),
+          a.lse);
   }
   profile_end(s);
   if (rc != PA_OK) return rc;

@@ -38,7 +38,9 @@ def _phase1_case(seed):
                 theta=float(rng.choice([1e4, 5e5])))
 
 
-@pytest.mark.parametrize("seed", range(12))
+# 599 and 923: bf16 cases whose short causal rows (one or six visible keys)
+# exceeded the lse tolerance while every row's Q / K were carried in fp16
+@pytest.mark.parametrize("seed", list(range(12)) + [599, 923])
 def test_phase1_random_shape(P, seed):
     c = _phase1_case(seed)
     L = c["n"] * c["block"]
