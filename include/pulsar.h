@@ -248,7 +248,9 @@ size_t pa_phase1_hosts_workspace_size(int64_t L, int32_t hq, int32_t hkv, int32_
  *
  * d must be 64 or 128, hq % hkv == 0.  For PA_BF16, rotated Q and K are
  * carried in fp16 for the QK^T product; P is rounded to bf16 for the PV
- * product; all sums are fp32.  For PA_F32 the whole path is fp32.
+ * product; all sums are fp32.  The first 32 rows of every host (too few
+ * visible keys to average the fp16 rounding out of their lse) are computed
+ * again in fp32 from the bf16 inputs.  For PA_F32 the whole path is fp32.
  * Limit (bf16): a rotated Q value times log2(e)/sqrt(d), or a rotated K
  * value, beyond 65504 is refused through the device status PA_ERR_RANGE
  * (pa_workspace_status); the outputs are then unspecified.
