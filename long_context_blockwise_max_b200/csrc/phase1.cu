@@ -320,16 +320,23 @@ __global__ void __launch_bounds__(256) phase1_head_rows_kernel(
   constexpr int HALF = D / 2, PER = D / 64;   // per lane: PER elements of each half
   __shared__ float ks[kHeadRows][D];
   __shared__ float vs[kHeadRows][D];
+  __shared__ float2 cs[kHeadRows][HALF];      // (cos, sin) of row j's position, frequency m
   const int host = blockIdx.x, kvh = blockIdx.y;
   const int64_t row0 = ht.row_off[host];
   const int64_t n_host = ht.row_off[host + 1] - row0;
   const int R = n_host < kHeadRows ? (int)n_host : kHeadRows;
+  // query row r and key row r share a position: the angles once per row
+  for (int e = threadIdx.x; e < R * HALF; e += blockDim.x) {
+    const int j = e / HALF, m = e % HALF;
+    double sn, cn;
+    sincos((double)rowpos[row0 + j] * f.omega[m], &sn, &cn);
+    cs[j][m] = make_float2((float)cn, (float)sn);
+  }
+  __syncthreads();
   for (int e = threadIdx.x; e < R * HALF; e += blockDim.x) {
     const int j = e / HALF, m = e % HALF;
     const int64_t pos = rowpos[row0 + j];
-    double sn, cn;
-    sincos((double)pos * f.omega[m], &sn, &cn);
-    const float c = (float)cn, sg = (float)sn;
+    const float c = cs[j][m].x, sg = cs[j][m].y;
     const __nv_bfloat16* kr = k + (pos * hkv + kvh) * (int64_t)D;
     const __nv_bfloat16* vr = v + (pos * hkv + kvh) * (int64_t)D;
     const float x1 = __bfloat162float(kr[m]), x2 = __bfloat162float(kr[m + HALF]);
@@ -350,9 +357,7 @@ __global__ void __launch_bounds__(256) phase1_head_rows_kernel(
 #pragma unroll
     for (int i = 0; i < PER; ++i) {
       const int m = lane + 32 * i;
-      double sn, cn;
-      sincos((double)pos * f.omega[m], &sn, &cn);
-      const float c = (float)cn, sg = (float)sn;
+      const float c = cs[r][m].x, sg = cs[r][m].y;
       const float x1 = __bfloat162float(qr[m]), x2 = __bfloat162float(qr[m + HALF]);
       qa[i] = x1 * c - x2 * sg;
       qb[i] = x2 * c + x1 * sg;
