@@ -286,11 +286,13 @@ class Step:
                                     merge_fn=merge, max_local=self.hosts[3])
 
     def launches(self):
-        """Kernels of ours one step launches: selection 3 (presence, min df,
-        top-k); Phase 1 3 (row map, RoPE, attention) plus the position map
-        of a compact host range; Phase 2 3 (query RoPE, partials, merge)
-        plus the exchange's merge of the gathered partials."""
-        n = 9
+        """Kernels of ours one step launches (bf16, as in the ncu launch list
+        of the step): selection 3 (presence, min df, top-k); Phase 1 4 (row
+        map, RoPE, attention, the fp32 pass over each host's first rows) plus
+        the position map of a compact host range; Phase 2 4 (query RoPE,
+        tensor-core partials, the exact pass over units with keys beyond fp16
+        range, merge) plus the exchange's merge of the gathered partials."""
+        n = 11
         if self.hosts:
             w, h0, h1 = self.w, self.h0, self.h1
             pre = w.sink + (h1 - 1) * w.k_chunks * w.chunk
